@@ -1,0 +1,388 @@
+"""Benchmark of the quantized MoE FFN layer forward on B200.
+
+Default workload: the Mixtral-like layer (H=4096, F=14336, E=8, top-2; gate
+3-bit, up 2-bit, down 4-bit, group 32 with fp16 scales) run as prefill of
+T=2048 tokens.  One step = one full layer forward (router, top-k, permute,
+gather, gate/up GEMM + SwiGLU, down GEMM, combine) over one batch.  Decode
+batches T=1/8/64 of the same layer are reported under "runs".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the CPU oracle (the plain C reference) on the host
+cores on a bounded sample of the same workload.  Multi-GPU (torchrun) runs
+independent replicas: each rank runs its own batch, no data-path collective.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gen.workloads as W  # noqa: E402
+
+METRIC = "MoE-layer tokens/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+CSRC = os.path.join(ROOT, "mixed_precision_quantized_fp32_b200", "csrc")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+KERNELS_PER_FORWARD_INT = 9     # router, top-k, 3 permute, gather, gate/up, down, combine
+KERNELS_PER_FORWARD_FP4 = 11    # + x quant, h quant
+
+
+def workload_desc(L: W.Layer, T: int, mode: str) -> str:
+    f = L.fmt[0]
+    return (f"{L.name} layer {mode} T={T} (H={L.H}, F={L.F}, E={L.E}, top-{L.k}, "
+            f"gate/up/down {int(f[0])}/{int(f[1])}/{int(f[2])}-bit group-32 fp16 scales)")
+
+
+def peaks():
+    if os.path.exists(PEAKS_FILE):
+        d = json.load(open(PEAKS_FILE))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def csrc_hash() -> str:
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(CSRC)):
+        if fn.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(CSRC, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key: str):
+    """Per-launch DRAM bytes of a kernel from a committed ncu summary, or None if the
+    summary is missing or was taken on different kernel sources."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    d = json.load(open(TRAFFIC_FILE))
+    if d.get("csrc_hash") != csrc_hash():
+        return None
+    v = d.get("kernels", {}).get(kernel_key)
+    return None if v is None else v.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        import torch
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            self.sel = str(device_index)
+
+    def start(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.sel, f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+def expert_gateup_bytes(L: W.Layer, moe) -> np.ndarray:
+    """Packed bytes (codes + scales) of the gate and up matrices of each expert."""
+    out = np.zeros(L.E)
+    for e in range(L.E):
+        for p in (0, 1):
+            f = int(L.fmt[e, p])
+            n = L.F * L.H
+            out[e] += n * (4 if f == 16 else f) / 8 + (n / 16)
+    return out
+
+
+def gpu_pack(L: W.Layer, moe, dev):
+    """Quantize and pack the layer on the GPU through the C ABI, a few experts at a time."""
+    import torch
+    fmt = np.ascontiguousarray(L.fmt.reshape(-1))
+    packed = moe.alloc_packed(moe.pack_layout(L.E, L.H, L.F, fmt)[0], dev)
+    per = max(1, min(L.E, (1 << 31) // (3 * L.H * L.F * 4)))
+    stage = torch.empty((per, 3, L.H * L.F), dtype=torch.float32, device=dev)
+    for e0 in range(0, L.E, per):
+        ne = min(per, L.E - e0)
+        moe.moe_pack(W.device_expert_weights(L, e0, ne, out=stage[:ne]), e0, L.E, L.H, L.F, fmt, packed)
+    torch.cuda.synchronize()
+    return moe.PackedLayer(L.E, L.H, L.F, fmt, packed)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    import mixed_precision_quantized_fp32_b200 as moe
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    L = W.layer("mixtral")
+    T = 2048
+    layer = gpu_pack(L, moe, dev)
+    x = torch.empty((T, L.H), dtype=torch.bfloat16, device=dev)
+    W.fill_device_bf16(x, rank, W.TID_X, 1.0)   # each replica its own tokens
+    Wr, b = W.device_router(L)
+    ws = moe.alloc_packed(moe.workspace_bytes(layer, T, L.k), dev)
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    nev = moe.MOE_STAGE_EVENTS
+
+    def forward(ev=None, xx=x, yy=y):
+        return moe.moe_layer_forward(xx, Wr, b, layer, L.k, y=yy, ws=ws, stage_events=ev)
+
+    # ---- device-resident timing
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    for row in evs:
+        for e in row:
+            e.record()
+    for _ in range(args.warmup):
+        forward()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.6)  # let the sampler take its first reading before the timed region
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        forward(evs[s])
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    step_ms = [evs[s][0].elapsed_time(evs[s][-1]) for s in range(args.steps)]
+    stage_ms = np.array([[evs[s][i].elapsed_time(evs[s][i + 1]) for i in range(nev - 1)]
+                         for s in range(args.steps)])
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * T * args.steps / (total_ms / 1e3)
+
+    # ---- end to end through the public API with host buffers (pinned)
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty_like(x_host).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(args.warmup):
+        x_dev.copy_(x_host, non_blocking=True)
+        forward(xx=x_dev)
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        forward(xx=x_dev)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * T * args.steps / (e2e_ms / 1e3)
+
+    # ---- roofline of the dominant kernel (gate/up GEMM with the SwiGLU epilogue)
+    pk, pk_kind = peaks()
+    gateup_ms = float(stage_ms[:, 3].mean())
+    down_ms = float(stage_ms[:, 5].mean())
+    flops_gateup = 2.0 * T * L.k * 2 * L.H * L.F
+    achieved = flops_gateup / (gateup_ms / 1e3) / 1e12
+    traffic = ncu_traffic("gateup_prefill_mixtral")
+    roofline = {"bound": "tensor", "kernel": "expert GEMM gate/up + SwiGLU (fp16 operands)",
+                "achieved": round(achieved, 2), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": traffic,
+                "peak_source": f"{pk_kind} dense bf16 (= fp16) burst, MEASURED_PEAKS.json"
+                if pk_kind == "measured" else "fallback 1.59 PFLOP/s",
+                "algorithmic_flops_per_launch": flops_gateup, "avg_launch_ms": round(gateup_ms, 4)}
+    stages = dict(zip(["router_topk", "permute", "gather", "gateup", "h_quant", "down", "combine"],
+                      [round(float(v), 4) for v in stage_ms.mean(0)]))
+
+    # ---- decode batches of the same layer (HBM-bound; L2 flushed between steps)
+    runs = []
+    if not args.no_decode:
+        flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        eb = expert_gateup_bytes(L, moe)
+        for Td in (1, 8, 64):
+            xd = torch.empty((Td, L.H), dtype=torch.bfloat16, device=dev)
+            W.fill_device_bf16(xd, rank, W.TID_X, 1.0)
+            wsd = moe.alloc_packed(moe.workspace_bytes(layer, Td, L.k), dev)
+            cnt = torch.zeros(L.E, dtype=torch.int32, device=dev)
+            moe.moe_layer_forward(xd, Wr, b, layer, L.k, ws=wsd, debug={"counts": cnt})
+            torch.cuda.synchronize()
+            active = cnt.cpu().numpy() > 0
+            nd = max(args.steps, 10)
+            evd = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(nd)]
+            for row in evd:
+                for e in row:
+                    e.record()
+            for _ in range(3):
+                moe.moe_layer_forward(xd, Wr, b, layer, L.k, ws=wsd)
+            for s in range(nd):
+                flush.zero_()
+                moe.moe_layer_forward(xd, Wr, b, layer, L.k, ws=wsd, stage_events=evd[s])
+            torch.cuda.synchronize()
+            st = np.array([[evd[s][i].elapsed_time(evd[s][i + 1]) for i in range(nev - 1)] for s in range(nd)])
+            stp = np.array([evd[s][0].elapsed_time(evd[s][-1]) for s in range(nd)])
+            gu = float(st[:, 3].mean())
+            by = float(eb[active].sum())
+            runs.append({"workload": workload_desc(L, Td, "decode"), "tokens_per_s": round(Td / (stp.mean() / 1e3), 1),
+                         "ms_per_step": round(float(stp.mean()), 4),
+                         "active_experts": int(active.sum()),
+                         "gateup": {"bound": "hbm", "achieved": round(by / (gu / 1e3) / 1e9, 1),
+                                    "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                    "frac": round(by / (gu / 1e3) / 1e9 / pk["hbm_gbs"], 4),
+                                    "algorithmic_bytes_per_launch": by, "avg_launch_ms": round(gu, 4)},
+                         "stages_ms": dict(zip(stages.keys(), [round(float(v), 4) for v in st.mean(0)]))})
+        del flush
+
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
+        "data": "synthetic (seeded counter-based generator; random-init weights)",
+        "config": {"workload": workload_desc(L, T, "prefill"), "global_batch": T * world,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (617 MB packed weights streamed per step)"},
+        "roofline": roofline,
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2)},
+        "gpu_launches": KERNELS_PER_FORWARD_INT * args.steps,
+        "clocks": clk, "stages_ms": stages, "runs": runs,
+    }
+    return out, layer
+
+
+# ------------------------------------------------------------------ oracle (CPU) timing
+def oracle_time(L: W.Layer, T_full: int, budget_s: float, x_seed: int = 0):
+    """Time the oracle forward on a growing sample of the batch until it takes
+    `budget_s` seconds; returns (tokens/s, sample description, threads)."""
+    import oracle as orc
+    Wr = W.router_w(L.E, L.H)
+    x_all = W.x_bf16_bits(T_full, L.H, seed=x_seed)
+    n = 2
+    buf = None
+    packed_experts = set()
+    while True:
+        xs = np.ascontiguousarray(x_all[:n])
+        idx = orc.topk_softmax(orc.router(xs, Wr, L.bias), L.k)[0]
+        need = set(np.unique(idx).tolist()) - packed_experts
+        for e in sorted(need):
+            buf = orc.pack_layer(W.expert_w(e, L.H, L.F)[None], e, L.E, L.H, L.F, L.fmt.reshape(-1), out=buf)
+        packed_experts |= need
+        t0 = time.perf_counter()
+        orc.moe_forward(buf, xs, Wr, L.bias, L.k)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or n >= T_full:
+            return n / dt, f"first {n} of {T_full} tokens (oracle packing excluded)", orc.num_threads()
+        n = min(T_full, n * 2 if dt < budget_s / 4 else int(n * budget_s / dt) + 1)
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    L = W.layer("mixtral")
+    T = 2048
+    per_step_budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, sample, cores = oracle_time(L, T, per_step_budget)
+        if i >= args.warmup:
+            vals.append(v)
+    value = float(np.mean(vals))
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * T / value, 1), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(L, T, "prefill"), "parallelism": "CPU oracle"},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode runs")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    out, _ = run_ours(args, rank, world, local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            v, sample, cores = oracle_time(W.layer("mixtral"), 2048, args.cpu_budget)
+            out["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                   "sample": sample}
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

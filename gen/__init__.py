@@ -96,6 +96,42 @@ def normal_bf16_bits(seed: int, tid: int, start: int, count: int, sigma: float =
     return f32_to_bf16_bits(normal_f32(seed, tid, start, count, sigma, idx))
 
 
+_host = None
+
+
+def _host_lib():
+    """ctypes handle of gen/libmoegen_host.so (built on first use)."""
+    global _host
+    if _host is None:
+        import ctypes as C
+        import os
+        import subprocess
+        here = os.path.dirname(os.path.abspath(__file__))
+        lib = os.path.join(here, "libmoegen_host.so")
+        src = os.path.join(here, "gen_host.c")
+        if not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(src):
+            subprocess.run(["gcc", "-std=c11", "-O2", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
+                            "-fvisibility=hidden", src, "-o", lib + ".tmp"], check=True)
+            os.replace(lib + ".tmp", lib)
+        L = C.CDLL(lib)
+        L.moegen_host_fill_f32.restype = None
+        L.moegen_host_fill_f32.argtypes = [C.c_void_p, C.c_uint64, C.c_uint64, C.c_uint64, C.c_uint64,
+                                           C.c_float]
+        _host = L
+    return _host
+
+
+def fill_f32(seed: int, tid: int, count: int, sigma: float = 1.0, start: int = 0,
+             out: np.ndarray | None = None) -> np.ndarray:
+    """Same values as normal_f32, filled by the multi-threaded C twin."""
+    import ctypes as C
+    if out is None:
+        out = np.empty(count, np.float32)
+    assert out.dtype == np.float32 and out.flags["C_CONTIGUOUS"] and out.size >= count
+    _host_lib().moegen_host_fill_f32(out.ctypes.data_as(C.c_void_p), seed, tid, start, count, sigma)
+    return out
+
+
 def expert_weights_f32(seed: int, e0: int, ne: int, H: int, F: int,
                        sigma: float = 0.02) -> np.ndarray:
     """fp32 expert weights [ne][3][N*K] in the order gate [F,H], up [F,H], down [H,F]
@@ -103,7 +139,7 @@ def expert_weights_f32(seed: int, e0: int, ne: int, H: int, F: int,
     out = np.empty((ne, 3, H * F), dtype=np.float32)
     for i in range(ne):
         for p in range(3):
-            out[i, p] = normal_f32(seed, tid_expert(e0 + i, p), 0, H * F, sigma)
+            fill_f32(seed, tid_expert(e0 + i, p), H * F, sigma, out=out[i, p])
     return out
 
 

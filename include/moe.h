@@ -1,0 +1,202 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) quantized Mixture-of-Experts FFN layer.
+ *
+ * Two calls:
+ *   moe_pack           quantizes fp32 expert weights into the packed layer buffer;
+ *   moe_layer_forward  runs the layer: fp32 router -> top-k with a softmax over
+ *                      the chosen k -> permutation of tokens by expert ->
+ *                      per-expert SwiGLU FFN on dequantized weights -> weighted
+ *                      combine.
+ *
+ * Where the method comes from (web pages; section numbers as printed there):
+ *  - "quantized MoE LLM inference" (cloud.baidu.com article 9434801), expert
+ *    routing section: logits = router(x); top-k indices; weights = softmax of
+ *    the chosen logits; output = weighted sum of the chosen experts.
+ *  - "MoE混合精度量化实战：门控保精度+专家激进压缩" (MoE mixed-precision
+ *    quantization in practice): sec. 2.1 keeps the gate/router unquantized and
+ *    quantizes expert-input activations per token with a live scale;
+ *    sec. 2.3 and 3.5 pack each expert in 128-column blocks, each block
+ *    quantized on its own, concatenated into one stream read by a custom
+ *    packed-linear kernel; sec. 3.3 gives the 4-bit code range [-8, 7].
+ *  - AlphaQ MoE quantization stack (mhpn.cn news 995352), sec. 2.2 and 4.2:
+ *    bit widths chosen per expert and per projection (gate 3-bit, middle 2-bit,
+ *    output 4-bit), group size 32.
+ *  - "Expert-aware quantisation: near-Q4 quality at near-Q2 size?": frequently
+ *    routed ("hot") experts at 4-bit, the rest ("cold") at 2-bit.
+ *
+ * Conventions for every call:
+ *  - Pointers are DEVICE pointers unless marked HOST.  The caller owns all
+ *    memory; the library allocates no device or pinned memory and keeps no
+ *    state between calls except a per-process cache of device properties.
+ *  - Calls are asynchronous on `stream`; nothing is synchronized inside.
+ *  - Errors are reported by the return code only.  Arguments are validated
+ *    before anything is launched, so a call that returns an error other than
+ *    MOE_ERR_CUDA has launched nothing.
+ *  - Device-side failures (a bounded wait that gave up, a range check) are
+ *    written as a moe_status value to moe_debug.status when that pointer is
+ *    given (the caller zeroes it and reads it after synchronizing).
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_ARG = 1,        /* null pointer, out-of-range count or index */
+  MOE_ERR_ALIGN = 2,      /* a pointer misses its required alignment */
+  MOE_ERR_SHAPE = 3,      /* H or F not a multiple of 128, E > 256, k > min(E, 8), ... */
+  MOE_ERR_WORKSPACE = 4,  /* workspace or output buffer too small */
+  MOE_ERR_FORMAT = 5,     /* unknown format code, NVFP4 mixed with integer formats,
+                             or a packed buffer whose header disagrees */
+  MOE_ERR_CUDA = 6,       /* a CUDA runtime call or launch failed */
+  MOE_ERR_TIMEOUT = 7,    /* device-side bounded wait gave up (status word only) */
+  MOE_ERR_UNSUPPORTED_DEVICE = 8 /* current device is not compute capability 10.x */
+} moe_status;
+
+/* Weight formats, chosen per expert and per projection. */
+enum {
+  MOE_FMT_INT2 = 2,   /* symmetric codes {-1,0,1}, fp16 scale per 32 inputs */
+  MOE_FMT_INT3 = 3,   /* symmetric codes [-3,3],   fp16 scale per 32 inputs */
+  MOE_FMT_INT4 = 4,   /* symmetric codes [-7,7],   fp16 scale per 32 inputs */
+  MOE_FMT_NVFP4 = 16  /* e2m1 codes, e4m3 scale per 16 inputs, fp32 scale per matrix */
+};
+
+/*
+ * Packed layer buffer (written by moe_pack; little-endian; read by the kernels).
+ *
+ * Header, 16384 bytes:
+ *   [0]     u32 magic 0x51454F4D        [4]  u32 version 1
+ *   [8]     i32 E   [12] i32 H   [16] i32 F   [20..32) zero
+ *   [32]    u8  fmt[768]        formats of (expert e, projection p) at e*3+p,
+ *                               p = 0 gate [F x H], 1 up [F x H], 2 down [H x F];
+ *                               entries past E*3 are zero
+ *   [800]   u64 code_off[768]   byte offset of each matrix's codes
+ *   [6944]  u64 scale_off[768]  byte offset of each matrix's scales
+ *   [13088] f32 tscale[768]     NVFP4 per-matrix scale (0 for integer formats)
+ *   [16160..16384) zero
+ * Sections follow from byte 16384 in (expert, projection) order, codes then
+ * scales, each starting on a 256-byte boundary.  Sizes for an N x K matrix:
+ * integer b-bit codes N*K*b/8 bytes, scales N*K/16 bytes (fp16 per 32);
+ * NVFP4 codes N*K/2 bytes, scales N*K/16 bytes (e4m3 per 16).
+ *
+ * Quantization of one N x K matrix (N outputs, K inputs, row-major fp32):
+ *   integer b-bit (qmax = 2^(b-1)-1; the code -2^(b-1) is not used):
+ *     per row n and group g of 32 consecutive inputs: amax = max|w|;
+ *     s = fp16 round-to-nearest-even of the fp32 quotient amax/qmax, saturated
+ *     to 65504; q = clamp(rint(w/s), -qmax, qmax) with an IEEE fp32 division
+ *     and round-half-even (s == 0 gives q = 0).  Dequantized weight = s*q.
+ *   NVFP4: sT = amax(matrix)/2688 in fp32 (1 if the matrix is all zero);
+ *     per row and block of 16 inputs: sb = e4m3(blockmax/(6*sT)) (round to
+ *     nearest even, saturate to 448); v = e2m1(w/(sb*sT)) (nearest even,
+ *     saturate to 6; sb == 0 gives v = 0).  Dequantized weight = e2m1(v)*sb*sT.
+ * Code layout: tiles of 128 outputs x 128 inputs, tile order output-block
+ * major, input-block minor.  Inside a tile, u32 words ordered
+ * [kg 0..3][word 0..b-1][n 0..127] (kg = group of 32 inputs inside the tile,
+ * b = 2, 3, 4 words per group; NVFP4 uses 4).  Stored integer code u = q+2^(b-1).
+ *   4-bit / NVFP4: code i of a group in word i/8, bits 4*(i%8)..+3
+ *   2-bit: code i in word i/16, bits 2*(i%16)..+1
+ *   3-bit: words 0-1 hold the low two bits of u as for 2-bit; bit i of word 2
+ *          holds bit 2 of u of code i.
+ * Scale layout: [N/128][K/gs][128] (gs = 32 integer, 16 NVFP4).
+ */
+
+/*
+ * moe_pack -- quantize and pack fp32 expert weights (the pages' expert packing,
+ * MoE mixed-precision page sec. 2.3/3.5; bit widths per expert/projection as on
+ * the AlphaQ page sec. 4.2).
+ *
+ * Size query: out == NULL -> *bytes_out = total size of the layer buffer; no
+ *   device work.  code_off / scale_off (HOST, [E*3], nullable) receive the
+ *   section offsets in both modes.
+ * Pack: writes the header and the sections of experts [e0, e0+ne) into `out`
+ *   (DEVICE, 256-byte aligned, out_bytes >= the queried size), so a layer too
+ *   large to stage in fp32 can be packed a few experts at a time.
+ *   W: DEVICE fp32 [ne][3][H*F] -- gate [F][H], up [F][H], down [H][F],
+ *   row-major, 16-byte aligned.  fmt: HOST u8 [E*3].
+ * Shapes: 1 <= E <= 256; H, F multiples of 128 (up to 32768).
+ * Errors: MOE_ERR_ARG (null W/fmt/bytes_out, bad e0/ne), MOE_ERR_SHAPE,
+ *   MOE_ERR_FORMAT, MOE_ERR_ALIGN, MOE_ERR_WORKSPACE (out_bytes too small),
+ *   MOE_ERR_UNSUPPORTED_DEVICE, MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_pack(const float* W, int32_t e0, int32_t ne, int32_t E, int32_t H, int32_t F,
+                    const uint8_t* fmt, void* out, uint64_t out_bytes, uint64_t* bytes_out,
+                    uint64_t* code_off, uint64_t* scale_off, cudaStream_t stream);
+
+/* A packed layer as moe_layer_forward reads it. */
+typedef struct {
+  int32_t E, H, F;
+  const uint8_t* fmt;   /* HOST [E*3]: must equal the fmt the buffer was packed with */
+  const void* packed;   /* DEVICE, 256-byte aligned, written by moe_pack */
+  uint64_t packed_bytes;
+} moe_weights;
+
+/* Optional outputs of moe_layer_forward; every pointer is DEVICE and nullable. */
+typedef struct {
+  int32_t* topk_idx;  /* [T*k] chosen experts, descending logit (ties: lower index) */
+  float* topk_w;      /* [T*k] softmax weights over the chosen k */
+  int32_t* perm;      /* [T*k] row r of the expert-sorted order holds entry t*k+j */
+  int32_t* inv;       /* [T*k] entry t*k+j -> its row */
+  int32_t* counts;    /* [E]   rows per expert */
+  uint8_t* xq;        /* [T*H] NVFP4 layers: e4m3 codes of x */
+  float* sx;          /* [T]   NVFP4 layers: per-token scale of x (amax/448) */
+  uint8_t* hq;        /* [T*k*F] NVFP4 layers: e4m3 codes of the SwiGLU output, sorted rows */
+  float* sh;          /* [T*k] NVFP4 layers: per-row scale of the SwiGLU output */
+  int32_t* status;    /* [1]   device-side error code (moe_status), 0 if none */
+  cudaEvent_t* stage_events; /* HOST [MOE_STAGE_EVENTS] or NULL: recorded on `stream` before
+                                router+top-k, permutation, activation gather/quantization,
+                                gate/up GEMM, h quantization (NVFP4), down GEMM, combine,
+                                and after combine, so stage times can be read back */
+} moe_debug;
+
+#define MOE_STAGE_EVENTS 8
+
+/*
+ * moe_layer_forward -- y = MoE(x).
+ *
+ * x: DEVICE bf16 [T][H], 16-byte aligned.  router_w: DEVICE fp32 [E][H]
+ *   (16-byte aligned); router_b: DEVICE fp32 [E] or NULL.  k: 1..min(E, 8).
+ * y: DEVICE bf16 [T][H] (16-byte aligned), fully overwritten.
+ * ws: DEVICE workspace, 256-byte aligned; ws == NULL -> *ws_bytes_out = the
+ *   size needed for (T, k, weights) and nothing runs.
+ * Steps (all on `stream`):
+ *   1. logits[t][e] = sum_h x[t][h]*Wr[e][h] (+ b[e]) accumulated in fp32
+ *      (the router stays unquantized: MoE mixed-precision page sec. 2.1);
+ *   2. top-k (ties to the lower expert index; NaN ranks lowest), then
+ *      w = softmax over the k chosen logits (expert-routing section of the
+ *      quantized-MoE-inference page);
+ *   3. counts per expert, exclusive offsets and a stable permutation (rows of
+ *      one expert in ascending token order);
+ *   4. NVFP4 layers only: per-token dynamic FP8 e4m3 codes of x with scale
+ *      amax/448 (MoE mixed-precision page sec. 2.1);
+ *   5. per expert: h = silu(Wg x) * (Wu x) with fp32 accumulation on
+ *      dequantized weights (integer formats: fp16 operands, weights rounded
+ *      once to fp16 as s*q; NVFP4: exact bf16 operands, scales applied after
+ *      the sum); NVFP4 layers then quantize each h row to e4m3 (amax/448);
+ *   6. o = Wd h per row; y[t] = bf16( sum_j w[t][j] * o[row(t,j)] ) summed in
+ *      fp32 in ascending j.
+ * Integer-format layers convert x and h to fp16, so |x| and |h| must stay
+ * below 65504.  Layers must be all-NVFP4 or all-integer (MOE_ERR_FORMAT).
+ * Errors: MOE_ERR_ARG, MOE_ERR_ALIGN, MOE_ERR_SHAPE, MOE_ERR_FORMAT,
+ *   MOE_ERR_WORKSPACE, MOE_ERR_UNSUPPORTED_DEVICE, MOE_ERR_CUDA.
+ */
+MOE_API moe_status moe_layer_forward(const void* x, int32_t T, const float* router_w, const float* router_b,
+                             const moe_weights* w, int32_t k, void* y, void* ws, uint64_t ws_bytes,
+                             uint64_t* ws_bytes_out, const moe_debug* dbg, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

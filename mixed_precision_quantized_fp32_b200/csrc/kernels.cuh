@@ -1,0 +1,29 @@
+// Launchers of the CUDA kernels, called by the host ABI (abi.cu).
+#pragma once
+#include "moe_common.cuh"
+
+namespace moe {
+
+cudaError_t launch_pack(const float* W, int e0, int ne, int E, int H, int F, const uint8_t* fmt_host,
+                        uint8_t* out, const uint64_t* code_off, const uint64_t* scale_off,
+                        cudaStream_t stream);
+
+cudaError_t launch_router_topk(const __nv_bfloat16* x, const float* Wr, const float* b, int T, int H,
+                               int E, int k, const Workspace& ws, int32_t* dbg_idx, float* dbg_w,
+                               cudaStream_t stream);
+
+cudaError_t launch_permute(int T, int k, int E, int chunk_rows, const Workspace& ws, int32_t* dbg_counts,
+                           int32_t* dbg_perm, int32_t* dbg_inv, cudaStream_t stream);
+
+cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4, const Workspace& ws,
+                          uint8_t* dbg_xq, float* dbg_sx, cudaStream_t stream);
+
+cudaError_t launch_act_quant_h(int R, int F, const Workspace& ws, uint8_t* dbg_hq, float* dbg_sh,
+                               cudaStream_t stream);
+
+cudaError_t launch_expert_gemm_mma(const uint8_t* packed, int E, int H, int F, int k, bool fp4, bool gateup,
+                                   int chunk_rows, int max_chunks, const Workspace& ws, cudaStream_t stream);
+
+cudaError_t launch_combine(int T, int k, int H, const Workspace& ws, __nv_bfloat16* y, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,139 @@
+// Shared device/host definitions of the packed layer layout and small helpers
+// for the CUDA library.  (The CPU oracle has its own, independent copy of the
+// layout definition; nothing here is shared with it.)
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr uint32_t kMagic = 0x51454F4Du;
+constexpr uint32_t kHdrBytes = 16384u;
+constexpr uint32_t kOffFmt = 32u;
+constexpr uint32_t kOffCode = 800u;
+constexpr uint32_t kOffScale = 6944u;
+constexpr uint32_t kOffTscale = 13088u;
+constexpr int kMaxE = 256;
+constexpr int kMaxK = 8;
+
+__host__ __device__ inline bool fmt_known(int f) {
+  return f == MOE_FMT_INT2 || f == MOE_FMT_INT3 || f == MOE_FMT_INT4 || f == MOE_FMT_NVFP4;
+}
+// u32 words per group of 32 inputs
+__host__ __device__ inline int fmt_words(int f) { return f == MOE_FMT_NVFP4 ? 4 : f; }
+
+__host__ __device__ inline uint64_t code_bytes(int f, uint64_t N, uint64_t K) {
+  return N * K * (uint64_t)fmt_words(f) / 8u;
+}
+__host__ __device__ inline uint64_t scale_bytes(int f, uint64_t N, uint64_t K) {
+  return f == MOE_FMT_NVFP4 ? N * (K / 16) : N * (K / 32) * 2u;
+}
+__host__ __device__ inline uint64_t up256(uint64_t x) { return (x + 255u) & ~(uint64_t)255u; }
+
+// N x K of projection p (0 gate, 1 up: F x H; 2 down: H x F)
+__host__ __device__ inline void proj_shape(int p, int H, int F, int& N, int& K) {
+  if (p < 2) { N = F; K = H; } else { N = H; K = F; }
+}
+
+// Section offsets of a whole layer; returns false on an unknown format.
+__host__ __device__ inline bool layer_layout(int E, int H, int F, const uint8_t* fmt,
+                                             uint64_t* code_off, uint64_t* scale_off,
+                                             uint64_t* total) {
+  uint64_t pos = kHdrBytes;
+  for (int e = 0; e < E; ++e)
+    for (int p = 0; p < 3; ++p) {
+      const int f = fmt[e * 3 + p];
+      if (!fmt_known(f)) return false;
+      int N, K;
+      proj_shape(p, H, F, N, K);
+      pos = up256(pos);
+      if (code_off) code_off[e * 3 + p] = pos;
+      pos += code_bytes(f, N, K);
+      pos = up256(pos);
+      if (scale_off) scale_off[e * 3 + p] = pos;
+      pos += scale_bytes(f, N, K);
+    }
+  if (total) *total = up256(pos);
+  return true;
+}
+
+// Word index (u32 units) of word w of the group holding input k of output n.
+__host__ __device__ inline uint64_t word_index(int n, int k, int K, int wpg, int w) {
+  const uint64_t nb = (uint64_t)(n >> 7), kb = (uint64_t)(k >> 7);
+  const uint64_t kg = (uint64_t)((k & 127) >> 5);
+  return (((nb * (uint64_t)(K >> 7) + kb) * 4u + kg) * (uint64_t)wpg + (uint64_t)w) * 128u +
+         (uint64_t)(n & 127);
+}
+// Scale index of (output n, group g) with `groups` groups per row.
+__host__ __device__ inline uint64_t scale_index(int n, int g, int groups) {
+  return ((uint64_t)(n >> 7) * (uint64_t)groups + (uint64_t)g) * 128u + (uint64_t)(n & 127);
+}
+
+// Device-side view of a packed layer header.
+struct LayerHdr {
+  int E, H, F;
+  const uint8_t* fmt;
+  const uint64_t* code_off;
+  const uint64_t* scale_off;
+  const float* tscale;
+  const uint8_t* base;
+};
+
+__host__ __device__ inline LayerHdr hdr_view(const void* packed, int E, int H, int F) {
+  LayerHdr h;
+  h.base = (const uint8_t*)packed;
+  h.E = E;
+  h.H = H;
+  h.F = F;
+  h.fmt = h.base + kOffFmt;
+  h.code_off = (const uint64_t*)(h.base + kOffCode);
+  h.scale_off = (const uint64_t*)(h.base + kOffScale);
+  h.tscale = (const float*)(h.base + kOffTscale);
+  return h;
+}
+
+// e2m1 code (sign<<3 | exp<<1 | man) -> float
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  const uint32_t m = c & 7u;
+  // magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6
+  const float mag = (m < 2u) ? 0.5f * (float)m : (float)((2u | (m & 1u)) << ((m >> 1) - 1u)) * 0.5f;
+  return (c & 8u) ? -mag : mag;
+}
+
+// e4m3 ("fn") code -> float (NaN codes not produced by this library)
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+  const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+  float v = (e == 0u) ? (float)m * 0.001953125f /* 2^-9 */
+                      : __uint_as_float(((e + 120u) << 23) | (m << 20));
+  return (c & 0x80u) ? -v : v;
+}
+
+// Workspace layout shared by the host ABI and the kernels.
+struct Workspace {
+  float* logits;       // [T*E]
+  int32_t* idx;        // [T*k]
+  float* wts;          // [T*k]
+  int32_t* counts;     // [E]
+  int32_t* offsets;    // [E+1]
+  int32_t* blk_hist;   // [nblk*E]
+  int32_t* rank;       // [T*k] stable rank of each entry inside its count block
+  int32_t* perm;       // [T*k]
+  int32_t* inv;        // [T*k]
+  int32_t* chunks;     // [max_chunks*3] (expert, row0, rows) + [1] count at chunk_count
+  int32_t* chunk_count;// [1]
+  uint8_t* xq;         // [T*H] NVFP4 activation codes
+  float* sx;           // [T]
+  void* xs;            // [T*k*H] 16-bit gathered activations (fp16 int / bf16 NVFP4)
+  void* h;             // [T*k*F] fp16 (int) / fp32 (NVFP4 pre-quant)
+  void* hb;            // [T*k*F] bf16 NVFP4 decoded h codes
+  uint8_t* hq;         // [T*k*F] NVFP4 h codes
+  float* sh;           // [T*k]
+  float* o;            // [T*k*H] fp32 expert outputs, sorted rows
+  int32_t* status;     // [1]
+};
+
+}  // namespace moe

@@ -1,0 +1,243 @@
+// Token permutation by expert (histogram -> exclusive scan -> stable scatter),
+// the gather of activation rows into expert-sorted order, and the per-row
+// dynamic FP8 activation quantization of NVFP4 layers (MoE mixed-precision
+// page sec. 2.1: per-token scales from the live min/max; e4m3, amax/448).
+#include <cuda_fp8.h>
+
+#include "moe_common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+constexpr int kPermBlock = 1024;
+
+// Pass 1: per block of 1024 entries (t*k+j order), the expert histogram and the
+// stable rank of each entry among the block's entries of the same expert.
+__global__ void __launch_bounds__(kPermBlock) perm_count_kernel(const int32_t* __restrict__ idx, int R,
+                                                                int E, int32_t* __restrict__ blk_hist,
+                                                                int32_t* __restrict__ rank) {
+  __shared__ int32_t wcnt[kPermBlock / 32][kMaxE];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < (kPermBlock / 32) * kMaxE; i += kPermBlock) (&wcnt[0][0])[i] = 0;
+  __syncthreads();
+  const int i = blockIdx.x * kPermBlock + tid;
+  const bool valid = i < R;
+  const int e = valid ? idx[i] : -1;
+  const unsigned same = __match_any_sync(0xffffffffu, e);
+  const int rw = __popc(same & ((1u << lane) - 1u));
+  if (valid && rw == 0) wcnt[warp][e] = __popc(same);
+  __syncthreads();
+  if (valid) {
+    int r = rw;
+    for (int w = 0; w < warp; ++w) r += wcnt[w][e];
+    rank[i] = r;
+  }
+  for (int ee = tid; ee < E; ee += kPermBlock) {
+    int s = 0;
+    for (int w = 0; w < kPermBlock / 32; ++w) s += wcnt[w][ee];
+    blk_hist[(size_t)blockIdx.x * E + ee] = s;
+  }
+}
+
+// Pass 2 (one block of 256 threads, thread e = expert e): per-expert totals,
+// exclusive offsets, per-block bases, and the list of (expert, first row,
+// rows) chunks of at most `chunk_rows` rows that the expert GEMMs walk.
+__global__ void __launch_bounds__(256) perm_scan_kernel(int32_t* __restrict__ blk_hist, int nblk, int E,
+                                                        int R, int chunk_rows, int32_t* __restrict__ counts,
+                                                        int32_t* __restrict__ offsets,
+                                                        int32_t* __restrict__ chunks,
+                                                        int32_t* __restrict__ chunk_count,
+                                                        int32_t* __restrict__ dbg_counts) {
+  __shared__ int32_t s_cnt[kMaxE], s_off[kMaxE + 1], s_nc[kMaxE], s_cstart[kMaxE + 1];
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E) {
+    for (int b = 0; b < nblk; ++b) {
+      const int v = blk_hist[(size_t)b * E + e];
+      blk_hist[(size_t)b * E + e] = total;
+      total += v;
+    }
+  }
+  s_cnt[e] = (e < E) ? total : 0;
+  s_nc[e] = (e < E) ? (total + chunk_rows - 1) / chunk_rows : 0;
+  __syncthreads();
+  if (e == 0) {
+    int run = 0, crun = 0;
+    for (int j = 0; j < E; ++j) {
+      s_off[j] = run;
+      run += s_cnt[j];
+      s_cstart[j] = crun;
+      crun += s_nc[j];
+    }
+    s_off[E] = run;
+    s_cstart[E] = crun;
+    *chunk_count = crun;
+    offsets[E] = run;
+  }
+  __syncthreads();
+  if (e < E) {
+    counts[e] = total;
+    offsets[e] = s_off[e];
+    if (dbg_counts) dbg_counts[e] = total;
+    for (int b = 0; b < nblk; ++b) blk_hist[(size_t)b * E + e] += s_off[e];
+    for (int c = 0; c < s_nc[e]; ++c) {
+      const int row0 = c * chunk_rows;
+      int32_t* ch = chunks + 3 * (size_t)(s_cstart[e] + c);
+      ch[0] = e;
+      ch[1] = s_off[e] + row0;
+      ch[2] = min(chunk_rows, total - row0);
+    }
+  }
+}
+
+// Pass 3: row = block base of the expert + stable rank; perm[row] = entry, inv[entry] = row.
+__global__ void __launch_bounds__(kPermBlock) perm_scatter_kernel(const int32_t* __restrict__ idx, int R,
+                                                                  int E, const int32_t* __restrict__ blk_hist,
+                                                                  const int32_t* __restrict__ rank,
+                                                                  int32_t* __restrict__ perm,
+                                                                  int32_t* __restrict__ inv,
+                                                                  int32_t* __restrict__ dbg_perm,
+                                                                  int32_t* __restrict__ dbg_inv) {
+  const int i = blockIdx.x * kPermBlock + threadIdx.x;
+  if (i >= R) return;
+  const int e = idx[i];
+  const int row = blk_hist[(size_t)blockIdx.x * E + e] + rank[i];
+  perm[row] = i;
+  inv[i] = row;
+  if (dbg_perm) dbg_perm[row] = i;
+  if (dbg_inv) dbg_inv[i] = row;
+}
+
+// Gather x rows into expert-sorted order as fp16 (integer-format layers).
+__global__ void gather_f16_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm,
+                                  int R, int H, int k, __half* __restrict__ xs) {
+  const int r = blockIdx.x;
+  const int t = perm[r] / k;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+  uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)r * H);
+  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
+    const uint4 v = __ldg(src + c);
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+    uint4 o;
+    __half2* h2 = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h2[i] = __float22half2_rn(__bfloat1622float2(b2[i]));
+    dst[c] = o;
+  }
+}
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    v = (lane < (int)(blockDim.x >> 5)) ? red[lane] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (lane == 0) red[0] = v;
+  }
+  __syncthreads();
+  v = red[0];
+  __syncthreads();
+  return v;
+}
+
+// Per-token e4m3 codes of x: s = amax/448 (1 if amax == 0); q = e4m3(x/s), RNE, saturating.
+__global__ void act_quant_x_kernel(const __nv_bfloat16* __restrict__ x, int H, uint8_t* __restrict__ xq,
+                                   float* __restrict__ sx, uint8_t* __restrict__ dbg_xq,
+                                   float* __restrict__ dbg_sx) {
+  __shared__ float red[32];
+  const int t = blockIdx.x;
+  const __nv_bfloat16* xr = x + (size_t)t * H;
+  float m = 0.0f;
+  for (int h = threadIdx.x; h < H; h += blockDim.x) m = fmaxf(m, fabsf(__bfloat162float(xr[h])));
+  const float amax = block_max(m, red);
+  const float s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+  for (int h = threadIdx.x; h < H; h += blockDim.x) {
+    const uint8_t c = __nv_cvt_float_to_fp8(__fdiv_rn(__bfloat162float(xr[h]), s), __NV_SATFINITE, __NV_E4M3);
+    xq[(size_t)t * H + h] = c;
+    if (dbg_xq) dbg_xq[(size_t)t * H + h] = c;
+  }
+  if (threadIdx.x == 0) {
+    sx[t] = s;
+    if (dbg_sx) dbg_sx[t] = s;
+  }
+}
+
+// Gather e4m3 activation codes into sorted rows as exact bf16 values.
+__global__ void gather_fp8_kernel(const uint8_t* __restrict__ xq, const int32_t* __restrict__ perm, int R,
+                                  int H, int k, __nv_bfloat16* __restrict__ xs) {
+  const int r = blockIdx.x;
+  const int t = perm[r] / k;
+  const uint2* src = reinterpret_cast<const uint2*>(xq + (size_t)t * H);
+  uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)r * H);
+  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
+    const uint2 v = __ldg(src + c);
+    uint4 o;
+    __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ob[i] = __float2bfloat16_rn(e4m3_value((v.x >> (8 * i)) & 255u));
+      ob[4 + i] = __float2bfloat16_rn(e4m3_value((v.y >> (8 * i)) & 255u));
+    }
+    dst[c] = o;
+  }
+}
+
+// Per-row e4m3 codes of the SwiGLU output (NVFP4 layers) and their exact bf16 values.
+__global__ void act_quant_h_kernel(const float* __restrict__ h, int F, uint8_t* __restrict__ hq,
+                                   float* __restrict__ sh, __nv_bfloat16* __restrict__ hb,
+                                   uint8_t* __restrict__ dbg_hq, float* __restrict__ dbg_sh) {
+  __shared__ float red[32];
+  const int r = blockIdx.x;
+  const float* hr = h + (size_t)r * F;
+  float m = 0.0f;
+  for (int i = threadIdx.x; i < F; i += blockDim.x) m = fmaxf(m, fabsf(hr[i]));
+  const float amax = block_max(m, red);
+  const float s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+  for (int i = threadIdx.x; i < F; i += blockDim.x) {
+    const uint8_t c = __nv_cvt_float_to_fp8(__fdiv_rn(hr[i], s), __NV_SATFINITE, __NV_E4M3);
+    hq[(size_t)r * F + i] = c;
+    hb[(size_t)r * F + i] = __float2bfloat16_rn(e4m3_value(c));
+    if (dbg_hq) dbg_hq[(size_t)r * F + i] = c;
+  }
+  if (threadIdx.x == 0) {
+    sh[r] = s;
+    if (dbg_sh) dbg_sh[r] = s;
+  }
+}
+
+cudaError_t launch_permute(int T, int k, int E, int chunk_rows, const Workspace& ws, int32_t* dbg_counts,
+                           int32_t* dbg_perm, int32_t* dbg_inv, cudaStream_t stream) {
+  const int R = T * k;
+  const int nblk = (R + kPermBlock - 1) / kPermBlock;
+  perm_count_kernel<<<nblk, kPermBlock, 0, stream>>>(ws.idx, R, E, ws.blk_hist, ws.rank);
+  perm_scan_kernel<<<1, 256, 0, stream>>>(ws.blk_hist, nblk, E, R, chunk_rows, ws.counts, ws.offsets,
+                                          ws.chunks, ws.chunk_count, dbg_counts);
+  perm_scatter_kernel<<<nblk, kPermBlock, 0, stream>>>(ws.idx, R, E, ws.blk_hist, ws.rank, ws.perm, ws.inv,
+                                                       dbg_perm, dbg_inv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4, const Workspace& ws,
+                          uint8_t* dbg_xq, float* dbg_sx, cudaStream_t stream) {
+  const int R = T * k;
+  if (fp4) {
+    act_quant_x_kernel<<<T, 256, 0, stream>>>(x, H, ws.xq, ws.sx, dbg_xq, dbg_sx);
+    gather_fp8_kernel<<<R, 128, 0, stream>>>(ws.xq, ws.perm, R, H, k, (__nv_bfloat16*)ws.xs);
+  } else {
+    gather_f16_kernel<<<R, 128, 0, stream>>>(x, ws.perm, R, H, k, (__half*)ws.xs);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_act_quant_h(int R, int F, const Workspace& ws, uint8_t* dbg_hq, float* dbg_sh,
+                               cudaStream_t stream) {
+  act_quant_h_kernel<<<R, 256, 0, stream>>>((const float*)ws.h, F, ws.hq, ws.sh, (__nv_bfloat16*)ws.hb,
+                                            dbg_hq, dbg_sh);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -283,6 +283,8 @@ ORC_EXPORT void orc_pack_int(const int8_t* q, const uint16_t* s16, int N, int K,
   memset(codes, 0, orc_code_bytes(bits, N, K));
   uint32_t* words = (uint32_t*)codes;
   const int off = 1 << (bits - 1);
+  /* rows own disjoint words, so rows can be packed in parallel */
+#pragma omp parallel for schedule(static)
   for (int n = 0; n < N; ++n)
     for (int k = 0; k < K; ++k)
       put_code(words, n, k, K, bits, (uint32_t)(q[(size_t)n * K + k] + off));
@@ -306,6 +308,7 @@ ORC_EXPORT void orc_pack_nvfp4(const uint8_t* v, const uint8_t* sb, int N, int K
                                uint8_t* scales) {
   memset(codes, 0, orc_code_bytes(ORC_NVFP4, N, K));
   uint32_t* words = (uint32_t*)codes;
+#pragma omp parallel for schedule(static)
   for (int n = 0; n < N; ++n)
     for (int k = 0; k < K; ++k) put_code(words, n, k, K, ORC_NVFP4, v[(size_t)n * K + k]);
   for (int n = 0; n < N; ++n)
@@ -410,6 +413,8 @@ ORC_EXPORT int orc_pack_layer(const float* W, int e0, int ne, int E, int H, int 
   memset(out + ORC_OFF_SCALE, 0, 768 * 8);
   memcpy(out + ORC_OFF_SCALE, scale_off, (size_t)E * 3 * 8);
   memset(out + ORC_OFF_TS + 3072, 0, ORC_HDR_BYTES - ORC_OFF_TS - 3072);
+  /* tensor-scale slots past the layer's E*3 entries are zero */
+  memset(out + ORC_OFF_TS + (size_t)E * 3 * 4, 0, (size_t)(768 - E * 3) * 4);
   float* ts = (float*)(out + ORC_OFF_TS);
   for (int i = 0; i < ne; ++i) {
     int e = e0 + i;

@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point declared in include/moe.h, sizes its buffers like the
+oracle's independent layout, and rejects bad arguments before launching.
+Pointers passed here are fake device addresses: validation must return
+before anything touches them."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+import gen.workloads as W
+import mixed_precision_quantized_fp32_b200 as moe
+from mixed_precision_quantized_fp32_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ST = {v: k for k, v in _lib.STATUS.items()}
+FAKE = 0x7F0000000000  # 256-byte aligned, never dereferenced
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"MOE_API\s+\w+\s+(\w+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol():
+    L = _lib.load()
+    names = declared_symbols()
+    assert {"moe_pack", "moe_layer_forward"} <= names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_layout_matches_oracle(orc):
+    for name in W.NAMES:
+        L = W.layer(name)
+        total, co, so = moe.pack_layout(L.E, L.H, L.F, L.fmt)
+        oco, oso, ototal = orc.layer_layout(L.E, L.H, L.F, L.fmt)
+        assert total == ototal
+        np.testing.assert_array_equal(co, oco)
+        np.testing.assert_array_equal(so, oso)
+
+
+def _pack(W_ptr, e0, ne, E, H, F, fmt, out, out_bytes, want_total=True):
+    total = C.c_uint64(0)
+    f = None if fmt is None else np.ascontiguousarray(fmt, np.uint8).ravel()
+    rc = _lib.load().moe_pack(W_ptr, e0, ne, E, H, F, None if f is None else f.ctypes.data, out, out_bytes,
+                              C.byref(total) if want_total else None, None, None, None)
+    return _lib.STATUS[rc], total.value
+
+
+def test_pack_argument_errors():
+    fmt = np.full((4, 3), 4, np.uint8)
+    total = moe.pack_layout(4, 256, 256, fmt)[0]
+    assert _pack(None, 0, 0, 4, 256, 256, fmt, None, 0)[0] == "MOE_OK"
+    assert _pack(None, 0, 0, 4, 256, 256, None, None, 0)[0] == "MOE_ERR_ARG"
+    assert _pack(None, 0, 0, 4, 200, 256, fmt, None, 0)[0] == "MOE_ERR_SHAPE"
+    assert _pack(None, 0, 0, 4, 256, 0, fmt, None, 0)[0] == "MOE_ERR_SHAPE"
+    assert _pack(None, 0, 0, 257, 256, 256, np.full((257, 3), 4), None, 0)[0] == "MOE_ERR_SHAPE"
+    bad = fmt.copy()
+    bad[2, 1] = 5
+    assert _pack(None, 0, 0, 4, 256, 256, bad, None, 0)[0] == "MOE_ERR_FORMAT"
+    assert _pack(None, 0, 0, 4, 256, 256, fmt, None, 0, want_total=False)[0] == "MOE_ERR_ARG"
+    assert _pack(None, 0, 1, 4, 256, 256, fmt, FAKE, total)[0] == "MOE_ERR_ARG"   # W null
+    assert _pack(FAKE, 3, 2, 4, 256, 256, fmt, FAKE, total)[0] == "MOE_ERR_ARG"   # e0+ne > E
+    assert _pack(FAKE, -1, 1, 4, 256, 256, fmt, FAKE, total)[0] == "MOE_ERR_ARG"
+    assert _pack(FAKE, 0, 1, 4, 256, 256, fmt, FAKE + 16, total)[0] == "MOE_ERR_ALIGN"
+    assert _pack(FAKE + 4, 0, 1, 4, 256, 256, fmt, FAKE, total)[0] == "MOE_ERR_ALIGN"
+    assert _pack(FAKE, 0, 1, 4, 256, 256, fmt, FAKE, total - 1)[0] == "MOE_ERR_WORKSPACE"
+
+
+def _fwd(T, k, E=8, H=256, F=512, fmt=None, x=FAKE, rw=FAKE, y=FAKE, packed=FAKE, packed_bytes=None,
+         ws=FAKE, ws_bytes=1 << 40, query=False):
+    fmt = np.full((E, 3), 4, np.uint8) if fmt is None else np.asarray(fmt, np.uint8)
+    f = np.ascontiguousarray(fmt).ravel()
+    if packed_bytes is None:
+        packed_bytes = moe.pack_layout(E, H, F, f)[0] if (E <= 256 and H % 128 == 0 and F % 128 == 0
+                                                          and set(f) <= {2, 3, 4, 16}) else 1 << 40
+    w = _lib.MoeWeights(E, H, F, f.ctypes.data, packed, packed_bytes)
+    need = C.c_uint64(0)
+    rc = _lib.load().moe_layer_forward(x, T, rw, None, C.byref(w), k, y, None if query else ws, ws_bytes,
+                                       C.byref(need), None, None)
+    return _lib.STATUS[rc], need.value
+
+
+def test_forward_argument_errors():
+    st, need = _fwd(16, 2, query=True)
+    assert st == "MOE_OK" and need > 0
+    st, need64 = _fwd(64, 2, query=True)
+    assert need64 > need
+    assert _fwd(16, 0)[0] == "MOE_ERR_SHAPE"
+    assert _fwd(16, 9, E=16)[0] == "MOE_ERR_SHAPE"
+    assert _fwd(16, 5, E=4)[0] == "MOE_ERR_SHAPE"
+    assert _fwd(-1, 2)[0] == "MOE_ERR_SHAPE"
+    assert _fwd(16, 2, H=200)[0] == "MOE_ERR_SHAPE"
+    mixed = np.full((8, 3), 16, np.uint8)
+    mixed[3, 2] = 4
+    assert _fwd(16, 2, fmt=mixed)[0] == "MOE_ERR_FORMAT"
+    assert _fwd(16, 2, fmt=np.full((8, 3), 7))[0] == "MOE_ERR_FORMAT"
+    assert _fwd(0, 2)[0] == "MOE_OK"                      # empty batch: nothing to do
+    assert _fwd(16, 2, x=None)[0] == "MOE_ERR_ARG"
+    assert _fwd(16, 2, y=None)[0] == "MOE_ERR_ARG"
+    assert _fwd(16, 2, rw=None)[0] == "MOE_ERR_ARG"
+    assert _fwd(16, 2, packed=None)[0] == "MOE_ERR_ARG"
+    assert _fwd(16, 2, x=FAKE + 8)[0] == "MOE_ERR_ALIGN"
+    assert _fwd(16, 2, packed=FAKE + 128)[0] == "MOE_ERR_ALIGN"
+    assert _fwd(16, 2, ws=FAKE + 64)[0] == "MOE_ERR_ALIGN"
+    assert _fwd(16, 2, ws_bytes=need - 1)[0] == "MOE_ERR_WORKSPACE"
+    total = moe.pack_layout(8, 256, 512, np.full((8, 3), 4))[0]
+    assert _fwd(16, 2, packed_bytes=total - 1)[0] == "MOE_ERR_WORKSPACE"
+
+
+def test_valid_call_without_gpu_fails_cleanly():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    st, _ = _fwd(16, 2)
+    assert st in ("MOE_ERR_CUDA", "MOE_ERR_UNSUPPORTED_DEVICE")

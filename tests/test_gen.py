@@ -34,3 +34,10 @@ def test_permutation():
     p = gen.permutation(0, gen.TID_PERM, 256)
     assert sorted(p.tolist()) == list(range(256))
     np.testing.assert_array_equal(p, gen.permutation(0, gen.TID_PERM, 256))
+
+
+def test_host_c_twin_matches_numpy():
+    for tid, sigma in [(1, 1.0), (17, 0.02), (gen.tid_expert(200, 2), 0.02)]:
+        a = gen.normal_f32(3, tid, 12345, 50_000, sigma)
+        b = gen.fill_f32(3, tid, 50_000, sigma, start=12345)
+        np.testing.assert_array_equal(a, b)

@@ -1,0 +1,317 @@
+"""GPU parity: the CUDA library (through the C ABI) against the CPU oracle.
+
+Bars (per layer):
+  * packed codes, scales and header bytes: bit-exact;
+  * permutation rows and per-expert counts: bit-exact;
+  * top-k sets: exact except where the oracle's k-th vs (k+1)-th logit gap is
+    below 1e-5 (counted; the oracle is then re-fed the GPU's choice);
+  * top-k weights: within 1e-6;
+  * NVFP4 layers: FP8 codes and scales of x bit-exact;
+  * outputs: max |y_gpu - y_oracle| <= 2e-2 * max |y_oracle|.
+"""
+import numpy as np
+import pytest
+
+import gen
+import gen.workloads as W
+import oracle as orc
+from tests import helpers as hp
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import mixed_precision_quantized_fp32_b200 as moe  # noqa: E402
+
+
+def custom(name, T, H, F, E, k, fmt, bias=None):
+    L = W.Layer(name, H, F, E, k, np.asarray(fmt, np.uint8).reshape(E, 3), (T,), (), bias)
+    return L
+
+
+def run_gpu(L, layer, T, x=None, Wr=None, b=None, k=None):
+    k = k or L.k
+    x = W.device_x(T, L.H) if x is None else x
+    if Wr is None:
+        Wr, b = W.device_router(L)
+    R = T * k
+    dbg = dict(topk_idx=torch.empty(R, dtype=torch.int32, device="cuda"),
+               topk_w=torch.empty(R, dtype=torch.float32, device="cuda"),
+               perm=torch.empty(R, dtype=torch.int32, device="cuda"),
+               inv=torch.empty(R, dtype=torch.int32, device="cuda"),
+               counts=torch.empty(L.E, dtype=torch.int32, device="cuda"),
+               status=torch.zeros(1, dtype=torch.int32, device="cuda"))
+    if L.fp4:
+        dbg.update(xq=torch.empty(T * L.H, dtype=torch.uint8, device="cuda"),
+                   sx=torch.empty(T, dtype=torch.float32, device="cuda"),
+                   hq=torch.empty(R * L.F, dtype=torch.uint8, device="cuda"),
+                   sh=torch.empty(R, dtype=torch.float32, device="cuda"))
+    y = moe.moe_layer_forward(x, Wr, b, layer, k, debug=dbg)
+    torch.cuda.synchronize()
+    out = {n: t.cpu().numpy() for n, t in dbg.items()}
+    out["y"] = y
+    assert out["status"][0] == 0
+    return out
+
+
+def check_layer(L, T, tokens=None, bias=None, router_zero=False, max_ties=None):
+    """Full parity of one layer / batch.  tokens: the subset whose outputs are
+    compared against the oracle (default all)."""
+    k = L.k
+    layer = hp.gpu_pack_cached(L) if L.name in W.NAMES else hp.gpu_pack(L)
+    x_bits = W.x_bf16_bits(T, L.H)
+    Wr_h = np.zeros((L.E, L.H), np.float32) if router_zero else W.router_w(L.E, L.H)
+    b_h = bias if bias is not None else L.bias
+    Wr = torch.from_numpy(Wr_h).cuda()
+    b = None if b_h is None else torch.from_numpy(np.asarray(b_h, np.float32)).cuda()
+    g = run_gpu(L, layer, T, Wr=Wr, b=b)
+
+    logits, idx_o, w_o = hp.oracle_route(x_bits, Wr_h, b_h, k)
+    idx_g = g["topk_idx"].reshape(T, k)
+    ties = hp.near_tie_tokens(logits, k, idx_g, idx_o)
+    if max_ties is not None:
+        assert len(ties) <= max_ties
+    same = np.setdiff1d(np.arange(T), ties)
+    np.testing.assert_array_equal(idx_g[same], idx_o[same])
+    np.testing.assert_allclose(g["topk_w"].reshape(T, k)[same], w_o[same], rtol=0, atol=1e-6)
+    # permutation of the GPU's own choice: bit-exact against the oracle's permutation step
+    counts, offsets, perm, inv = orc.permute(idx_g.astype(np.int32), L.E)
+    np.testing.assert_array_equal(g["counts"], counts)
+    np.testing.assert_array_equal(g["perm"], perm)
+    np.testing.assert_array_equal(g["inv"], inv)
+    if L.fp4:
+        xq, sx = orc.act_quant_e4m3(gen.bf16_bits_to_f32(x_bits))
+        np.testing.assert_array_equal(g["xq"].reshape(T, L.H), xq)
+        np.testing.assert_array_equal(g["sx"], sx)
+
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens)
+    experts = np.unique(np.concatenate([idx_o[tokens].ravel(), idx_g[tokens].ravel()]))
+    buf = hp.oracle_pack(L, experts)
+    y_ref, _, _ = hp.oracle_forward_rows(buf, x_bits, Wr_h, b_h, k, tokens=tokens,
+                                         idx_override=idx_g if ties else None, fp4=L.fp4)
+    ratio = hp.check_output(g["y"][torch.from_numpy(tokens).cuda()], y_ref)
+    return dict(ties=len(ties), err_ratio=ratio, counts=g["counts"])
+
+
+# ------------------------------------------------------------------ generator / packing
+def test_device_generator_matches_host():
+    for tid, sigma, n in [(1, 1.0, 100_003), (gen.tid_expert(3, 2), 0.02, 65_536)]:
+        t = torch.empty(n, dtype=torch.float32, device="cuda")
+        W.fill_device_f32(t, 0, tid, sigma, start=77)
+        np.testing.assert_array_equal(t.cpu().numpy(), gen.normal_f32(0, tid, 77, n, sigma))
+        b = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        W.fill_device_bf16(b, 0, tid, sigma)
+        np.testing.assert_array_equal(b.view(torch.int16).cpu().numpy().view(np.uint16),
+                                      gen.normal_bf16_bits(0, tid, 0, n, sigma))
+
+
+PACK_CASES = [
+    ("int4", 384, 256, 3, [[4, 4, 4]] * 3),
+    ("mixed", 256, 640, 6, [[3, 2, 4], [4, 4, 4], [2, 2, 2], [4, 4, 2], [3, 3, 3], [2, 4, 3]]),
+    ("nvfp4", 256, 384, 4, [[16, 16, 16]] * 4),
+]
+
+
+@pytest.mark.parametrize("name,H,F,E,fmt", PACK_CASES)
+def test_pack_bit_exact(name, H, F, E, fmt):
+    L = custom(name, 1, H, F, E, 1, fmt)
+    layer = hp.gpu_pack(L, experts_per_call=2)
+    got = layer.packed.cpu().numpy()
+    want = hp.oracle_pack(L, range(E))
+    np.testing.assert_array_equal(got, want)
+
+
+def test_pack_edge_values_bit_exact():
+    # all-zero expert, tiny values (fp16-subnormal scales), a large-magnitude group
+    L = custom("edge", 1, 256, 256, 3, 1, [[4, 3, 2], [16, 16, 16], [2, 4, 3]])
+    fmt = L.fmt.reshape(-1)
+    Wh = np.stack([W.expert_w(e, 256, 256) for e in range(3)])
+    Wh[0, 1] = 0.0
+    Wh[1, 0, :4096] *= np.float32(1e-7)
+    Wh[2, 2, :64] *= np.float32(3000.0)
+    total = moe.pack_layout(3, 256, 256, fmt)[0]
+    packed = moe.alloc_packed(total)
+    moe.moe_pack(torch.from_numpy(Wh).cuda(), 0, 3, 256, 256, fmt, packed)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(packed.cpu().numpy(), orc.pack_layer(Wh, 0, 3, 256, 256, fmt))
+
+
+@pytest.mark.parametrize("name", ["tiny", "mixtral", "hotcold", "nvfp4", "large"])
+def test_pack_bit_exact_configs(name):
+    L = W.layer(name)
+    layer = hp.gpu_pack_cached(L)
+    if name == "tiny":
+        sample = range(L.E)
+    elif name == "hotcold":
+        hot = L.notes["hot_experts"]
+        sample = [hot[0], next(e for e in range(L.E) if e not in hot), L.E - 1]
+    else:
+        sample = [0, L.E - 1]
+    want = hp.oracle_pack(L, sample)
+    got_hdr = layer.packed[:orc.HDR_BYTES].cpu().numpy()
+    # header: identical except tensor scales of experts the oracle did not pack
+    ts_g = got_hdr[13088:13088 + 3072].view(np.float32).copy()
+    ts_w = want[13088:13088 + 3072].view(np.float32).copy()
+    for e in range(L.E):
+        if e not in sample:
+            ts_g[3 * e:3 * e + 3] = 0
+    np.testing.assert_array_equal(ts_g, ts_w)
+    gh = got_hdr.copy()
+    gh[13088:13088 + 3072] = 0
+    wh = want[:orc.HDR_BYTES].copy()
+    wh[13088:13088 + 3072] = 0
+    np.testing.assert_array_equal(gh, wh)
+    for e in sample:
+        for off, n in hp.sections(L, e):
+            np.testing.assert_array_equal(layer.packed[off:off + n].cpu().numpy(), want[off:off + n],
+                                          err_msg=f"{name} expert {e} section @{off}")
+
+
+# ------------------------------------------------------------------ forward, small shapes
+def test_forward_tiny_layer():
+    r = check_layer(W.layer("tiny"), 16)
+    assert r["ties"] == 0
+
+
+def test_forward_ragged_mixed_formats():
+    # several 128-row tiles, a ragged token count, every integer format
+    L = custom("ragged", 37, 384, 640, 12, 3,
+               [[3, 2, 4], [4, 4, 4], [2, 2, 2], [4, 4, 2], [3, 3, 3], [2, 4, 3]] * 2)
+    check_layer(L, 37)
+
+
+def test_forward_prefill_chunks_and_tails():
+    # more than 16 rows per expert: 64-row chunks, several per expert, ragged tails
+    L = custom("chunks", 300, 256, 384, 4, 2, [[4, 4, 4], [3, 2, 4], [2, 2, 2], [4, 3, 2]])
+    check_layer(L, 300)
+
+
+def test_forward_nvfp4_small():
+    L = custom("fp4small", 23, 256, 384, 16, 6, [[16, 16, 16]] * 16)
+    check_layer(L, 23)
+
+
+def test_forward_nvfp4_prefill_chunks():
+    L = custom("fp4chunks", 200, 256, 256, 8, 2, [[16, 16, 16]] * 8)
+    check_layer(L, 200)
+
+
+def test_nvfp4_down_stage_refeed():
+    # feed the GPU's e4m3 codes of h into the oracle's down stage: output parity of the
+    # down GEMM + combine alone (h codes depend on summation order and are not required
+    # to match bit for bit).
+    L = custom("fp4refeed", 9, 256, 256, 8, 2, [[16, 16, 16]] * 8)
+    T, k = 9, 2
+    layer = hp.gpu_pack(L)
+    g = run_gpu(L, layer, T)
+    x_bits = W.x_bf16_bits(T, L.H)
+    buf = hp.oracle_pack(L, range(L.E))
+    idx = g["topk_idx"].reshape(T, k)
+    counts, offsets, perm, inv = orc.permute(idx.astype(np.int32), L.E)
+    hq = g["hq"].reshape(T * k, L.F)
+    sh = g["sh"]
+    o = np.zeros((T * k, L.H))
+    for e in range(L.E):
+        r0, r1 = offsets[e], offsets[e + 1]
+        if r1 > r0:
+            o[r0:r1] = orc.down(buf, e, orc.e4m3_table()[hq[r0:r1]], sh[r0:r1].astype(np.float64))
+    y_ref = np.zeros((T, L.H))
+    w = g["topk_w"].reshape(T, k)
+    for t in range(T):
+        for j in range(k):
+            y_ref[t] += float(w[t, j]) * o[inv[t * k + j]]
+    hp.check_output(g["y"], y_ref)
+    # and the h codes themselves: count disagreements with the oracle's own h codes
+    a = orc.e4m3_table()[orc.act_quant_e4m3(gen.bf16_bits_to_f32(x_bits))[0]]
+    sx = orc.act_quant_e4m3(gen.bf16_bits_to_f32(x_bits))[1]
+    n_diff = 0
+    for e in range(L.E):
+        r0, r1 = offsets[e], offsets[e + 1]
+        if r1 > r0:
+            ts = perm[r0:r1] // k
+            h = orc.gateup(buf, e, a[ts], sx[ts].astype(np.float64))
+            hq_o, _ = orc.act_quant_e4m3(h.astype(np.float32))
+            n_diff += int(np.count_nonzero(hq_o != hq[r0:r1]))
+    assert n_diff <= 0.01 * hq.size, f"{n_diff} of {hq.size} h codes differ"
+
+
+def test_forward_single_token():
+    L = custom("one", 1, 256, 256, 8, 2, [[4, 2, 3]] * 8)
+    check_layer(L, 1)
+
+
+def test_forward_all_tokens_one_expert():
+    # bias sends every token to expert 3 (k = 1): one expert, 200 rows, 4 chunks
+    L = custom("onehot", 200, 256, 256, 8, 1, [[4, 4, 4]] * 8)
+    b = np.zeros(8, np.float32)
+    b[3] = 100.0
+    r = check_layer(L, 200, bias=b)
+    assert r["counts"][3] == 200 and r["counts"].sum() == 200
+
+
+def test_forward_k_equals_E_equal_logits_is_mean():
+    L = custom("mean", 5, 256, 256, 8, 8, [[4, 3, 2]] * 8)
+    r = check_layer(L, 5, bias=np.zeros(8, np.float32), router_zero=True)
+    assert np.all(r["counts"] == 5)
+
+
+def test_forward_zero_expert():
+    L = custom("zero", 12, 256, 256, 4, 2, [[4, 4, 4]] * 4)
+    layer = hp.gpu_pack(L)
+    # overwrite expert 1 with zero weights through the ABI
+    zeros = torch.zeros((1, 3, L.H * L.F), dtype=torch.float32, device="cuda")
+    moe.moe_pack(zeros, 1, L.E, L.H, L.F, L.fmt.reshape(-1), layer.packed)
+    b = np.array([0, 50, 49, -50], np.float32)  # every token -> experts {1, 2}
+    Wr = torch.zeros((L.E, L.H), dtype=torch.float32, device="cuda")
+    g = run_gpu(L, layer, 12, Wr=Wr, b=torch.from_numpy(b).cuda())
+    assert np.all(np.sort(g["topk_idx"].reshape(12, 2), 1) == [1, 2])
+    Wh = np.stack([W.expert_w(e, L.H, L.F) for e in range(L.E)])
+    Wh[1] = 0
+    buf = orc.pack_layer(Wh, 0, L.E, L.H, L.F, L.fmt.reshape(-1))
+    y_ref, _, _ = hp.oracle_forward_rows(buf, W.x_bf16_bits(12, L.H), np.zeros((L.E, L.H), np.float32), b, 2)
+    hp.check_output(g["y"], y_ref)
+
+
+def test_forward_deterministic_and_empty_batch():
+    L = W.layer("tiny")
+    layer = hp.gpu_pack(L)
+    x = W.device_x(40, L.H)
+    Wr, b = W.device_router(L)
+    y1 = moe.moe_layer_forward(x, Wr, b, layer, L.k)
+    y2 = moe.moe_layer_forward(x, Wr, b, layer, L.k)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    y0 = moe.moe_layer_forward(x[:0], Wr, b, layer, L.k)
+    assert y0.shape == (0, L.H)
+
+
+def test_stage_events_record():
+    L = W.layer("tiny")
+    layer = hp.gpu_pack(L)
+    x = W.device_x(16, L.H)
+    Wr, b = W.device_router(L)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_STAGE_EVENTS)]
+    for e in ev:
+        e.record()
+    moe.moe_layer_forward(x, Wr, b, layer, L.k, stage_events=ev)
+    torch.cuda.synchronize()
+    times = [ev[i].elapsed_time(ev[i + 1]) for i in range(len(ev) - 1)]
+    assert all(t >= 0 for t in times) and ev[0].elapsed_time(ev[-1]) > 0
+
+
+# ------------------------------------------------------------------ forward, the five layers
+CONFIG_RUNS = [
+    ("mixtral", 1, None), ("mixtral", 8, None), ("mixtral", 64, None),
+    ("hotcold", 32, None), ("nvfp4", 16, None), ("large", 64, [0, 1, 2, 63]),
+    ("mixtral", 2048, [0, 1, 1000, 2047]), ("hotcold", 4096, [0, 4095]),
+    ("nvfp4", 8192, [0, 8191]), ("large", 8192, [0, 8191]),
+]
+
+
+@pytest.mark.parametrize("name,T,tokens", CONFIG_RUNS, ids=[f"{n}-T{t}" for n, t, _ in CONFIG_RUNS])
+def test_forward_config(name, T, tokens):
+    L = W.layer(name)
+    r = check_layer(L, T, tokens=tokens)
+    print(f"{name} T={T}: near-ties {r['ties']}, err/max {r['err_ratio']:.3g}")
