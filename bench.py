@@ -295,28 +295,53 @@ def run_ours(args, rank, world, local_rank):
 
 
 # ------------------------------------------------------------------ oracle (CPU) timing
-def oracle_time(L: W.Layer, T_full: int, budget_s: float, x_seed: int = 0):
-    """Time the oracle forward on a growing sample of the batch until it takes
-    `budget_s` seconds; returns (tokens/s, sample description, threads)."""
-    import oracle as orc
-    Wr = W.router_w(L.E, L.H)
-    x_all = W.x_bf16_bits(T_full, L.H, seed=x_seed)
-    n = 2
-    buf = None
-    packed_experts = set()
-    while True:
-        xs = np.ascontiguousarray(x_all[:n])
-        idx = orc.topk_softmax(orc.router(xs, Wr, L.bias), L.k)[0]
-        need = set(np.unique(idx).tolist()) - packed_experts
-        for e in sorted(need):
-            buf = orc.pack_layer(W.expert_w(e, L.H, L.F)[None], e, L.E, L.H, L.F, L.fmt.reshape(-1), out=buf)
-        packed_experts |= need
+class OracleSample:
+    """The CPU oracle on a bounded sample (the first n tokens) of a batch."""
+
+    def __init__(self, L: W.Layer, T_full: int, x_seed: int = 0):
+        import oracle as orc
+        self.orc, self.L, self.T_full = orc, L, T_full
+        self.Wr = W.router_w(L.E, L.H)
+        self.x_all = W.x_bf16_bits(T_full, L.H, seed=x_seed)
+        self.buf = None
+        self.packed = set()
+
+    def _prepare(self, n: int):
+        orc, L = self.orc, self.L
+        xs = np.ascontiguousarray(self.x_all[:n])
+        idx = orc.topk_softmax(orc.router(xs, self.Wr, L.bias), L.k)[0]
+        for e in sorted(set(np.unique(idx).tolist()) - self.packed):   # oracle packing, untimed
+            self.buf = orc.pack_layer(W.expert_w(e, L.H, L.F)[None], e, L.E, L.H, L.F, L.fmt.reshape(-1),
+                                      out=self.buf)
+            self.packed.add(e)
+        return xs
+
+    def step(self, n: int) -> float:
+        """Seconds for one oracle forward over the first n tokens."""
+        xs = self._prepare(n)
         t0 = time.perf_counter()
-        orc.moe_forward(buf, xs, Wr, L.bias, L.k)
-        dt = time.perf_counter() - t0
-        if dt >= budget_s or n >= T_full:
-            return n / dt, f"first {n} of {T_full} tokens (oracle packing excluded)", orc.num_threads()
-        n = min(T_full, n * 2 if dt < budget_s / 4 else int(n * budget_s / dt) + 1)
+        self.orc.moe_forward(self.buf, xs, self.Wr, self.L.bias, self.L.k)
+        return time.perf_counter() - t0
+
+    def calibrate(self, budget_s: float) -> int:
+        """Smallest doubling of n whose forward takes about budget_s (capped at the batch)."""
+        n = 2
+        while True:
+            dt = self.step(n)
+            if dt >= budget_s or n >= self.T_full:
+                return n
+            n = min(self.T_full, max(n + 1, int(n * min(4.0, 0.9 * budget_s / dt))))
+
+    def describe(self, n: int) -> str:
+        return f"first {n} of {self.T_full} tokens of the same batch (oracle packing untimed)"
+
+
+def oracle_time(L: W.Layer, T_full: int, budget_s: float, x_seed: int = 0):
+    """(tokens/s, sample description, threads) of the oracle on a sample taking ~budget_s."""
+    s = OracleSample(L, T_full, x_seed)
+    n = s.calibrate(budget_s)
+    dt = s.step(n)
+    return n / dt, s.describe(n), s.orc.num_threads()
 
 
 def run_reference(args, rank, world):
@@ -324,20 +349,20 @@ def run_reference(args, rank, world):
         return None
     L = W.layer("mixtral")
     T = 2048
-    per_step_budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
-    vals = []
-    for i in range(args.warmup + args.steps):
-        v, sample, cores = oracle_time(L, T, per_step_budget)
-        if i >= args.warmup:
-            vals.append(v)
-    value = float(np.mean(vals))
+    s = OracleSample(L, T)
+    n = s.calibrate(max(2.0, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        s.step(n)
+    times = [s.step(n) for _ in range(args.steps)]
+    value = n * args.steps / sum(times)
     return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(1e3 * T / value, 1), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload_desc(L, T, "prefill"), "parallelism": "CPU oracle"},
-            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                             "sample": sample},
+            "ms_per_step": round(1e3 * sum(times) / args.steps, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(L, T, "prefill"), "parallelism": "CPU oracle",
+                       "step": f"one oracle forward over the {s.describe(n)}"},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": s.orc.num_threads(),
+                             "kind": "oracle", "sample": s.describe(n)},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 

@@ -52,10 +52,12 @@ int grid_for(uint64_t count) {
 
 }  // namespace
 
+#define MOEGEN_API __attribute__((visibility("default")))
+
 extern "C" {
 
 // Fill out[0..count) with fp32 values of elements [start, start+count) of tensor tid.
-int moegen_fill_f32(float* out, uint64_t seed, uint64_t tid, uint64_t start, uint64_t count,
+MOEGEN_API int moegen_fill_f32(float* out, uint64_t seed, uint64_t tid, uint64_t start, uint64_t count,
                     float sigma, cudaStream_t stream) {
   if (count == 0) return 0;
   fill_f32_kernel<<<grid_for(count), 256, 0, stream>>>(out, seed, tid, start, count, sigma);
@@ -63,7 +65,7 @@ int moegen_fill_f32(float* out, uint64_t seed, uint64_t tid, uint64_t start, uin
 }
 
 // Same as moegen_fill_f32, rounded to bf16 (round-to-nearest-even).
-int moegen_fill_bf16(void* out, uint64_t seed, uint64_t tid, uint64_t start, uint64_t count,
+MOEGEN_API int moegen_fill_bf16(void* out, uint64_t seed, uint64_t tid, uint64_t start, uint64_t count,
                      float sigma, cudaStream_t stream) {
   if (count == 0) return 0;
   fill_bf16_kernel<<<grid_for(count), 256, 0, stream>>>((__nv_bfloat16*)out, seed, tid, start,

@@ -105,10 +105,16 @@ enum {
  * major, input-block minor.  Inside a tile, u32 words ordered
  * [kg 0..3][word 0..b-1][n 0..127] (kg = group of 32 inputs inside the tile,
  * b = 2, 3, 4 words per group; NVFP4 uses 4).  Stored integer code u = q+2^(b-1).
- *   4-bit / NVFP4: code i of a group in word i/8, bits 4*(i%8)..+3
- *   2-bit: code i in word i/16, bits 2*(i%16)..+1
- *   3-bit: words 0-1 hold the low two bits of u as for 2-bit; bit i of word 2
- *          holds bit 2 of u of code i.
+ * Inside an integer word the two codes of each pair (2j, 2j+1) sit 16 bits
+ * apart (even code in the low half-word), so one mask of a shifted word
+ * yields both:
+ *   4-bit: codes 8w..8w+7 in word w; code 8w+2j at bits 4j..4j+3, code
+ *          8w+2j+1 at bits 16+4j..16+4j+3 (j = 0..3)
+ *   2-bit: codes 16w..16w+15 in word w; code 16w+2j at bits 2j..2j+1, code
+ *          16w+2j+1 at bits 16+2j..17+2j (j = 0..7)
+ *   3-bit: words 0-1 hold the low two bits of u as for 2-bit; word 2 holds
+ *          bit 2 of u: code 2j at bit j, code 2j+1 at bit 16+j (j = 0..15)
+ *   NVFP4: codes 8w..8w+7 in word w, code 8w+i at bits 4i..4i+3.
  * Scale layout: [N/128][K/gs][128] (gs = 32 integer, 16 NVFP4).
  */
 

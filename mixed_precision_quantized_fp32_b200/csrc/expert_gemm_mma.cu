@@ -97,14 +97,15 @@ __device__ __forceinline__ float code_value(const Frag& f, int fmt, int gi, int 
     return e2m1_value(c) * e4m3_value(sb);  // exact (<= 6 significant bits)
   }
   const float s = __half2float(__ushort_as_half((uint16_t)(f.sc >> (16 * gi))));
+  // code i of a pair-interleaved word: pair i/2 at the low (even i) or high (odd i) half-word
   int q;
   if (fmt == MOE_FMT_INT4) {
-    q = (int)((f.w[gi][i >> 3] >> (4 * (i & 7))) & 15u) - 8;
+    q = (int)((f.w[gi][i >> 3] >> ((i & 1) * 16 + ((i & 7) >> 1) * 4)) & 15u) - 8;
   } else if (fmt == MOE_FMT_INT2) {
-    q = (int)((f.w[gi][i >> 4] >> (2 * (i & 15))) & 3u) - 2;
+    q = (int)((f.w[gi][i >> 4] >> ((i & 1) * 16 + ((i & 15) >> 1) * 2)) & 3u) - 2;
   } else {
-    const uint32_t lo = (f.w[gi][i >> 4] >> (2 * (i & 15))) & 3u;
-    const uint32_t hi = (f.w[gi][2] >> i) & 1u;
+    const uint32_t lo = (f.w[gi][i >> 4] >> ((i & 1) * 16 + ((i & 15) >> 1) * 2)) & 3u;
+    const uint32_t hi = (f.w[gi][2] >> ((i & 1) * 16 + (i >> 1))) & 1u;
     q = (int)(lo | (hi << 2)) - 4;
   }
   return s * (float)q;  // exact in fp32; rounded once to the 16-bit operand type

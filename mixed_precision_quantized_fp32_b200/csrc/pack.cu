@@ -103,35 +103,32 @@ __global__ void pack_int_kernel(const float* __restrict__ W, int N, int K, uint3
     }
     u[i] = (uint32_t)(q + OFF);
   }
+  // Inside a word, the two codes of a pair (2j, 2j+1) sit 16 bits apart, so a
+  // mask of the shifted word yields both as the low bits of two half-words.
   const int k0 = g * 32;
   if (BITS == 4) {
 #pragma unroll
     for (int wd = 0; wd < 4; ++wd) {
       uint32_t v = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v |= u[wd * 8 + i] << (4 * i);
+      for (int j = 0; j < 4; ++j) v |= (u[wd * 8 + 2 * j] << (4 * j)) | (u[wd * 8 + 2 * j + 1] << (16 + 4 * j));
       codes[word_index(n, k0, K, 4, wd)] = v;
     }
-  } else if (BITS == 2) {
-#pragma unroll
-    for (int wd = 0; wd < 2; ++wd) {
-      uint32_t v = 0;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) v |= u[wd * 16 + i] << (2 * i);
-      codes[word_index(n, k0, K, 2, wd)] = v;
-    }
   } else {
-    uint32_t hi = 0;
 #pragma unroll
     for (int wd = 0; wd < 2; ++wd) {
       uint32_t v = 0;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v |= (u[wd * 16 + i] & 3u) << (2 * i);
-      codes[word_index(n, k0, K, 3, wd)] = v;
+      for (int j = 0; j < 8; ++j)
+        v |= ((u[wd * 16 + 2 * j] & 3u) << (2 * j)) | ((u[wd * 16 + 2 * j + 1] & 3u) << (16 + 2 * j));
+      codes[word_index(n, k0, K, BITS, wd)] = v;
     }
+    if (BITS == 3) {
+      uint32_t hi = 0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) hi |= ((u[i] >> 2) & 1u) << i;
-    codes[word_index(n, k0, K, 3, 2)] = hi;
+      for (int j = 0; j < 16; ++j) hi |= (((u[2 * j] >> 2) & 1u) << j) | (((u[2 * j + 1] >> 2) & 1u) << (16 + j));
+      codes[word_index(n, k0, K, 3, 2)] = hi;
+    }
   }
   scales[scale_index(n, g, G)] = sbits;
 }

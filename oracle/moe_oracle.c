@@ -230,10 +230,15 @@ ORC_EXPORT void orc_quant_nvfp4(const float* W, int N, int K, uint8_t* v, uint8_
 /* in the order [kg 0..3][word 0..b-1][n 0..127], where kg is the group of 32 */
 /* inputs inside the tile and b the word count of a group (2, 3, 4; NVFP4 4).*/
 /* Stored code u = q + 2^(b-1) (offset binary); NVFP4 stores the e2m1 code.   */
-/*   b = 4: code i of the group in word i/8, bits 4*(i%8)..                  */
-/*   b = 2: code i in word i/16, bits 2*(i%16)..                             */
-/*   b = 3: words 0-1 hold the low two bits of u exactly as b = 2; bit i of  */
-/*          word 2 holds bit 2 of u for code i.                              */
+/* Inside a word, the two codes of each consecutive pair (2j, 2j+1) sit 16    */
+/* bits apart (code 2j in the low half-word, code 2j+1 in the high one):      */
+/*   b = 4: codes 8w..8w+7 in word w; code 8w+2j at bits 4j..4j+3, code      */
+/*          8w+2j+1 at bits 16+4j..16+4j+3 (j = 0..3);                       */
+/*   b = 2: codes 16w..16w+15 in word w; code 16w+2j at bits 2j..2j+1, code  */
+/*          16w+2j+1 at bits 16+2j..17+2j (j = 0..7);                        */
+/*   b = 3: words 0-1 hold the low two bits of u exactly as b = 2; word 2     */
+/*          holds bit 2 of u: code 2j at bit j, code 2j+1 at bit 16+j.        */
+/*   NVFP4: codes 8w..8w+7 in word w, code 8w+i at bits 4i..4i+3.            */
 /* Scales: fp16 (int) or e4m3 bytes (NVFP4) in [N/128][K/gs][128] order,      */
 /* gs = 32 (int) or 16 (NVFP4).                                               */
 /* ------------------------------------------------------------------------- */
@@ -243,26 +248,34 @@ static size_t word_index(int n, int k, int K, int wpg, int w) {
   return (((nb * (size_t)(K / 128) + kb) * 4 + kg) * (size_t)wpg + (size_t)w) * 128 + (size_t)(n % 128);
 }
 
+/* bit offset of code i (0..31 of its group) inside its word, integer formats */
+static int pair_shift(int i, int width, int per_word) {
+  int c = i % per_word; /* position inside the word's run of codes */
+  return (c % 2) * 16 + (c / 2) * width;
+}
+
 /* code (already offset / e2m1, 0..15) of element (n, k) is placed into words */
 static void put_code(uint32_t* words, int n, int k, int K, int fmt, uint32_t u) {
   int i = k % 32;
-  if (fmt == ORC_INT4 || fmt == ORC_NVFP4) {
+  if (fmt == ORC_NVFP4) {
     words[word_index(n, k, K, 4, i / 8)] |= (u & 15u) << (4 * (i % 8));
+  } else if (fmt == ORC_INT4) {
+    words[word_index(n, k, K, 4, i / 8)] |= (u & 15u) << pair_shift(i, 4, 8);
   } else if (fmt == ORC_INT2) {
-    words[word_index(n, k, K, 2, i / 16)] |= (u & 3u) << (2 * (i % 16));
+    words[word_index(n, k, K, 2, i / 16)] |= (u & 3u) << pair_shift(i, 2, 16);
   } else { /* INT3 */
-    words[word_index(n, k, K, 3, i / 16)] |= (u & 3u) << (2 * (i % 16));
-    words[word_index(n, k, K, 3, 2)] |= ((u >> 2) & 1u) << i;
+    words[word_index(n, k, K, 3, i / 16)] |= (u & 3u) << pair_shift(i, 2, 16);
+    words[word_index(n, k, K, 3, 2)] |= ((u >> 2) & 1u) << pair_shift(i, 1, 32);
   }
 }
 
 static uint32_t get_code(const uint32_t* words, int n, int k, int K, int fmt) {
   int i = k % 32;
-  if (fmt == ORC_INT4 || fmt == ORC_NVFP4)
-    return (words[word_index(n, k, K, 4, i / 8)] >> (4 * (i % 8))) & 15u;
-  if (fmt == ORC_INT2) return (words[word_index(n, k, K, 2, i / 16)] >> (2 * (i % 16))) & 3u;
-  uint32_t lo = (words[word_index(n, k, K, 3, i / 16)] >> (2 * (i % 16))) & 3u;
-  uint32_t hi = (words[word_index(n, k, K, 3, 2)] >> i) & 1u;
+  if (fmt == ORC_NVFP4) return (words[word_index(n, k, K, 4, i / 8)] >> (4 * (i % 8))) & 15u;
+  if (fmt == ORC_INT4) return (words[word_index(n, k, K, 4, i / 8)] >> pair_shift(i, 4, 8)) & 15u;
+  if (fmt == ORC_INT2) return (words[word_index(n, k, K, 2, i / 16)] >> pair_shift(i, 2, 16)) & 3u;
+  uint32_t lo = (words[word_index(n, k, K, 3, i / 16)] >> pair_shift(i, 2, 16)) & 3u;
+  uint32_t hi = (words[word_index(n, k, K, 3, 2)] >> pair_shift(i, 1, 32)) & 1u;
   return lo | (hi << 2);
 }
 

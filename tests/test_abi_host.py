@@ -121,3 +121,14 @@ def test_valid_call_without_gpu_fails_cleanly():
         pytest.skip("a GPU is present")
     st, _ = _fwd(16, 2)
     assert st in ("MOE_ERR_CUDA", "MOE_ERR_UNSUPPORTED_DEVICE")
+
+
+def test_generator_libraries_load_and_export():
+    import ctypes
+    import gen
+    from gen import workloads
+    L = workloads._dev_lib()
+    for name in ("moegen_fill_f32", "moegen_fill_bf16"):
+        assert hasattr(L, name)
+    assert hasattr(gen._host_lib(), "moegen_host_fill_f32")
+    assert isinstance(L, ctypes.CDLL)
