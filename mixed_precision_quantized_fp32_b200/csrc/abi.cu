@@ -43,14 +43,18 @@ int layer_kind(int E, const uint8_t* fmt) {
 }
 
 struct Plan {
-  int chunk_rows;
-  int max_chunks;
+  int chunk_rows;  // rows per work chunk of one expert
+  int max_chunks;  // upper bound on the number of chunks
+  bool tc;         // tcgen05 expert GEMMs (many rows per expert) or warp-MMA (few rows per expert)
 };
 
+// Few rows per expert (decode): 16-row chunks on the warp-level MMA kernel.
+// Many rows per expert (prefill): 256-row chunks on the tcgen05 kernel.
 Plan make_plan(int T, int k, int E) {
   Plan p;
   const long long R = (long long)T * k;
-  p.chunk_rows = (R <= 16LL * E) ? 16 : 64;
+  p.tc = R > 16LL * E && R >= 256;
+  p.chunk_rows = p.tc ? 256 : 16;
   p.max_chunks = (int)(E + (R + p.chunk_rows - 1) / p.chunk_rows);
   return p;
 }
@@ -170,15 +174,17 @@ extern "C" moe_status moe_layer_forward(const void* x, int32_t T, const float* r
   if (!mark(2)) return MOE_ERR_CUDA;
   if (launch_gather(xb, T, H, k, fp4, wsp, d.xq, d.sx, stream) != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(3)) return MOE_ERR_CUDA;
-  if (launch_expert_gemm_mma(packed, E, H, F, k, fp4, true, plan.chunk_rows, plan.max_chunks, wsp, stream) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
+  int32_t* status = d.status ? d.status : wsp.status;
+  auto gemm = [&](bool gateup) -> cudaError_t {
+    return plan.tc ? launch_expert_gemm_tc(packed, E, H, F, T, k, fp4, gateup, wsp, status, stream)
+                   : launch_expert_gemm_mma(packed, E, H, F, k, fp4, gateup, plan.chunk_rows, plan.max_chunks, wsp,
+                                            stream);
+  };
+  if (gemm(true) != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(4)) return MOE_ERR_CUDA;
   if (fp4 && launch_act_quant_h(T * k, F, wsp, d.hq, d.sh, stream) != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(5)) return MOE_ERR_CUDA;
-  if (launch_expert_gemm_mma(packed, E, H, F, k, fp4, false, plan.chunk_rows, plan.max_chunks, wsp, stream) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
+  if (gemm(false) != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(6)) return MOE_ERR_CUDA;
   if (launch_combine(T, k, H, wsp, (__nv_bfloat16*)y, stream) != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(7)) return MOE_ERR_CUDA;

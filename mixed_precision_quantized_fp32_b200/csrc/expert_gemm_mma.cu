@@ -33,18 +33,6 @@ struct MmaType<__half> {
   }
   __device__ static __forceinline__ __half from_float(float v) { return __float2half_rn(v); }
 };
-template <>
-struct MmaType<__nv_bfloat16> {
-  __device__ static __forceinline__ void mma(float* d, const uint32_t* a, const uint32_t* b) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};\n"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-  }
-  __device__ static __forceinline__ __nv_bfloat16 from_float(float v) { return __float2bfloat16_rn(v); }
-};
-
 __device__ __forceinline__ void ldsm_x4(uint32_t* r, const void* p) {
   const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
@@ -94,7 +82,7 @@ __device__ __forceinline__ float code_value(const Frag& f, int fmt, int gi, int 
   if (fmt == MOE_FMT_NVFP4) {
     const uint32_t c = (f.w[gi][i >> 3] >> (4 * (i & 7))) & 15u;
     const uint32_t sb = (f.sc >> (8 * (2 * gi + (i >> 4)))) & 255u;
-    return e2m1_value(c) * e4m3_value(sb);  // exact (<= 6 significant bits)
+    return e2m1_value(c) * e4m3_value(sb);  // exact in fp16 (<= 6 significant bits, within range)
   }
   const float s = __half2float(__ushort_as_half((uint16_t)(f.sc >> (16 * gi))));
   // code i of a pair-interleaved word: pair i/2 at the low (even i) or high (odd i) half-word
@@ -313,8 +301,6 @@ cudaError_t launch_expert_gemm_mma(const uint8_t* packed, int E, int H, int F, i
     g.act = ws.xs;
     g.row_scale = fp4 ? ws.sx : nullptr;
     g.out = ws.h;
-    if (fp4) return chunk_rows == 16 ? launch_one<__nv_bfloat16, 16, true>(g, max_chunks, stream)
-                                     : launch_one<__nv_bfloat16, 64, true>(g, max_chunks, stream);
     return chunk_rows == 16 ? launch_one<__half, 16, true>(g, max_chunks, stream)
                             : launch_one<__half, 64, true>(g, max_chunks, stream);
   }
@@ -325,8 +311,6 @@ cudaError_t launch_expert_gemm_mma(const uint8_t* packed, int E, int H, int F, i
   g.act = fp4 ? ws.hb : ws.h;
   g.row_scale = fp4 ? ws.sh : nullptr;
   g.out = ws.o;
-  if (fp4) return chunk_rows == 16 ? launch_one<__nv_bfloat16, 16, false>(g, max_chunks, stream)
-                                   : launch_one<__nv_bfloat16, 64, false>(g, max_chunks, stream);
   return chunk_rows == 16 ? launch_one<__half, 16, false>(g, max_chunks, stream)
                           : launch_one<__half, 64, false>(g, max_chunks, stream);
 }

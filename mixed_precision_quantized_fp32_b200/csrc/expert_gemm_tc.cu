@@ -1,0 +1,470 @@
+// Dequant-fused grouped expert GEMM on the 5th-generation tensor cores
+// (tcgen05.mma kind::f16, fp32 accumulators in TMEM) for batches with many
+// token rows per expert (prefill).
+//
+// This is the pages' "packed linear" operator (MoE mixed-precision page,
+// sec. 2.3 / 3.5: experts stored as independently quantized 128-column blocks
+// that a custom kernel unpacks) with the activation fused into the epilogue
+// (its sec. 3.6, "fused linear + activation"), built for sm_100a:
+//   * one persistent CTA per SM walks (token chunk, 128-row weight tile) work
+//     items; chunk = up to 256 consecutive expert-sorted rows of one expert;
+//   * warp 8 (one lane) streams each 64-input stage: the activation tile with a
+//     2D TMA load (128-byte swizzle) and the packed codes + scales of the weight
+//     tile with 1D bulk copies (both never multicast);
+//   * warps 0-7 turn codes into fp16 operands (exponent-bias unpack: a code u
+//     OR'ed into the mantissa of 1024.0 gives 1024+u exactly; one subtract
+//     and one multiply by the group scale) written straight into the 128-byte
+//     swizzled K-major layout the tensor core reads;
+//   * warp 9 (one lane) issues tcgen05.mma M=128 (weight rows) x N<=256 (token
+//     rows) x K=16 and commits to mbarriers;
+//   * warps 0-7 then drain TMEM (tcgen05.ld) into the SwiGLU / scale epilogue.
+// Every mbarrier wait is bounded; a wait that gives up raises an abort flag so
+// every role leaves its loop, writes MOE_ERR_TIMEOUT to the status word and
+// the CTA frees its TMEM before returning.
+#include <cudaTypedefs.h>
+
+#include "moe_common.cuh"
+#include "kernels.cuh"
+#include "tc_ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kTcBM = 128;   // weight rows per work item (MMA M)
+constexpr int kTcBN = 256;   // token rows per work item (max MMA N)
+constexpr int kTcBK = 64;    // inputs per pipeline stage (one 128-byte swizzle row of fp16)
+constexpr int kTcThreads = 320;
+constexpr int kTmaWarp = 8, kMmaWarp = 9;
+constexpr int kDeqThreads = 256;
+constexpr long long kWaitLimit = 4000000000LL;  // clock cycles, ~2 s
+
+template <int NMAT>
+struct TcCfg {
+  static constexpr int kStages = NMAT == 2 ? 3 : 4;
+  static constexpr int kBBytes = kTcBN * kTcBK * 2;
+  static constexpr int kABytes = kTcBM * kTcBK * 2;
+  static constexpr int kCodeBytes = 4096;  // <= 4 words x 2 groups x 128 rows x 4 bytes
+  static constexpr int kScaleBytes = 512;  // 2 fp16 groups or 4 e4m3 blocks x 128 rows
+  static constexpr int kOffB = 0;
+  static constexpr int kOffA = kBBytes;
+  static constexpr int kOffCodes = kOffA + NMAT * kABytes;
+  static constexpr int kOffScales = kOffCodes + NMAT * kCodeBytes;
+  static constexpr int kStageBytes = (kOffScales + NMAT * kScaleBytes + 1023) / 1024 * 1024;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmem = kStages * kStageBytes + kBarBytes + 1024;
+};
+static_assert(TcCfg<2>::kSmem <= 232448, "gate/up stages exceed shared memory");
+static_assert(TcCfg<1>::kSmem <= 232448, "down stages exceed shared memory");
+
+struct TcArgs {
+  const uint8_t* packed;
+  int E, H, F;
+  int N, K;                // output rows (weight rows) and inputs of this GEMM
+  int proj;                // 0: gate+up with SwiGLU epilogue; 2: down
+  const int32_t* chunks;   // (expert, first row, rows) triples
+  const int32_t* chunk_count;
+  const float* row_scale;  // NVFP4: gate/up -> per-token sx, down -> per-row sh; null for integer layers
+  const int32_t* perm;
+  int topk;
+  void* out;               // gate/up: h [rows][F] (fp16, or fp32 for NVFP4); down: o fp32 [rows][H]
+  int32_t* status;
+};
+
+__device__ __forceinline__ uint32_t h2sub(uint32_t a, uint32_t b) {
+  __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t h2mul(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// Four e2m1 pairs (one 32-bit word, byte b = codes 2b, 2b+1) -> four fp16 pairs.
+__device__ __forceinline__ void e2m1x8_to_f16(uint32_t w, uint32_t* o) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+      : "r"(w));
+}
+
+// Dequantize group gi (32 inputs) of weight row n of one matrix from the staged
+// codes/scales into four 16-byte chunks (8 inputs each) of the swizzled A tile.
+__device__ __forceinline__ void dequant_group(int fmt, const uint32_t* __restrict__ codes,
+                                              const uint8_t* __restrict__ scales, int n, int gi, uint8_t* A) {
+  uint32_t v[16];  // 16 fp16 pairs = 32 inputs in natural order
+  if (fmt == MOE_FMT_NVFP4) {
+    const float s0 = e4m3_value(scales[(2 * gi) * 128 + n]);
+    const float s1 = e4m3_value(scales[(2 * gi + 1) * 128 + n]);
+    const __half2 h0 = __float2half2_rn(s0), h1 = __float2half2_rn(s1);
+    const uint32_t p0 = *reinterpret_cast<const uint32_t*>(&h0), p1 = *reinterpret_cast<const uint32_t*>(&h1);
+#pragma unroll
+    for (int wd = 0; wd < 4; ++wd) {
+      uint32_t o[4];
+      e2m1x8_to_f16(codes[(gi * 4 + wd) * 128 + n], o);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) v[wd * 4 + b] = h2mul(o[b], wd < 2 ? p0 : p1);  // exact
+    }
+  } else {
+    const uint32_t s = reinterpret_cast<const uint16_t*>(scales)[gi * 128 + n];
+    const uint32_t s2 = s | (s << 16);
+    if (fmt == MOE_FMT_INT4) {
+#pragma unroll
+      for (int wd = 0; wd < 4; ++wd) {
+        const uint32_t w = codes[(gi * 4 + wd) * 128 + n];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          v[wd * 4 + j] = h2mul(h2sub(((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u, 0x64086408u), s2);
+      }
+    } else if (fmt == MOE_FMT_INT2) {
+#pragma unroll
+      for (int wd = 0; wd < 2; ++wd) {
+        const uint32_t w = codes[(gi * 2 + wd) * 128 + n];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          v[wd * 8 + j] = h2mul(h2sub(((w >> (2 * j)) & 0x00030003u) | 0x64006400u, 0x64026402u), s2);
+      }
+    } else {  // INT3
+      const uint32_t hi = codes[(gi * 3 + 2) * 128 + n];
+#pragma unroll
+      for (int wd = 0; wd < 2; ++wd) {
+        const uint32_t lo = codes[(gi * 3 + wd) * 128 + n];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t u = ((lo >> (2 * j)) & 0x00030003u) | (((hi >> (8 * wd + j)) & 0x00010001u) << 2);
+          v[wd * 8 + j] = h2mul(h2sub(u | 0x64006400u, 0x64046404u), s2);
+        }
+      }
+    }
+  }
+  uint8_t* row = A + (n >> 3) * 1024 + (n & 7) * 128;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int chunk = (4 * gi + c) ^ (n & 7);
+    *reinterpret_cast<uint4*>(row + chunk * 16) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  }
+}
+
+__device__ __forceinline__ uint64_t code_stage_offset(int mt, int ks, int K, int wpg) {
+  // bytes of words [kg = 2*(ks%2) .. +1][word][n] of tile (mt, ks/2); contiguous wpg*1024 bytes
+  return ((((uint64_t)mt * (uint64_t)(K >> 7) + (uint64_t)(ks >> 1)) * 4u + (uint64_t)(ks & 1) * 2u) *
+          (uint64_t)wpg * 128u) * 4u;
+}
+__device__ __forceinline__ uint64_t scale_stage_offset(int mt, int ks, int K, int fmt) {
+  if (fmt == MOE_FMT_NVFP4) return ((uint64_t)mt * (uint64_t)(K >> 4) + (uint64_t)ks * 4u) * 128u;
+  return ((uint64_t)mt * (uint64_t)(K >> 5) + (uint64_t)ks * 2u) * 256u;
+}
+
+template <int NMAT>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
+  using C = TcCfg<NMAT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* load_full = bars;
+  uint64_t* a_full = bars + C::kStages;
+  uint64_t* stage_empty = bars + 2 * C::kStages;
+  uint64_t* acc_full = bars + 3 * C::kStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      ptx::mbar_init(&load_full[s], 1);
+      ptx::mbar_init(&a_full[s], kDeqThreads);
+      ptx::mbar_init(&stage_empty[s], 1);
+    }
+    ptx::mbar_init(acc_full, 1);
+    ptx::mbar_init(acc_empty, kDeqThreads);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  if (warp == kTmaWarp && lane == 0) ptx::prefetch_tmap(&tmap_b);
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int m_tiles = a.N / kTcBM;
+  const int total = *a.chunk_count * m_tiles;
+  const int ksteps = a.K / kTcBK;
+  const LayerHdr L = hdr_view(a.packed, a.E, a.H, a.F);
+  bool ok = true;
+
+  // Every role runs its loop with whole warps: waits are taken by all lanes and
+  // made warp-uniform, and only lane 0 issues TMA / MMA / commit, so no warp
+  // reaches the final block barrier diverged.
+  auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort_flag, kWaitLimit)) != 0;
+  };
+
+  if (warp == kTmaWarp) {
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0, issued_phase = 0;  // per stage: a load was armed, and its parity
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const int c = t / m_tiles, mt = t % m_tiles;
+      const int e = a.chunks[3 * c], row0 = a.chunks[3 * c + 1];
+      const uint8_t* cbase[NMAT];
+      const uint8_t* sbase[NMAT];
+      int fmt[NMAT];
+      uint32_t bytes = C::kBBytes;
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m) {
+        const int i = e * 3 + a.proj + m;
+        fmt[m] = L.fmt[i];
+        cbase[m] = L.base + L.code_off[i];
+        sbase[m] = L.base + L.scale_off[i];
+        bytes += (uint32_t)fmt_words(fmt[m]) * 1024u + (uint32_t)C::kScaleBytes;
+      }
+      for (int ks = 0; ks < ksteps; ++ks) {
+        if (!wait_all(&stage_empty[stage], phase ^ 1u)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          uint8_t* sb = smem + stage * C::kStageBytes;
+          ptx::mbar_arrive_expect_tx(&load_full[stage], bytes);
+          ptx::tma_load_2d(sb + C::kOffB, &tmap_b, ks * kTcBK, row0, &load_full[stage]);
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m) {
+            const int wpg = fmt_words(fmt[m]);
+            ptx::bulk_load(sb + C::kOffCodes + m * C::kCodeBytes, cbase[m] + code_stage_offset(mt, ks, a.K, wpg),
+                           (uint32_t)wpg * 1024u, &load_full[stage]);
+            ptx::bulk_load(sb + C::kOffScales + m * C::kScaleBytes,
+                           sbase[m] + scale_stage_offset(mt, ks, a.K, fmt[m]), (uint32_t)C::kScaleBytes,
+                           &load_full[stage]);
+          }
+        }
+        __syncwarp();
+        issued |= 1u << stage;
+        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // never leave while a copy may still be landing in shared memory
+    for (int s = 0; s < C::kStages; ++s)
+      if (issued & (1u << s)) ptx::mbar_wait(&load_full[s], (issued_phase >> s) & 1u, abort_flag, kWaitLimit / 4);
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    int stage = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    const uint32_t sbase = ptx::smem_u32(smem);
+    bool committed = false;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const int c = t / m_tiles;
+      const int rows = a.chunks[3 * c + 2];
+      const int nmma = min(kTcBN, (rows + 15) & ~15);
+      const uint32_t idesc = ptx::idesc_f16_f32(kTcBM, nmma);
+      if (!wait_all(acc_empty, acc_phase ^ 1u)) {
+        ok = false;
+        break;
+      }
+      acc_phase ^= 1u;
+      ptx::tc_fence_after();
+      for (int ks = 0; ks < ksteps; ++ks) {
+        if (!wait_all(&a_full[stage], phase) || !wait_all(&load_full[stage], phase)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        if (lane == 0) {
+          const uint32_t st = sbase + (uint32_t)(stage * C::kStageBytes);
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+            for (int k16 = 0; k16 < kTcBK / 16; ++k16)
+              ptx::mma_f16_ss(tmem + (uint32_t)(m * 256), ptx::sw128_desc(st + C::kOffA + m * C::kABytes + k16 * 32),
+                              ptx::sw128_desc(st + C::kOffB + k16 * 32), idesc, (ks | k16) != 0);
+          ptx::mma_commit(&stage_empty[stage]);
+        }
+        __syncwarp();
+        committed = true;
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) ptx::mma_commit(acc_full);
+      __syncwarp();
+    }
+    if (committed) {  // the last commit lands once every MMA issued by this CTA has completed
+      const int last = (stage + C::kStages - 1) % C::kStages;
+      const uint32_t par = (stage == 0) ? (phase ^ 1u) : phase;
+      ptx::mbar_wait(&stage_empty[last], par, abort_flag, kWaitLimit / 4);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------- dequant + epilogue
+    const int n = threadIdx.x & 127, gi = threadIdx.x >> 7;
+    const int q = warp & 3, chalf = warp >> 2;
+    int stage = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const int c = t / m_tiles, mt = t % m_tiles;
+      const int e = a.chunks[3 * c], row0 = a.chunks[3 * c + 1], rows = a.chunks[3 * c + 2];
+      int fmt[NMAT];
+      float tsc[NMAT];
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m) {
+        const int i = e * 3 + a.proj + m;
+        fmt[m] = L.fmt[i];
+        tsc[m] = fmt[m] == MOE_FMT_NVFP4 ? L.tscale[i] : 1.0f;
+      }
+      for (int ks = 0; ks < ksteps; ++ks) {
+        if (!wait_all(&load_full[stage], phase)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sb = smem + stage * C::kStageBytes;
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m)
+          dequant_group(fmt[m], reinterpret_cast<const uint32_t*>(sb + C::kOffCodes + m * C::kCodeBytes),
+                        sb + C::kOffScales + m * C::kScaleBytes, n, gi, sb + C::kOffA + m * C::kABytes);
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(&a_full[stage]);
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (!wait_all(acc_full, acc_phase)) {
+        ok = false;
+        break;
+      }
+      acc_phase ^= 1u;
+      ptx::tc_fence_after();
+      const int nrow = mt * kTcBM + q * 32 + lane;
+      const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+      for (int cb = chalf * 128; cb < chalf * 128 + 128 && cb < rows; cb += 32) {
+        uint32_t r0[32], r1[32];
+        ptx::tmem_ld32(lane_base + (uint32_t)cb, r0);
+        if (NMAT == 2) ptx::tmem_ld32(lane_base + 256u + (uint32_t)cb, r1);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int tok = cb + j;
+          if (tok >= rows) break;
+          const int r = row0 + tok;
+          if (NMAT == 2) {
+            float g = __uint_as_float(r0[j]), u = __uint_as_float(r1[j]);
+            if (a.row_scale) {
+              const float sx = a.row_scale[a.perm[r] / a.topk];
+              g *= sx * tsc[0];
+              u *= sx * tsc[1];
+              reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = g / (1.0f + __expf(-g)) * u;
+            } else {
+              reinterpret_cast<__half*>(a.out)[(size_t)r * a.N + nrow] = __float2half_rn(g / (1.0f + __expf(-g)) * u);
+            }
+          } else {
+            float o = __uint_as_float(r0[j]);
+            if (a.row_scale) o *= a.row_scale[r] * tsc[0];
+            reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = o;
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(acc_empty);
+    }
+  }
+
+  if (!ok) {
+    *abort_flag = 1;
+    if (a.status) atomicExch(a.status, (int32_t)MOE_ERR_TIMEOUT);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+int sm_count() {
+  static int n[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (n[dev] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    n[dev] = v > 0 ? v : 148;
+  }
+  return n[dev];
+}
+
+template <int NMAT>
+cudaError_t launch_tc(const TcArgs& a, const void* act, int rows_total, cudaStream_t stream) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)rows_total};
+  const cuuint64_t strides[1] = {(cuuint64_t)a.K * 2u};
+  const cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)kTcBN};
+  const cuuint32_t estr[2] = {1u, 1u};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(act), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  auto kern = expert_gemm_tc_kernel<NMAT>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<NMAT>::kSmem);
+  if (err != cudaSuccess) return err;
+  kern<<<sm_count(), kTcThreads, TcCfg<NMAT>::kSmem, stream>>>(map, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_expert_gemm_tc(const uint8_t* packed, int E, int H, int F, int T, int k, bool fp4, bool gateup,
+                                  const Workspace& ws, int32_t* status, cudaStream_t stream) {
+  TcArgs a{};
+  a.packed = packed;
+  a.E = E;
+  a.H = H;
+  a.F = F;
+  a.chunks = ws.chunks;
+  a.chunk_count = ws.chunk_count;
+  a.perm = ws.perm;
+  a.topk = k;
+  a.status = status;
+  const int R = T * k;
+  if (gateup) {
+    a.N = F;
+    a.K = H;
+    a.proj = 0;
+    a.row_scale = fp4 ? ws.sx : nullptr;
+    a.out = ws.h;
+    return launch_tc<2>(a, ws.xs, R, stream);
+  }
+  a.N = H;
+  a.K = F;
+  a.proj = 2;
+  a.row_scale = fp4 ? ws.sh : nullptr;
+  a.out = ws.o;
+  return launch_tc<1>(a, fp4 ? ws.hb : ws.h, R, stream);
+}
+
+}  // namespace moe

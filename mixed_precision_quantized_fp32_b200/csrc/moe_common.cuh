@@ -127,9 +127,9 @@ struct Workspace {
   int32_t* chunk_count;// [1]
   uint8_t* xq;         // [T*H] NVFP4 activation codes
   float* sx;           // [T]
-  void* xs;            // [T*k*H] 16-bit gathered activations (fp16 int / bf16 NVFP4)
+  void* xs;            // [T*k*H] fp16 gathered activations (NVFP4: exact e4m3 values)
   void* h;             // [T*k*F] fp16 (int) / fp32 (NVFP4 pre-quant)
-  void* hb;            // [T*k*F] bf16 NVFP4 decoded h codes
+  void* hb;            // [T*k*F] fp16 NVFP4 decoded h codes (exact)
   uint8_t* hq;         // [T*k*F] NVFP4 h codes
   float* sh;           // [T*k]
   float* o;            // [T*k*H] fp32 expert outputs, sorted rows

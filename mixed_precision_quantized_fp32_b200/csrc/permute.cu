@@ -166,9 +166,9 @@ __global__ void act_quant_x_kernel(const __nv_bfloat16* __restrict__ x, int H, u
   }
 }
 
-// Gather e4m3 activation codes into sorted rows as exact bf16 values.
+// Gather e4m3 activation codes into sorted rows as exact fp16 values.
 __global__ void gather_fp8_kernel(const uint8_t* __restrict__ xq, const int32_t* __restrict__ perm, int R,
-                                  int H, int k, __nv_bfloat16* __restrict__ xs) {
+                                  int H, int k, __half* __restrict__ xs) {
   const int r = blockIdx.x;
   const int t = perm[r] / k;
   const uint2* src = reinterpret_cast<const uint2*>(xq + (size_t)t * H);
@@ -176,19 +176,19 @@ __global__ void gather_fp8_kernel(const uint8_t* __restrict__ xq, const int32_t*
   for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
     const uint2 v = __ldg(src + c);
     uint4 o;
-    __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(&o);
+    __half* ob = reinterpret_cast<__half*>(&o);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      ob[i] = __float2bfloat16_rn(e4m3_value((v.x >> (8 * i)) & 255u));
-      ob[4 + i] = __float2bfloat16_rn(e4m3_value((v.y >> (8 * i)) & 255u));
+      ob[i] = __float2half_rn(e4m3_value((v.x >> (8 * i)) & 255u));
+      ob[4 + i] = __float2half_rn(e4m3_value((v.y >> (8 * i)) & 255u));
     }
     dst[c] = o;
   }
 }
 
-// Per-row e4m3 codes of the SwiGLU output (NVFP4 layers) and their exact bf16 values.
+// Per-row e4m3 codes of the SwiGLU output (NVFP4 layers) and their exact fp16 values.
 __global__ void act_quant_h_kernel(const float* __restrict__ h, int F, uint8_t* __restrict__ hq,
-                                   float* __restrict__ sh, __nv_bfloat16* __restrict__ hb,
+                                   float* __restrict__ sh, __half* __restrict__ hb,
                                    uint8_t* __restrict__ dbg_hq, float* __restrict__ dbg_sh) {
   __shared__ float red[32];
   const int r = blockIdx.x;
@@ -200,7 +200,7 @@ __global__ void act_quant_h_kernel(const float* __restrict__ h, int F, uint8_t* 
   for (int i = threadIdx.x; i < F; i += blockDim.x) {
     const uint8_t c = __nv_cvt_float_to_fp8(__fdiv_rn(hr[i], s), __NV_SATFINITE, __NV_E4M3);
     hq[(size_t)r * F + i] = c;
-    hb[(size_t)r * F + i] = __float2bfloat16_rn(e4m3_value(c));
+    hb[(size_t)r * F + i] = __float2half_rn(e4m3_value(c));
     if (dbg_hq) dbg_hq[(size_t)r * F + i] = c;
   }
   if (threadIdx.x == 0) {
@@ -226,7 +226,7 @@ cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4,
   const int R = T * k;
   if (fp4) {
     act_quant_x_kernel<<<T, 256, 0, stream>>>(x, H, ws.xq, ws.sx, dbg_xq, dbg_sx);
-    gather_fp8_kernel<<<R, 128, 0, stream>>>(ws.xq, ws.perm, R, H, k, (__nv_bfloat16*)ws.xs);
+    gather_fp8_kernel<<<R, 128, 0, stream>>>(ws.xq, ws.perm, R, H, k, (__half*)ws.xs);
   } else {
     gather_f16_kernel<<<R, 128, 0, stream>>>(x, ws.perm, R, H, k, (__half*)ws.xs);
   }
@@ -235,7 +235,7 @@ cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4,
 
 cudaError_t launch_act_quant_h(int R, int F, const Workspace& ws, uint8_t* dbg_hq, float* dbg_sh,
                                cudaStream_t stream) {
-  act_quant_h_kernel<<<R, 256, 0, stream>>>((const float*)ws.h, F, ws.hq, ws.sh, (__nv_bfloat16*)ws.hb,
+  act_quant_h_kernel<<<R, 256, 0, stream>>>((const float*)ws.h, F, ws.hq, ws.sh, (__half*)ws.hb,
                                             dbg_hq, dbg_sh);
   return cudaGetLastError();
 }

@@ -39,7 +39,9 @@ __global__ void router_warp_kernel(const __nv_bfloat16* __restrict__ x, const fl
 
 // ---------------------------------------------------------------- router, many tokens
 // Tiled fp32 GEMM: block tile 64 tokens x TE experts, k-tile 32; 256 threads,
-// each computing 4 tokens x TE/16 experts.
+// each computing 4 tokens x TE/16 experts.  Each k-tile is summed on its own and
+// the tile sums are added with Kahan compensation, so the rounding error stays
+// near that of a pairwise sum even for H = 12288.
 template <int TE>
 __global__ void __launch_bounds__(256) router_tile_kernel(const __nv_bfloat16* __restrict__ x,
                                                           const float* __restrict__ Wr,
@@ -51,11 +53,11 @@ __global__ void __launch_bounds__(256) router_tile_kernel(const __nv_bfloat16* _
   const int tid = threadIdx.x;
   const int t0 = blockIdx.x * TT, e0 = blockIdx.y * TE;
   const int ty = tid >> 4, tx = tid & 15;
-  float acc[4][PE];
+  float acc[4][PE], comp[4][PE];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < PE; ++j) acc[i][j] = 0.0f;
+    for (int j = 0; j < PE; ++j) acc[i][j] = comp[i][j] = 0.0f;
 
   for (int k0 = 0; k0 < H; k0 += BK) {
     {  // x tile: 64 tokens x 32 h = 256 chunks of 8 bf16
@@ -88,6 +90,11 @@ __global__ void __launch_bounds__(256) router_tile_kernel(const __nv_bfloat16* _
       ws[hh + 3][ee] = v.w;
     }
     __syncthreads();
+    float part[4][PE];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < PE; ++j) part[i][j] = 0.0f;
 #pragma unroll 8
     for (int kk = 0; kk < BK; ++kk) {
       float a[4], w[PE];
@@ -98,8 +105,17 @@ __global__ void __launch_bounds__(256) router_tile_kernel(const __nv_bfloat16* _
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < PE; ++j) acc[i][j] = fmaf(a[i], w[j], acc[i][j]);
+        for (int j = 0; j < PE; ++j) part[i][j] = fmaf(a[i], w[j], part[i][j]);
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < PE; ++j) {  // Kahan: acc += part
+        const float y = __fsub_rn(part[i][j], comp[i][j]);
+        const float t = __fadd_rn(acc[i][j], y);
+        comp[i][j] = __fsub_rn(__fsub_rn(t, acc[i][j]), y);
+        acc[i][j] = t;
+      }
     __syncthreads();
   }
 #pragma unroll
