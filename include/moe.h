@@ -201,6 +201,36 @@ MOE_API moe_status moe_layer_forward(const void* x, int32_t T, const float* rout
                              const moe_weights* w, int32_t k, void* y, void* ws, uint64_t ws_bytes,
                              uint64_t* ws_bytes_out, const moe_debug* dbg, cudaStream_t stream);
 
+/*
+ * moe_layer_forward_noalloc -- moe_layer_forward for callers that cannot
+ * allocate device memory: code running inside a CUDA graph or an allocator
+ * callback, embedded runtimes without cudaMalloc, or hosts whose memory pool
+ * must not grow.  (The method on the pages has no counterpart; this is a
+ * calling convenience of this library.)
+ *
+ * The workspace is a fixed array of MOE_NOALLOC_SCRATCH_BYTES (32 MiB) inside
+ * this library (a file-scope __device__ array, so every GPU that loads the
+ * library holds it until the process exits).  The call allocates nothing and
+ * calls no allocating CUDA or library routine; the caller still provides x,
+ * the router weights, the packed layer, y and (optionally) dbg, exactly as for
+ * moe_layer_forward.  Batches whose workspace (the ws_bytes_out query of
+ * moe_layer_forward) exceeds the array are rejected with MOE_ERR_WORKSPACE
+ * before anything runs; decode-sized batches of the five reference layers
+ * fit (the largest, 64 tokens of the 12288 x 14336 layer, needs ~13 MiB).
+ *
+ * The first call on a device looks up the array's device address with
+ * cudaGetSymbolAddress (with that device current) and caches it; make that
+ * first call before any stream capture.  Every call shares the one array and
+ * leaves its contents behind, so calls that overlap on the GPU (other streams,
+ * other host threads) race on it: serialize them.  Nothing in the array needs
+ * to start at zero: every byte the forward reads is written earlier in the
+ * same call.  Errors: as moe_layer_forward.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES (32ull << 20)
+MOE_API moe_status moe_layer_forward_noalloc(const void* x, int32_t T, const float* router_w,
+                                             const float* router_b, const moe_weights* w, int32_t k, void* y,
+                                             const moe_debug* dbg, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -6,9 +6,9 @@ fails loudly if the library has not been built.
 """
 from ._lib import MOE_STAGE_EVENTS, MoeError, load as _load
 from .api import (FMT_INT2, FMT_INT3, FMT_INT4, FMT_NVFP4, DEBUG_FIELDS, PackedLayer, alloc_packed,
-                  moe_layer_forward, moe_pack, pack_layout, workspace_bytes)
+                  moe_layer_forward, moe_layer_forward_noalloc, moe_pack, pack_layout, workspace_bytes)
 
 _load()
 
 __all__ = ["FMT_INT2", "FMT_INT3", "FMT_INT4", "FMT_NVFP4", "DEBUG_FIELDS", "MOE_STAGE_EVENTS", "MoeError",
-           "PackedLayer", "alloc_packed", "moe_layer_forward", "moe_pack", "pack_layout", "workspace_bytes"]
+           "PackedLayer", "alloc_packed", "moe_layer_forward", "moe_layer_forward_noalloc", "moe_pack", "pack_layout", "workspace_bytes"]

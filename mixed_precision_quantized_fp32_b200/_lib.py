@@ -19,7 +19,8 @@ STATUS = {
     5: "MOE_ERR_FORMAT", 6: "MOE_ERR_CUDA", 7: "MOE_ERR_TIMEOUT", 8: "MOE_ERR_UNSUPPORTED_DEVICE",
 }
 
-EXPORTS = ("moe_pack", "moe_layer_forward")
+EXPORTS = ("moe_pack", "moe_layer_forward", "moe_layer_forward_noalloc")
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class MoeWeights(C.Structure):
@@ -58,6 +59,9 @@ def load() -> C.CDLL:
         L.moe_layer_forward.restype = C.c_int
         L.moe_layer_forward.argtypes = [P, i32, P, P, C.POINTER(MoeWeights), i32, P, P, u64, P,
                                         C.POINTER(MoeDebug), P]
+        L.moe_layer_forward_noalloc.restype = C.c_int
+        L.moe_layer_forward_noalloc.argtypes = [P, i32, P, P, C.POINTER(MoeWeights), i32, P,
+                                                C.POINTER(MoeDebug), P]
         _lib = L
     return _lib
 

@@ -128,5 +128,19 @@ def moe_layer_forward(x: torch.Tensor, router_w: torch.Tensor, router_b: torch.T
     return y
 
 
+def moe_layer_forward_noalloc(x: torch.Tensor, router_w: torch.Tensor, router_b: torch.Tensor | None,
+                              layer: PackedLayer, k: int, y: torch.Tensor,
+                              stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """y = MoE(x) with the workspace in the library's fixed device array (for callers
+    that cannot allocate device memory; batches whose workspace exceeds the array
+    raise MoeError MOE_ERR_WORKSPACE).  y must be preallocated: this call makes no
+    allocation of its own.  Calls that overlap on the GPU share the array and race."""
+    w = layer.weights_struct()
+    rc = _lib.load().moe_layer_forward_noalloc(_ptr(x), x.shape[0], _ptr(router_w), _ptr(router_b), C.byref(w), k,
+                                               _ptr(y), None, _stream(stream))
+    check("moe_layer_forward_noalloc", rc)
+    return y
+
+
 __all__ = ["FMT_INT2", "FMT_INT3", "FMT_INT4", "FMT_NVFP4", "MoeError", "PackedLayer", "alloc_packed",
-           "moe_layer_forward", "moe_pack", "pack_layout", "workspace_bytes"]
+           "moe_layer_forward", "moe_layer_forward_noalloc", "moe_pack", "pack_layout", "workspace_bytes"]
