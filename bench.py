@@ -53,11 +53,14 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+TRAFFIC_SOURCES = ("expert_gemm_tc.cu", "tc_ptx.cuh", "moe_common.cuh")
+
+
 def csrc_hash() -> str:
+    """Hash of the sources that define the dominant kernel (the tcgen05 expert GEMM)."""
     h = hashlib.sha256()
-    for fn in sorted(os.listdir(CSRC)):
-        if fn.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(CSRC, fn), "rb").read())
+    for fn in TRAFFIC_SOURCES:
+        h.update(open(os.path.join(CSRC, fn), "rb").read())
     return h.hexdigest()[:16]
 
 

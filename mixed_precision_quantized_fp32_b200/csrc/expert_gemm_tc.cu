@@ -8,12 +8,13 @@
 // (its sec. 3.6, "fused linear + activation"), built for sm_100a:
 //   * one persistent CTA per SM walks (token chunk, 128-row weight tile) work
 //     items; chunk = up to 256 consecutive expert-sorted rows of one expert;
-//   * warp 8 (one lane) streams each 64-input stage: the activation tile with a
-//     2D TMA load (128-byte swizzle) and the packed codes + scales of the weight
-//     tile with 1D bulk copies (both never multicast);
+//   * warp 8 (one lane) streams each 32-input stage (one quantization group):
+//     the activation tile with a 2D TMA load (64-byte swizzle) and the packed
+//     codes + scales of the weight tile with 1D bulk copies (never multicast);
+//     short stages let 6 (gate/up) or 8 (down) of them be in flight;
 //   * warps 0-7 turn codes into fp16 operands (exponent-bias unpack: a code u
 //     OR'ed into the mantissa of 1024.0 gives 1024+u exactly; one subtract
-//     and one multiply by the group scale) written straight into the 128-byte
+//     and one multiply by the group scale) written straight into the 64-byte
 //     swizzled K-major layout the tensor core reads;
 //   * warp 9 (one lane) issues tcgen05.mma M=128 (weight rows) x N<=256 (token
 //     rows) x K=16 and commits to mbarriers;
@@ -32,7 +33,7 @@ namespace {
 
 constexpr int kTcBM = 128;   // weight rows per work item (MMA M)
 constexpr int kTcBN = 256;   // token rows per work item (max MMA N)
-constexpr int kTcBK = 64;    // inputs per pipeline stage (one 128-byte swizzle row of fp16)
+constexpr int kTcBK = 32;    // inputs per pipeline stage: one quantization group, a 64-byte fp16 row
 constexpr int kTcThreads = 320;
 constexpr int kTmaWarp = 8, kMmaWarp = 9;
 constexpr int kDeqThreads = 256;
@@ -40,21 +41,20 @@ constexpr long long kWaitLimit = 4000000000LL;  // clock cycles, ~2 s
 
 template <int NMAT>
 struct TcCfg {
-  static constexpr int kStages = NMAT == 2 ? 3 : 4;
-  static constexpr int kBBytes = kTcBN * kTcBK * 2;
-  static constexpr int kABytes = kTcBM * kTcBK * 2;
-  static constexpr int kCodeBytes = 4096;  // <= 4 words x 2 groups x 128 rows x 4 bytes
-  static constexpr int kScaleBytes = 512;  // 2 fp16 groups or 4 e4m3 blocks x 128 rows
+  static constexpr int kBBytes = kTcBN * kTcBK * 2;  // 16 KB activation tile
+  static constexpr int kABytes = kTcBM * kTcBK * 2;  // 8 KB dequantized weight tile
+  static constexpr int kCodeBytes = 2048;  // <= 4 words x 128 rows x 4 bytes (one group)
+  static constexpr int kScaleBytes = 256;  // one fp16 group or two e4m3 blocks x 128 rows
   static constexpr int kOffB = 0;
   static constexpr int kOffA = kBBytes;
   static constexpr int kOffCodes = kOffA + NMAT * kABytes;
   static constexpr int kOffScales = kOffCodes + NMAT * kCodeBytes;
   static constexpr int kStageBytes = (kOffScales + NMAT * kScaleBytes + 1023) / 1024 * 1024;
   static constexpr int kBarBytes = 256;
+  static constexpr int kStages = (232448 - kBarBytes - 1024) / kStageBytes;  // as many as fit
   static constexpr int kSmem = kStages * kStageBytes + kBarBytes + 1024;
 };
-static_assert(TcCfg<2>::kSmem <= 232448, "gate/up stages exceed shared memory");
-static_assert(TcCfg<1>::kSmem <= 232448, "down stages exceed shared memory");
+static_assert(TcCfg<2>::kStages >= 6 && TcCfg<1>::kStages >= 8, "pipeline too shallow");
 
 struct TcArgs {
   const uint8_t* packed;
@@ -88,71 +88,60 @@ __device__ __forceinline__ void e2m1x8_to_f16(uint32_t w, uint32_t* o) {
       : "r"(w));
 }
 
-// Dequantize group gi (32 inputs) of weight row n of one matrix from the staged
-// codes/scales into four 16-byte chunks (8 inputs each) of the swizzled A tile.
-__device__ __forceinline__ void dequant_group(int fmt, const uint32_t* __restrict__ codes,
-                                              const uint8_t* __restrict__ scales, int n, int gi, uint8_t* A) {
-  uint32_t v[16];  // 16 fp16 pairs = 32 inputs in natural order
+// Eight inputs (chunk c = inputs 8c..8c+7 of the staged group) of weight row n
+// as four fp16 pairs in natural order.  codes: the group's words [word][128
+// rows]; scales: [128] fp16 (integer) or [2 blocks][128] e4m3 (NVFP4).
+__device__ __forceinline__ uint4 dequant_chunk(int fmt, const uint32_t* __restrict__ codes,
+                                              const uint8_t* __restrict__ scales, int n, int c) {
+  uint32_t v[4];
   if (fmt == MOE_FMT_NVFP4) {
-    const float s0 = e4m3_value(scales[(2 * gi) * 128 + n]);
-    const float s1 = e4m3_value(scales[(2 * gi + 1) * 128 + n]);
-    const __half2 h0 = __float2half2_rn(s0), h1 = __float2half2_rn(s1);
-    const uint32_t p0 = *reinterpret_cast<const uint32_t*>(&h0), p1 = *reinterpret_cast<const uint32_t*>(&h1);
+    const __half2 s2 = __float2half2_rn(e4m3_value(scales[(c >> 1) * 128 + n]));
+    const uint32_t p = *reinterpret_cast<const uint32_t*>(&s2);
+    e2m1x8_to_f16(codes[c * 128 + n], v);
 #pragma unroll
-    for (int wd = 0; wd < 4; ++wd) {
-      uint32_t o[4];
-      e2m1x8_to_f16(codes[(gi * 4 + wd) * 128 + n], o);
-#pragma unroll
-      for (int b = 0; b < 4; ++b) v[wd * 4 + b] = h2mul(o[b], wd < 2 ? p0 : p1);  // exact
-    }
+    for (int b = 0; b < 4; ++b) v[b] = h2mul(v[b], p);  // exact: <= 6 significant bits
   } else {
-    const uint32_t s = reinterpret_cast<const uint16_t*>(scales)[gi * 128 + n];
+    const uint32_t s = reinterpret_cast<const uint16_t*>(scales)[n];
     const uint32_t s2 = s | (s << 16);
     if (fmt == MOE_FMT_INT4) {
+      const uint32_t w = codes[c * 128 + n];
 #pragma unroll
-      for (int wd = 0; wd < 4; ++wd) {
-        const uint32_t w = codes[(gi * 4 + wd) * 128 + n];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          v[wd * 4 + j] = h2mul(h2sub(((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u, 0x64086408u), s2);
-      }
+      for (int j = 0; j < 4; ++j)
+        v[j] = h2mul(h2sub(((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u, 0x64086408u), s2);
     } else if (fmt == MOE_FMT_INT2) {
+      const uint32_t w = codes[(c >> 1) * 128 + n] >> (8 * (c & 1));
 #pragma unroll
-      for (int wd = 0; wd < 2; ++wd) {
-        const uint32_t w = codes[(gi * 2 + wd) * 128 + n];
+      for (int j = 0; j < 4; ++j)
+        v[j] = h2mul(h2sub(((w >> (2 * j)) & 0x00030003u) | 0x64006400u, 0x64026402u), s2);
+    } else {  // INT3: low bits as INT2, bit 2 of pair J at bits J and 16+J of word 2
+      const uint32_t lo = codes[(c >> 1) * 128 + n] >> (8 * (c & 1));
+      const uint32_t hi = codes[2 * 128 + n] >> (4 * c);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          v[wd * 8 + j] = h2mul(h2sub(((w >> (2 * j)) & 0x00030003u) | 0x64006400u, 0x64026402u), s2);
-      }
-    } else {  // INT3
-      const uint32_t hi = codes[(gi * 3 + 2) * 128 + n];
-#pragma unroll
-      for (int wd = 0; wd < 2; ++wd) {
-        const uint32_t lo = codes[(gi * 3 + wd) * 128 + n];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t u = ((lo >> (2 * j)) & 0x00030003u) | (((hi >> (8 * wd + j)) & 0x00010001u) << 2);
-          v[wd * 8 + j] = h2mul(h2sub(u | 0x64006400u, 0x64046404u), s2);
-        }
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t u = ((lo >> (2 * j)) & 0x00030003u) | (((hi >> j) & 0x00010001u) << 2);
+        v[j] = h2mul(h2sub(u | 0x64006400u, 0x64046404u), s2);
       }
     }
   }
-  uint8_t* row = A + (n >> 3) * 1024 + (n & 7) * 128;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const int chunk = (4 * gi + c) ^ (n & 7);
-    *reinterpret_cast<uint4*>(row + chunk * 16) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-  }
+  return make_uint4(v[0], v[1], v[2], v[3]);
 }
 
-__device__ __forceinline__ uint64_t code_stage_offset(int mt, int ks, int K, int wpg) {
-  // bytes of words [kg = 2*(ks%2) .. +1][word][n] of tile (mt, ks/2); contiguous wpg*1024 bytes
-  return ((((uint64_t)mt * (uint64_t)(K >> 7) + (uint64_t)(ks >> 1)) * 4u + (uint64_t)(ks & 1) * 2u) *
-          (uint64_t)wpg * 128u) * 4u;
+// Byte offset of chunk c (16 bytes) of row n in a K-major tile of 64-byte rows
+// with the 64-byte swizzle (8-row atoms of 512 bytes; chunk index XOR row/2).
+__device__ __forceinline__ int sw64_offset(int n, int c) {
+  return (n >> 3) * 512 + (n & 7) * 64 + ((c ^ ((n >> 1) & 3)) << 4);
 }
-__device__ __forceinline__ uint64_t scale_stage_offset(int mt, int ks, int K, int fmt) {
-  if (fmt == MOE_FMT_NVFP4) return ((uint64_t)mt * (uint64_t)(K >> 4) + (uint64_t)ks * 4u) * 128u;
-  return ((uint64_t)mt * (uint64_t)(K >> 5) + (uint64_t)ks * 2u) * 256u;
+
+// Byte offset of the words of group g (inputs 32g..32g+31) of weight tile mt:
+// [word][128 rows], contiguous wpg*512 bytes.
+__device__ __forceinline__ uint64_t code_stage_offset(int mt, int g, int K, int wpg) {
+  return ((((uint64_t)mt * (uint64_t)(K >> 7) + (uint64_t)(g >> 2)) * 4u + (uint64_t)(g & 3)) * (uint64_t)wpg *
+          128u) * 4u;
+}
+// Byte offset of the scales of group g of weight tile mt (256 contiguous bytes).
+__device__ __forceinline__ uint64_t scale_stage_offset(int mt, int g, int K, int fmt) {
+  if (fmt == MOE_FMT_NVFP4) return ((uint64_t)mt * (uint64_t)(K >> 4) + (uint64_t)g * 2u) * 128u;
+  return ((uint64_t)mt * (uint64_t)(K >> 5) + (uint64_t)g) * 256u;
 }
 
 template <int NMAT>
@@ -222,7 +211,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         fmt[m] = L.fmt[i];
         cbase[m] = L.base + L.code_off[i];
         sbase[m] = L.base + L.scale_off[i];
-        bytes += (uint32_t)fmt_words(fmt[m]) * 1024u + (uint32_t)C::kScaleBytes;
+        bytes += (uint32_t)fmt_words(fmt[m]) * 512u + (uint32_t)C::kScaleBytes;
       }
       for (int ks = 0; ks < ksteps; ++ks) {
         if (!wait_all(&stage_empty[stage], phase ^ 1u)) {
@@ -237,7 +226,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int m = 0; m < NMAT; ++m) {
             const int wpg = fmt_words(fmt[m]);
             ptx::bulk_load(sb + C::kOffCodes + m * C::kCodeBytes, cbase[m] + code_stage_offset(mt, ks, a.K, wpg),
-                           (uint32_t)wpg * 1024u, &load_full[stage]);
+                           (uint32_t)wpg * 512u, &load_full[stage]);
             ptx::bulk_load(sb + C::kOffScales + m * C::kScaleBytes,
                            sbase[m] + scale_stage_offset(mt, ks, a.K, fmt[m]), (uint32_t)C::kScaleBytes,
                            &load_full[stage]);
@@ -284,8 +273,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int m = 0; m < NMAT; ++m)
 #pragma unroll
             for (int k16 = 0; k16 < kTcBK / 16; ++k16)
-              ptx::mma_f16_ss(tmem + (uint32_t)(m * 256), ptx::sw128_desc(st + C::kOffA + m * C::kABytes + k16 * 32),
-                              ptx::sw128_desc(st + C::kOffB + k16 * 32), idesc, (ks | k16) != 0);
+              ptx::mma_f16_ss(tmem + (uint32_t)(m * 256), ptx::sw64_desc(st + C::kOffA + m * C::kABytes + k16 * 32),
+                              ptx::sw64_desc(st + C::kOffB + k16 * 32), idesc, (ks | k16) != 0);
           ptx::mma_commit(&stage_empty[stage]);
         }
         __syncwarp();
@@ -307,7 +296,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------- dequant + epilogue
-    const int n = threadIdx.x & 127, gi = threadIdx.x >> 7;
+    // gate/up: thread -> (matrix t/128, row t%128), all 4 chunks of the group;
+    // down: thread -> (chunk pair t/128, row t%128), 2 chunks.
+    const int n = threadIdx.x & 127, sel = threadIdx.x >> 7;
     const int q = warp & 3, chalf = warp >> 2;
     int stage = 0;
     uint32_t phase = 0, acc_phase = 0;
@@ -322,16 +313,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         fmt[m] = L.fmt[i];
         tsc[m] = fmt[m] == MOE_FMT_NVFP4 ? L.tscale[i] : 1.0f;
       }
+      const int my_m = NMAT == 2 ? sel : 0;
+      const int my_fmt = (NMAT == 2 && sel) ? fmt[NMAT - 1] : fmt[0];
       for (int ks = 0; ks < ksteps; ++ks) {
         if (!wait_all(&load_full[stage], phase)) {
           ok = false;
           break;
         }
         uint8_t* sb = smem + stage * C::kStageBytes;
+        const uint32_t* codes = reinterpret_cast<const uint32_t*>(sb + C::kOffCodes + my_m * C::kCodeBytes);
+        const uint8_t* scales = sb + C::kOffScales + my_m * C::kScaleBytes;
+        uint8_t* A = sb + C::kOffA + my_m * C::kABytes;
+        constexpr int kChunks = NMAT == 2 ? 4 : 2;
 #pragma unroll
-        for (int m = 0; m < NMAT; ++m)
-          dequant_group(fmt[m], reinterpret_cast<const uint32_t*>(sb + C::kOffCodes + m * C::kCodeBytes),
-                        sb + C::kOffScales + m * C::kScaleBytes, n, gi, sb + C::kOffA + m * C::kABytes);
+        for (int i = 0; i < kChunks; ++i) {
+          const int ch = NMAT == 2 ? i : 2 * sel + i;
+          *reinterpret_cast<uint4*>(A + sw64_offset(n, ch)) = dequant_chunk(my_fmt, codes, scales, n, ch);
+        }
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(&a_full[stage]);
         if (++stage == C::kStages) {
@@ -426,7 +424,7 @@ cudaError_t launch_tc(const TcArgs& a, const void* act, int rows_total, cudaStre
   const cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)kTcBN};
   const cuuint32_t estr[2] = {1u, 1u};
   if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(act), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   auto kern = expert_gemm_tc_kernel<NMAT>;

@@ -11,13 +11,13 @@ namespace moe {
 
 // ---------------------------------------------------------------- router, few tokens
 // One warp per (token, expert) dot product; lanes stride over H with 8-byte
-// bf16 and 16-byte fp32 loads.  Used when T is small (decode).
+// bf16 and 16-byte fp32 loads.  Used when T or E is small.
 __global__ void router_warp_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ Wr,
                                    const float* __restrict__ b, int T, int H, int E,
                                    float* __restrict__ logits) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * (blockDim.x >> 5) + warp;
-  const int t = blockIdx.y;
+  const int e = blockIdx.y * (blockDim.x >> 5) + warp;
+  const int t = blockIdx.x;
   if (e >= E) return;
   const __nv_bfloat16* xr = x + (size_t)t * H;
   const float* wr = Wr + (size_t)e * H;
@@ -197,12 +197,9 @@ __global__ void topk_softmax_kernel(const float* __restrict__ logits, int T, int
 cudaError_t launch_router_topk(const __nv_bfloat16* x, const float* Wr, const float* b, int T, int H,
                                int E, int k, const Workspace& ws, int32_t* dbg_idx, float* dbg_w,
                                cudaStream_t stream) {
-  if (T <= 64) {
-    dim3 grid((E + 7) / 8, T);
+  if (T <= 64 || E <= 32) {  // one warp per dot product: plenty of parallelism when E is small
+    dim3 grid(T, (E + 7) / 8);
     router_warp_kernel<<<grid, 256, 0, stream>>>(x, Wr, b, T, H, E, ws.logits);
-  } else if (E <= 16) {
-    dim3 grid((T + 63) / 64, (E + 15) / 16);
-    router_tile_kernel<16><<<grid, 256, 0, stream>>>(x, Wr, b, T, H, E, ws.logits);
   } else {
     dim3 grid((T + 63) / 64, (E + 63) / 64);
     router_tile_kernel<64><<<grid, 256, 0, stream>>>(x, Wr, b, T, H, E, ws.logits);

@@ -130,6 +130,17 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t start) {
   return d;
 }
 
+// Same for 64-byte swizzled rows (8-row atoms of 512 bytes).
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t start) {
+  uint64_t d = 0;
+  d |= (uint64_t)((start >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;
+  d |= (uint64_t)(512u >> 4) << 32;                // stride byte offset: 8 rows x 64 bytes
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)4u << 61;                         // swizzle mode: 64 bytes
+  return d;
+}
+
 // Instruction descriptor, kind::f16: fp16 A and B (K-major), fp32 accumulator.
 __host__ __device__ __forceinline__ uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4)                      // D format: f32
