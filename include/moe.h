@@ -164,7 +164,18 @@ typedef struct {
                                 router+top-k, permutation, activation gather/quantization,
                                 gate/up GEMM, h quantization (NVFP4), down GEMM, combine,
                                 and after combine, so stage times can be read back */
+  uint64_t* trace;    /* [MOE_TRACE_WORDS] or NULL: diagnostics of the tcgen05 gate/up GEMM
+                         (batches with many rows per expert): clock64 stamps taken by CTA 0,
+                         MOE_TRACE_EVENTS rows of MOE_TRACE_STAGES pipeline stages; row 0:
+                         producer got a free stage, 1: producer issued its copies, 2: dequant
+                         warp 0 saw the stage land, 3: dequant warp 0 released it, 4: MMA lane
+                         saw it ready, 5: MMA issued and committed it; row 6 holds, per work
+                         item, the epilogue start, row 7 its end.  Zero it before the call. */
 } moe_debug;
+
+#define MOE_TRACE_EVENTS 8
+#define MOE_TRACE_STAGES 1024
+#define MOE_TRACE_WORDS (MOE_TRACE_EVENTS * MOE_TRACE_STAGES)
 
 #define MOE_STAGE_EVENTS 8
 

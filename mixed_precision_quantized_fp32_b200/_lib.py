@@ -13,6 +13,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmoe_b200.so")
 
 MOE_STAGE_EVENTS = 8
+MOE_TRACE_EVENTS = 8
+MOE_TRACE_STAGES = 1024
 
 STATUS = {
     0: "MOE_OK", 1: "MOE_ERR_ARG", 2: "MOE_ERR_ALIGN", 3: "MOE_ERR_SHAPE", 4: "MOE_ERR_WORKSPACE",
@@ -32,7 +34,7 @@ class MoeDebug(C.Structure):
     _fields_ = [("topk_idx", C.c_void_p), ("topk_w", C.c_void_p), ("perm", C.c_void_p),
                 ("inv", C.c_void_p), ("counts", C.c_void_p), ("xq", C.c_void_p), ("sx", C.c_void_p),
                 ("hq", C.c_void_p), ("sh", C.c_void_p), ("status", C.c_void_p),
-                ("stage_events", C.c_void_p)]
+                ("stage_events", C.c_void_p), ("trace", C.c_void_p)]
 
 
 class MoeError(RuntimeError):

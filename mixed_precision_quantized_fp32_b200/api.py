@@ -91,7 +91,7 @@ def workspace_bytes(layer: PackedLayer, T: int, k: int) -> int:
     return int(need.value)
 
 
-DEBUG_FIELDS = ("topk_idx", "topk_w", "perm", "inv", "counts", "xq", "sx", "hq", "sh", "status")
+DEBUG_FIELDS = ("topk_idx", "topk_w", "perm", "inv", "counts", "xq", "sx", "hq", "sh", "status", "trace")
 
 
 def moe_layer_forward(x: torch.Tensor, router_w: torch.Tensor, router_b: torch.Tensor | None,

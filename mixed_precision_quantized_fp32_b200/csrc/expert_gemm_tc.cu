@@ -8,17 +8,16 @@
 // (its sec. 3.6, "fused linear + activation"), built for sm_100a:
 //   * one persistent CTA per SM walks (token chunk, 128-row weight tile) work
 //     items; chunk = up to 256 consecutive expert-sorted rows of one expert;
-//   * warp 8 (one lane) streams each 32-input stage (one quantization group):
-//     the activation tile with a 2D TMA load (64-byte swizzle) and the packed
+//   * warp 16 (one lane) streams each 64-input stage (two quantization groups):
+//     the activation tile with a 2D TMA load (128-byte swizzle) and the packed
 //     codes + scales of the weight tile with 1D bulk copies (never multicast);
-//     short stages let 6 (gate/up) or 8 (down) of them be in flight;
-//   * warps 0-7 turn codes into fp16 operands (exponent-bias unpack: a code u
+//   * warps 0-15 turn codes into fp16 operands (exponent-bias unpack: a code u
 //     OR'ed into the mantissa of 1024.0 gives 1024+u exactly; one subtract
-//     and one multiply by the group scale) written straight into the 64-byte
-//     swizzled K-major layout the tensor core reads;
-//   * warp 9 (one lane) issues tcgen05.mma M=128 (weight rows) x N<=256 (token
+//     and one multiply by the group scale) written straight into the swizzled
+//     K-major layout the tensor core reads;
+//   * warp 17 (one lane) issues tcgen05.mma M=128 (weight rows) x N<=256 (token
 //     rows) x K=16 and commits to mbarriers;
-//   * warps 0-7 then drain TMEM (tcgen05.ld) into the SwiGLU / scale epilogue.
+//   * warps 0-15 then drain TMEM (tcgen05.ld) into the SwiGLU / scale epilogue.
 // Every mbarrier wait is bounded; a wait that gives up raises an abort flag so
 // every role leaves its loop, writes MOE_ERR_TIMEOUT to the status word and
 // the CTA frees its TMEM before returning.
@@ -33,18 +32,30 @@ namespace {
 
 constexpr int kTcBM = 128;   // weight rows per work item (MMA M)
 constexpr int kTcBN = 256;   // token rows per work item (max MMA N)
-constexpr int kTcBK = 32;    // inputs per pipeline stage: one quantization group, a 64-byte fp16 row
-constexpr int kTcThreads = 320;
-constexpr int kTmaWarp = 8, kMmaWarp = 9;
-constexpr int kDeqThreads = 256;
+#ifndef MOE_TC_BK
+#define MOE_TC_BK 64
+#endif
+constexpr int kTcBK = MOE_TC_BK;        // inputs per pipeline stage (32 or 64)
+constexpr int kGroups = kTcBK / 32;     // quantization groups per stage
+constexpr int kRowBytes = kTcBK * 2;    // bytes of one fp16 tile row = swizzle span (64 or 128)
+static_assert(kTcBK == 32 || kTcBK == 64, "stage depth");
+#ifndef MOE_TC_DEQ_WARPS
+#define MOE_TC_DEQ_WARPS 16
+#endif
+constexpr int kDeqWarps = MOE_TC_DEQ_WARPS;  // dequantize + epilogue warps (8 or 16)
+static_assert(kDeqWarps == 8 || kDeqWarps == 16, "dequant warps");
+constexpr int kThreadsPerRow = kDeqWarps * 32 / 128;
+constexpr int kTmaWarp = kDeqWarps, kMmaWarp = kDeqWarps + 1;
+constexpr int kTcThreads = 32 * (kDeqWarps + 2);
 constexpr long long kWaitLimit = 4000000000LL;  // clock cycles, ~2 s
+constexpr int kPrefetchAhead = 4;                 // stages of packed codes warmed in L2 ahead of their copy
 
 template <int NMAT>
 struct TcCfg {
-  static constexpr int kBBytes = kTcBN * kTcBK * 2;  // 16 KB activation tile
-  static constexpr int kABytes = kTcBM * kTcBK * 2;  // 8 KB dequantized weight tile
-  static constexpr int kCodeBytes = 2048;  // <= 4 words x 128 rows x 4 bytes (one group)
-  static constexpr int kScaleBytes = 256;  // one fp16 group or two e4m3 blocks x 128 rows
+  static constexpr int kBBytes = kTcBN * kRowBytes;   // activation tile
+  static constexpr int kABytes = kTcBM * kRowBytes;   // dequantized weight tile
+  static constexpr int kCodeBytes = kGroups * 2048;   // <= 4 words x 128 rows x 4 bytes per group
+  static constexpr int kScaleBytes = kGroups * 256;   // one fp16 group or two e4m3 blocks x 128 rows
   static constexpr int kOffB = 0;
   static constexpr int kOffA = kBBytes;
   static constexpr int kOffCodes = kOffA + NMAT * kABytes;
@@ -54,7 +65,7 @@ struct TcCfg {
   static constexpr int kStages = (232448 - kBarBytes - 1024) / kStageBytes;  // as many as fit
   static constexpr int kSmem = kStages * kStageBytes + kBarBytes + 1024;
 };
-static_assert(TcCfg<2>::kStages >= 6 && TcCfg<1>::kStages >= 8, "pipeline too shallow");
+static_assert(TcCfg<2>::kStages >= 3 && TcCfg<1>::kStages >= 4 && TcCfg<1>::kStages <= 8, "pipeline depth");
 
 struct TcArgs {
   const uint8_t* packed;
@@ -68,7 +79,13 @@ struct TcArgs {
   int topk;
   void* out;               // gate/up: h [rows][F] (fp16, or fp32 for NVFP4); down: o fp32 [rows][H]
   int32_t* status;
+  unsigned long long* trace;  // diagnostics: per-stage clock64 stamps of CTA 0 (or null)
 };
+
+// Stamp event `ev` of global stage counter `i` (CTA 0 only, first MOE_TRACE_STAGES stages).
+__device__ __forceinline__ void trace_stamp(unsigned long long* tr, int ev, int i) {
+  if (tr && blockIdx.x == 0 && i < MOE_TRACE_STAGES) tr[ev * MOE_TRACE_STAGES + i] = (unsigned long long)clock64();
+}
 
 __device__ __forceinline__ uint32_t h2sub(uint32_t a, uint32_t b) {
   __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
@@ -90,11 +107,13 @@ __device__ __forceinline__ void e2m1x8_to_f16(uint32_t w, uint32_t* o) {
 
 // Eight inputs (chunk c = inputs 8c..8c+7 of the staged group) of weight row n
 // as four fp16 pairs in natural order.  codes: the group's words [word][128
-// rows]; scales: [128] fp16 (integer) or [2 blocks][128] e4m3 (NVFP4).
-__device__ __forceinline__ uint4 dequant_chunk(int fmt, const uint32_t* __restrict__ codes,
-                                              const uint8_t* __restrict__ scales, int n, int c) {
+// rows]; scales: [128] fp16 (integer) or [2 blocks][128] e4m3 (NVFP4).  The
+// format is a template parameter so a stage's chunks are straight-line code.
+template <int FMT>
+__device__ __forceinline__ uint4 dequant_chunk(const uint32_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                              int n, int c) {
   uint32_t v[4];
-  if (fmt == MOE_FMT_NVFP4) {
+  if (FMT == MOE_FMT_NVFP4) {
     const __half2 s2 = __float2half2_rn(e4m3_value(scales[(c >> 1) * 128 + n]));
     const uint32_t p = *reinterpret_cast<const uint32_t*>(&s2);
     e2m1x8_to_f16(codes[c * 128 + n], v);
@@ -103,12 +122,12 @@ __device__ __forceinline__ uint4 dequant_chunk(int fmt, const uint32_t* __restri
   } else {
     const uint32_t s = reinterpret_cast<const uint16_t*>(scales)[n];
     const uint32_t s2 = s | (s << 16);
-    if (fmt == MOE_FMT_INT4) {
+    if (FMT == MOE_FMT_INT4) {
       const uint32_t w = codes[c * 128 + n];
 #pragma unroll
       for (int j = 0; j < 4; ++j)
         v[j] = h2mul(h2sub(((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u, 0x64086408u), s2);
-    } else if (fmt == MOE_FMT_INT2) {
+    } else if (FMT == MOE_FMT_INT2) {
       const uint32_t w = codes[(c >> 1) * 128 + n] >> (8 * (c & 1));
 #pragma unroll
       for (int j = 0; j < 4; ++j)
@@ -126,22 +145,101 @@ __device__ __forceinline__ uint4 dequant_chunk(int fmt, const uint32_t* __restri
   return make_uint4(v[0], v[1], v[2], v[3]);
 }
 
-// Byte offset of chunk c (16 bytes) of row n in a K-major tile of 64-byte rows
-// with the 64-byte swizzle (8-row atoms of 512 bytes; chunk index XOR row/2).
-__device__ __forceinline__ int sw64_offset(int n, int c) {
+// Byte offset of 16-byte chunk c of row n in a K-major tile of kRowBytes rows
+// with the matching swizzle (8-row atoms; chunk index XOR'ed with the row bits
+// the swizzle mode uses: row%8 for 128-byte rows, (row/2)%4 for 64-byte rows).
+__device__ __forceinline__ int tile_offset(int n, int c) {
+  if (kRowBytes == 128) return (n >> 3) * 1024 + (n & 7) * 128 + ((c ^ (n & 7)) << 4);
   return (n >> 3) * 512 + (n & 7) * 64 + ((c ^ ((n >> 1) & 3)) << 4);
 }
+__device__ __forceinline__ uint64_t tile_desc(uint32_t start) {
+  return kRowBytes == 128 ? ptx::sw128_desc(start) : ptx::sw64_desc(start);
+}
 
-// Byte offset of the words of group g (inputs 32g..32g+31) of weight tile mt:
-// [word][128 rows], contiguous wpg*512 bytes.
+// Byte offset of the words of groups g..g+kGroups-1 (inputs 32g..) of weight tile
+// mt: [group][word][128 rows], contiguous kGroups*wpg*512 bytes (g % kGroups == 0).
 __device__ __forceinline__ uint64_t code_stage_offset(int mt, int g, int K, int wpg) {
   return ((((uint64_t)mt * (uint64_t)(K >> 7) + (uint64_t)(g >> 2)) * 4u + (uint64_t)(g & 3)) * (uint64_t)wpg *
           128u) * 4u;
 }
-// Byte offset of the scales of group g of weight tile mt (256 contiguous bytes).
+// Byte offset of the scales of groups g..g+kGroups-1 of weight tile mt (kGroups*256 bytes).
 __device__ __forceinline__ uint64_t scale_stage_offset(int mt, int g, int K, int fmt) {
   if (fmt == MOE_FMT_NVFP4) return ((uint64_t)mt * (uint64_t)(K >> 4) + (uint64_t)g * 2u) * 128u;
   return ((uint64_t)mt * (uint64_t)(K >> 5) + (uint64_t)g) * 256u;
+}
+
+// Dequantize every stage of one work item (formats F0 = first matrix, F1 =
+// second): wait for the stage's codes, convert this thread's units, publish
+// them to the tensor core and release the stage to the MMA warp.  Returns
+// false if a bounded wait gave up.
+template <int NMAT, int F0, int F1>
+__device__ __noinline__ bool dequant_item(uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
+                                          volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
+                                          uint32_t& phase, int& gstage, unsigned long long* trace) {
+  using C = TcCfg<NMAT>;
+  constexpr int kUnits = NMAT * kGroups * 4 / kThreadsPerRow;
+  static_assert(NMAT == 1 || kUnits % 2 == 0, "units must alternate matrices evenly");
+  const int lane = threadIdx.x & 31;
+  const int cg0 = u0 / NMAT;
+  for (int ks = 0; ks < ksteps; ++ks) {
+    if (!__all_sync(0xffffffffu, ptx::mbar_wait(&load_full[stage], phase, abort_flag, kWaitLimit))) return false;
+    if (threadIdx.x == 0) trace_stamp(trace, 2, gstage);
+    uint8_t* sb = smem + stage * C::kStageBytes;
+    uint4 v[kUnits];
+#pragma unroll
+    for (int i = 0; i < kUnits; ++i) {
+      const int m = i % NMAT, cg = cg0 + i / NMAT, g = cg >> 2;
+      const uint8_t* scales = sb + C::kOffScales + m * C::kScaleBytes + g * 256;
+      if (m == 0) {
+        const uint32_t* codes = reinterpret_cast<const uint32_t*>(sb + C::kOffCodes) + g * fmt_words(F0) * 128;
+        v[i] = dequant_chunk<F0>(codes, scales, n, cg & 3);
+      } else {
+        const uint32_t* codes = reinterpret_cast<const uint32_t*>(sb + C::kOffCodes + C::kCodeBytes) +
+                                g * fmt_words(F1) * 128;
+        v[i] = dequant_chunk<F1>(codes, scales, n, cg & 3);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kUnits; ++i) {
+      const int m = i % NMAT, cg = cg0 + i / NMAT;
+      *reinterpret_cast<uint4*>(sb + C::kOffA + m * C::kABytes + tile_offset(n, cg)) = v[i];
+    }
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&a_full[stage]);
+    if (threadIdx.x == 0) trace_stamp(trace, 3, gstage);
+    ++gstage;
+    if (++stage == C::kStages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+  return true;
+}
+
+// Runtime format pair -> the matching dequant_item instantiation.
+template <int NMAT, int F0>
+__device__ __forceinline__ bool dequant_item_f1(int f1, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
+                                                volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
+                                                uint32_t& phase, int& gstage, unsigned long long* trace) {
+  if (NMAT == 1) return dequant_item<NMAT, F0, F0>(smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+  switch (f1) {
+    case MOE_FMT_INT2: return dequant_item<NMAT, F0, MOE_FMT_INT2>(smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT3: return dequant_item<NMAT, F0, MOE_FMT_INT3>(smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT4: return dequant_item<NMAT, F0, MOE_FMT_INT4>(smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    default: return dequant_item<NMAT, F0, MOE_FMT_NVFP4>(smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+  }
+}
+template <int NMAT>
+__device__ __forceinline__ bool dequant_item_any(int f0, int f1, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
+                                                 volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
+                                                 uint32_t& phase, int& gstage, unsigned long long* trace) {
+  switch (f0) {
+    case MOE_FMT_INT2: return dequant_item_f1<NMAT, MOE_FMT_INT2>(f1, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT3: return dequant_item_f1<NMAT, MOE_FMT_INT3>(f1, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT4: return dequant_item_f1<NMAT, MOE_FMT_INT4>(f1, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    default: return dequant_item_f1<NMAT, MOE_FMT_NVFP4>(f1, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+  }
 }
 
 template <int NMAT>
@@ -163,11 +261,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       ptx::mbar_init(&load_full[s], 1);
-      ptx::mbar_init(&a_full[s], kDeqThreads);
+      ptx::mbar_init(&a_full[s], kDeqWarps);  // one arrival per dequant warp
       ptx::mbar_init(&stage_empty[s], 1);
     }
     ptx::mbar_init(acc_full, 1);
-    ptx::mbar_init(acc_empty, kDeqThreads);
+    ptx::mbar_init(acc_empty, kDeqWarps);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -195,43 +293,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   };
 
   if (warp == kTmaWarp) {
-    int stage = 0;
+    int stage = 0, gstage = 0;
     uint32_t phase = 0;
     uint32_t issued = 0, issued_phase = 0;  // per stage: a load was armed, and its parity
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const int c = t / m_tiles, mt = t % m_tiles;
       const int e = a.chunks[3 * c], row0 = a.chunks[3 * c + 1];
-      const uint8_t* cbase[NMAT];
-      const uint8_t* sbase[NMAT];
-      int fmt[NMAT];
+      // A weight tile's codes (and scales) are contiguous along K, so each stage's
+      // slice is the tile base plus ks times a fixed stride.
+      const uint8_t* cptr[NMAT];
+      const uint8_t* sptr[NMAT];
+      uint32_t cbytes[NMAT];
       uint32_t bytes = C::kBBytes;
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) {
         const int i = e * 3 + a.proj + m;
-        fmt[m] = L.fmt[i];
-        cbase[m] = L.base + L.code_off[i];
-        sbase[m] = L.base + L.scale_off[i];
-        bytes += (uint32_t)fmt_words(fmt[m]) * 512u + (uint32_t)C::kScaleBytes;
+        const int f = L.fmt[i];
+        cbytes[m] = (uint32_t)(fmt_words(f) * 512 * kGroups);
+        cptr[m] = L.base + L.code_off[i] + code_stage_offset(mt, 0, a.K, fmt_words(f));
+        sptr[m] = L.base + L.scale_off[i] + scale_stage_offset(mt, 0, a.K, f);
+        bytes += cbytes[m] + (uint32_t)C::kScaleBytes;
       }
       for (int ks = 0; ks < ksteps; ++ks) {
+        if (lane == 0 && ks + kPrefetchAhead < ksteps) {  // warm L2 with the codes a few stages ahead
+#pragma unroll
+          for (int m = 0; m < NMAT; ++m)
+            ptx::prefetch_l2(cptr[m] + (size_t)(ks + kPrefetchAhead) * cbytes[m], cbytes[m]);
+        }
         if (!wait_all(&stage_empty[stage], phase ^ 1u)) {
           ok = false;
           break;
         }
         if (lane == 0) {
+          trace_stamp(a.trace, 0, gstage);
           uint8_t* sb = smem + stage * C::kStageBytes;
           ptx::mbar_arrive_expect_tx(&load_full[stage], bytes);
           ptx::tma_load_2d(sb + C::kOffB, &tmap_b, ks * kTcBK, row0, &load_full[stage]);
 #pragma unroll
           for (int m = 0; m < NMAT; ++m) {
-            const int wpg = fmt_words(fmt[m]);
-            ptx::bulk_load(sb + C::kOffCodes + m * C::kCodeBytes, cbase[m] + code_stage_offset(mt, ks, a.K, wpg),
-                           (uint32_t)wpg * 512u, &load_full[stage]);
-            ptx::bulk_load(sb + C::kOffScales + m * C::kScaleBytes,
-                           sbase[m] + scale_stage_offset(mt, ks, a.K, fmt[m]), (uint32_t)C::kScaleBytes,
+            ptx::bulk_load(sb + C::kOffCodes + m * C::kCodeBytes, cptr[m] + (size_t)ks * cbytes[m], cbytes[m],
                            &load_full[stage]);
+            ptx::bulk_load(sb + C::kOffScales + m * C::kScaleBytes, sptr[m] + (size_t)ks * C::kScaleBytes,
+                           (uint32_t)C::kScaleBytes, &load_full[stage]);
           }
+          trace_stamp(a.trace, 1, gstage);
         }
+        ++gstage;
         __syncwarp();
         issued |= 1u << stage;
         issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -246,7 +353,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (issued & (1u << s)) ptx::mbar_wait(&load_full[s], (issued_phase >> s) & 1u, abort_flag, kWaitLimit / 4);
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    int stage = 0;
+    int stage = 0, gstage = 0;
     uint32_t phase = 0, acc_phase = 0;
     const uint32_t sbase = ptx::smem_u32(smem);
     bool committed = false;
@@ -267,16 +374,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         ptx::tc_fence_after();
+        if (lane == 0) trace_stamp(a.trace, 4, gstage);
         if (lane == 0) {
           const uint32_t st = sbase + (uint32_t)(stage * C::kStageBytes);
 #pragma unroll
           for (int m = 0; m < NMAT; ++m)
 #pragma unroll
             for (int k16 = 0; k16 < kTcBK / 16; ++k16)
-              ptx::mma_f16_ss(tmem + (uint32_t)(m * 256), ptx::sw64_desc(st + C::kOffA + m * C::kABytes + k16 * 32),
-                              ptx::sw64_desc(st + C::kOffB + k16 * 32), idesc, (ks | k16) != 0);
+              ptx::mma_f16_ss(tmem + (uint32_t)(m * 256), tile_desc(st + C::kOffA + m * C::kABytes + k16 * 32),
+                              tile_desc(st + C::kOffB + k16 * 32), idesc, (ks | k16) != 0);
           ptx::mma_commit(&stage_empty[stage]);
+          trace_stamp(a.trace, 5, gstage);
         }
+        ++gstage;
         __syncwarp();
         committed = true;
         if (++stage == C::kStages) {
@@ -296,13 +406,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------- dequant + epilogue
-    // gate/up: thread -> (matrix t/128, row t%128), all 4 chunks of the group;
-    // down: thread -> (chunk pair t/128, row t%128), 2 chunks.
+    // kThreadsPerRow threads per weight row n.  The row's units of a stage (chunk
+    // of 8 inputs x matrix, matrices alternating) are split evenly: thread
+    // sel = tid/128 takes kUnits consecutive units, as many of each matrix.
     const int n = threadIdx.x & 127, sel = threadIdx.x >> 7;
-    const int q = warp & 3, chalf = warp >> 2;
-    int stage = 0;
+    constexpr int kColGroups = kDeqWarps / 4;            // epilogue column groups
+    constexpr int kColsPerWarp = kTcBN / kColGroups;
+    const int q = warp & 3, cq = warp >> 2;               // epilogue: TMEM lane quarter, column group
+    constexpr int kUnits = NMAT * kGroups * 4 / kThreadsPerRow;
+    const int u0 = sel * kUnits;
+    int stage = 0, gstage = 0, item = 0;
     uint32_t phase = 0, acc_phase = 0;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++item) {
       const int c = t / m_tiles, mt = t % m_tiles;
       const int e = a.chunks[3 * c], row0 = a.chunks[3 * c + 1], rows = a.chunks[3 * c + 2];
       int fmt[NMAT];
@@ -313,29 +428,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         fmt[m] = L.fmt[i];
         tsc[m] = fmt[m] == MOE_FMT_NVFP4 ? L.tscale[i] : 1.0f;
       }
-      const int my_m = NMAT == 2 ? sel : 0;
-      const int my_fmt = (NMAT == 2 && sel) ? fmt[NMAT - 1] : fmt[0];
-      for (int ks = 0; ks < ksteps; ++ks) {
-        if (!wait_all(&load_full[stage], phase)) {
-          ok = false;
-          break;
-        }
-        uint8_t* sb = smem + stage * C::kStageBytes;
-        const uint32_t* codes = reinterpret_cast<const uint32_t*>(sb + C::kOffCodes + my_m * C::kCodeBytes);
-        const uint8_t* scales = sb + C::kOffScales + my_m * C::kScaleBytes;
-        uint8_t* A = sb + C::kOffA + my_m * C::kABytes;
-        constexpr int kChunks = NMAT == 2 ? 4 : 2;
-#pragma unroll
-        for (int i = 0; i < kChunks; ++i) {
-          const int ch = NMAT == 2 ? i : 2 * sel + i;
-          *reinterpret_cast<uint4*>(A + sw64_offset(n, ch)) = dequant_chunk(my_fmt, codes, scales, n, ch);
-        }
-        ptx::fence_proxy_async_smem();
-        ptx::mbar_arrive(&a_full[stage]);
-        if (++stage == C::kStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
+      if (!dequant_item_any<NMAT>(fmt[0], fmt[NMAT - 1], smem, load_full, a_full, abort_flag, ksteps, n, u0, stage,
+                                  phase, gstage, a.trace)) {
+        ok = false;
+        break;
       }
       if (!ok) break;
       if (!wait_all(acc_full, acc_phase)) {
@@ -343,16 +439,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         break;
       }
       acc_phase ^= 1u;
+      if (threadIdx.x == 0) trace_stamp(a.trace, 6, item);
       ptx::tc_fence_after();
       const int nrow = mt * kTcBM + q * 32 + lane;
       const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-      for (int cb = chalf * 128; cb < chalf * 128 + 128 && cb < rows; cb += 32) {
-        uint32_t r0[32], r1[32];
-        ptx::tmem_ld32(lane_base + (uint32_t)cb, r0);
-        if (NMAT == 2) ptx::tmem_ld32(lane_base + 256u + (uint32_t)cb, r1);
+      for (int cb = cq * kColsPerWarp; cb < cq * kColsPerWarp + kColsPerWarp && cb < rows; cb += 16) {
+        uint32_t r0[16], r1[16];
+        ptx::tmem_ld16(lane_base + (uint32_t)cb, r0);
+        if (NMAT == 2) ptx::tmem_ld16(lane_base + 256u + (uint32_t)cb, r1);
         ptx::tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < 16; ++j) {
           const int tok = cb + j;
           if (tok >= rows) break;
           const int r = row0 + tok;
@@ -374,7 +471,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       ptx::tc_fence_before();
-      ptx::mbar_arrive(acc_empty);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(acc_empty);
+      if (threadIdx.x == 0) trace_stamp(a.trace, 7, item);
     }
   }
 
@@ -422,9 +521,10 @@ cudaError_t launch_tc(const TcArgs& a, const void* act, int rows_total, cudaStre
   const cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)rows_total};
   const cuuint64_t strides[1] = {(cuuint64_t)a.K * 2u};
   const cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)kTcBN};
+  const CUtensorMapSwizzle swz = kRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   const cuuint32_t estr[2] = {1u, 1u};
   if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(act), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   auto kern = expert_gemm_tc_kernel<NMAT>;
@@ -437,8 +537,9 @@ cudaError_t launch_tc(const TcArgs& a, const void* act, int rows_total, cudaStre
 }  // namespace
 
 cudaError_t launch_expert_gemm_tc(const uint8_t* packed, int E, int H, int F, int T, int k, bool fp4, bool gateup,
-                                  const Workspace& ws, int32_t* status, cudaStream_t stream) {
+                                  const Workspace& ws, int32_t* status, uint64_t* trace, cudaStream_t stream) {
   TcArgs a{};
+  a.trace = gateup ? reinterpret_cast<unsigned long long*>(trace) : nullptr;
   a.packed = packed;
   a.E = E;
   a.H = H;

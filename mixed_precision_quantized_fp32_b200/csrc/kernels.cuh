@@ -25,7 +25,7 @@ cudaError_t launch_expert_gemm_mma(const uint8_t* packed, int E, int H, int F, i
                                    int chunk_rows, int max_chunks, const Workspace& ws, cudaStream_t stream);
 
 cudaError_t launch_expert_gemm_tc(const uint8_t* packed, int E, int H, int F, int T, int k, bool fp4, bool gateup,
-                                  const Workspace& ws, int32_t* status, cudaStream_t stream);
+                                  const Workspace& ws, int32_t* status, uint64_t* trace, cudaStream_t stream);
 
 cudaError_t launch_combine(int T, int k, int H, const Workspace& ws, __nv_bfloat16* y, cudaStream_t stream);
 
