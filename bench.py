@@ -297,6 +297,72 @@ def run_ours(args, rank, world, local_rank):
     return out, layer
 
 
+# ------------------------------------------------------------------ all layers (report)
+def matrix_bytes(L: W.Layer, e: int, p: int) -> float:
+    f = int(L.fmt[e, p])
+    n = L.F * L.H
+    return n * (4 if f == 16 else f) / 8 + n / 16
+
+
+def run_suite(args):
+    """Every layer of the workload set, decode and prefill batches: tokens/s and the
+    roofline of the gate/up and down kernels.  One JSON line per batch."""
+    import torch
+
+    import mixed_precision_quantized_fp32_b200 as moe
+    dev = torch.device("cuda", 0)
+    pk, _ = peaks()
+    nev = moe.MOE_STAGE_EVENTS
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    for name in args.suite.split(","):
+        L = W.layer(name)
+        layer = gpu_pack(L, moe, dev)
+        Wr, b = W.device_router(L)
+        for T in list(L.decode_T) + list(L.prefill_T):
+            decode = T in L.decode_T
+            x = torch.empty((T, L.H), dtype=torch.bfloat16, device=dev)
+            W.fill_device_bf16(x, 0, W.TID_X, 1.0)
+            ws = moe.alloc_packed(moe.workspace_bytes(layer, T, L.k), dev)
+            cnt = torch.zeros(L.E, dtype=torch.int32, device=dev)
+            moe.moe_layer_forward(x, Wr, b, layer, L.k, ws=ws, debug={"counts": cnt})
+            torch.cuda.synchronize()
+            counts = cnt.cpu().numpy()
+            active = np.nonzero(counts)[0]
+            n = 10
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(n)]
+            for row in ev:
+                for e_ in row:
+                    e_.record()
+            for _ in range(3):
+                moe.moe_layer_forward(x, Wr, b, layer, L.k, ws=ws)
+            for i in range(n):
+                if decode:
+                    flush.zero_()
+                moe.moe_layer_forward(x, Wr, b, layer, L.k, ws=ws, stage_events=ev[i])
+            torch.cuda.synchronize()
+            st = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(nev - 1)] for i in range(n)]).mean(0)
+            step = float(np.mean([ev[i][0].elapsed_time(ev[i][-1]) for i in range(n)]))
+            gu, dn = float(st[3]), float(st[5])
+            out = {"layer": name, "T": T, "mode": "decode" if decode else "prefill", "tokens_per_s": round(T / step * 1e3, 1),
+                   "ms_per_step": round(step, 4), "active_experts": int(len(active)),
+                   "stages_ms": dict(zip(["router_topk", "permute", "gather", "gateup", "h_quant", "down", "combine"],
+                                         [round(float(v), 4) for v in st]))}
+            if decode:
+                bg = sum(matrix_bytes(L, int(e), 0) + matrix_bytes(L, int(e), 1) for e in active)
+                bd = sum(matrix_bytes(L, int(e), 2) for e in active)
+                out["gateup"] = {"GB/s": round(bg / gu / 1e6, 1), "frac_hbm": round(bg / gu / 1e6 / pk["hbm_gbs"], 4)}
+                out["down"] = {"GB/s": round(bd / dn / 1e6, 1), "frac_hbm": round(bd / dn / 1e6 / pk["hbm_gbs"], 4)}
+                out["layer_GB/s_weights"] = round((bg + bd) / step / 1e6, 1)
+            else:
+                fl = 2.0 * T * L.k * L.H * L.F
+                out["gateup"] = {"TFLOP/s": round(2 * fl / gu / 1e9, 1), "frac_tensor": round(2 * fl / gu / 1e9 / pk["bf16_tflops"], 4)}
+                out["down"] = {"TFLOP/s": round(fl / dn / 1e9, 1), "frac_tensor": round(fl / dn / 1e9 / pk["bf16_tflops"], 4)}
+            print(json.dumps(out), flush=True)
+            del ws, x
+        del layer
+        torch.cuda.empty_cache()
+
+
 # ------------------------------------------------------------------ oracle (CPU) timing
 class OracleSample:
     """The CPU oracle on a bounded sample (the first n tokens) of a batch."""
@@ -379,7 +445,12 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--suite", default="", help="comma-separated layers to report instead of the contract line "
+                                                "(tiny,mixtral,hotcold,nvfp4,large)")
     args = ap.parse_args()
+    if args.suite:
+        run_suite(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
 

@@ -48,13 +48,14 @@ struct Plan {
   bool tc;         // tcgen05 expert GEMMs (many rows per expert) or warp-MMA (few rows per expert)
 };
 
-// Few rows per expert (decode): 16-row chunks on the warp-level MMA kernel.
-// Many rows per expert (prefill): 256-row chunks on the tcgen05 kernel.
+// Few rows per expert (decode): chunks of 8 (or 16 when the batch averages more
+// than 8 rows per expert) on the register GEMV (warp MMA).  Many rows per expert
+// (prefill): 256-row chunks on the tcgen05 kernel.
 Plan make_plan(int T, int k, int E) {
   Plan p;
   const long long R = (long long)T * k;
   p.tc = R > 16LL * E && R >= 256;
-  p.chunk_rows = p.tc ? 256 : 16;
+  p.chunk_rows = p.tc ? 256 : (R <= 8LL * E ? 8 : 16);
   p.max_chunks = (int)(E + (R + p.chunk_rows - 1) / p.chunk_rows);
   return p;
 }
@@ -177,8 +178,7 @@ extern "C" moe_status moe_layer_forward(const void* x, int32_t T, const float* r
   int32_t* status = d.status ? d.status : wsp.status;
   auto gemm = [&](bool gateup) -> cudaError_t {
     return plan.tc ? launch_expert_gemm_tc(packed, E, H, F, T, k, fp4, gateup, wsp, status, d.trace, stream)
-                   : launch_expert_gemm_mma(packed, E, H, F, k, fp4, gateup, plan.chunk_rows, plan.max_chunks, wsp,
-                                            stream);
+                   : launch_expert_gemv(packed, E, H, F, k, fp4, gateup, plan.max_chunks, plan.chunk_rows, wsp, stream);
   };
   if (gemm(true) != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(4)) return MOE_ERR_CUDA;

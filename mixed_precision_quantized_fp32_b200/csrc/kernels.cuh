@@ -21,11 +21,11 @@ cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4,
 cudaError_t launch_act_quant_h(int R, int F, const Workspace& ws, uint8_t* dbg_hq, float* dbg_sh,
                                cudaStream_t stream);
 
-cudaError_t launch_expert_gemm_mma(const uint8_t* packed, int E, int H, int F, int k, bool fp4, bool gateup,
-                                   int chunk_rows, int max_chunks, const Workspace& ws, cudaStream_t stream);
-
 cudaError_t launch_expert_gemm_tc(const uint8_t* packed, int E, int H, int F, int T, int k, bool fp4, bool gateup,
                                   const Workspace& ws, int32_t* status, uint64_t* trace, cudaStream_t stream);
+
+cudaError_t launch_expert_gemv(const uint8_t* packed, int E, int H, int F, int k, bool fp4, bool gateup,
+                               int max_chunks, int chunk_rows, const Workspace& ws, cudaStream_t stream);
 
 cudaError_t launch_combine(int T, int k, int H, const Workspace& ws, __nv_bfloat16* y, cudaStream_t stream);
 
