@@ -76,6 +76,27 @@ def ncu_traffic(kernel_key: str):
     return None if v is None else v.get("dram_bytes_per_launch")
 
 
+# ------------------------------------------------------------------ replicas (N > 1)
+def replica_seed(rank: int) -> int:
+    """Seed of rank `rank`'s tokens: every replica runs its own batch of the same layer."""
+    return rank
+
+
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """Max over ranks of a per-rank duration; every rank calls it at the same point."""
+    if world <= 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: the tokens all ranks processed over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (max_ms / 1e3)
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     def __init__(self, device_index: int):
@@ -160,7 +181,7 @@ def run_ours(args, rank, world, local_rank):
     T = 2048
     layer = gpu_pack(L, moe, dev)
     x = torch.empty((T, L.H), dtype=torch.bfloat16, device=dev)
-    W.fill_device_bf16(x, rank, W.TID_X, 1.0)   # each replica its own tokens
+    W.fill_device_bf16(x, replica_seed(rank), W.TID_X, 1.0)   # each replica its own tokens
     Wr, b = W.device_router(L)
     ws = moe.alloc_packed(moe.workspace_bytes(layer, T, L.k), dev)
     y = torch.empty_like(x)
@@ -193,12 +214,8 @@ def run_ours(args, rank, world, local_rank):
     step_ms = [evs[s][0].elapsed_time(evs[s][-1]) for s in range(args.steps)]
     stage_ms = np.array([[evs[s][i].elapsed_time(evs[s][i + 1]) for i in range(nev - 1)]
                          for s in range(args.steps)])
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * T * args.steps / (total_ms / 1e3)
+    total_ms = max_over_ranks(float(sum(step_ms)), world, dev)
+    value = job_tokens_per_s(T, args.steps, world, total_ms)
 
     # ---- end to end through the public API with host buffers (pinned)
     x_host = x.cpu().pin_memory()
@@ -219,12 +236,8 @@ def run_ours(args, rank, world, local_rank):
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * T * args.steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = job_tokens_per_s(T, args.steps, world, e2e_ms)
 
     # ---- roofline of the dominant kernel (gate/up GEMM with the SwiGLU epilogue)
     pk, pk_kind = peaks()
@@ -249,7 +262,7 @@ def run_ours(args, rank, world, local_rank):
         eb = expert_gateup_bytes(L, moe)
         for Td in (1, 8, 64):
             xd = torch.empty((Td, L.H), dtype=torch.bfloat16, device=dev)
-            W.fill_device_bf16(xd, rank, W.TID_X, 1.0)
+            W.fill_device_bf16(xd, replica_seed(rank), W.TID_X, 1.0)
             wsd = moe.alloc_packed(moe.workspace_bytes(layer, Td, L.k), dev)
             cnt = torch.zeros(L.E, dtype=torch.int32, device=dev)
             moe.moe_layer_forward(xd, Wr, b, layer, L.k, ws=wsd, debug={"counts": cnt})
@@ -319,6 +332,8 @@ def run_suite(args):
         layer = gpu_pack(L, moe, dev)
         Wr, b = W.device_router(L)
         for T in list(L.decode_T) + list(L.prefill_T):
+            if args.batch and T != args.batch:
+                continue
             decode = T in L.decode_T
             x = torch.empty((T, L.H), dtype=torch.bfloat16, device=dev)
             W.fill_device_bf16(x, 0, W.TID_X, 1.0)
@@ -447,6 +462,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--suite", default="", help="comma-separated layers to report instead of the contract line "
                                                 "(tiny,mixtral,hotcold,nvfp4,large)")
+    ap.add_argument("--batch", type=int, default=0, help="with --suite: only this batch size")
     args = ap.parse_args()
     if args.suite:
         run_suite(args)
