@@ -164,13 +164,18 @@ typedef struct {
                                 router+top-k, permutation, activation gather/quantization,
                                 gate/up GEMM, h quantization (NVFP4), down GEMM, combine,
                                 and after combine, so stage times can be read back */
-  uint64_t* trace;    /* [MOE_TRACE_WORDS] or NULL: diagnostics of the tcgen05 gate/up GEMM
-                         (batches with many rows per expert): clock64 stamps taken by CTA 0,
-                         MOE_TRACE_EVENTS rows of MOE_TRACE_STAGES pipeline stages; row 0:
-                         producer got a free stage, 1: producer issued its copies, 2: dequant
-                         warp 0 saw the stage land, 3: dequant warp 0 released it, 4: MMA lane
-                         saw it ready, 5: MMA issued and committed it; row 6 holds, per work
-                         item, the epilogue start, row 7 its end.  Zero it before the call. */
+  uint64_t* trace;    /* [MOE_TRACE_WORDS] or NULL: diagnostics of the gate/up expert GEMM:
+                         clock64 stamps taken by CTA 0, MOE_TRACE_EVENTS rows of
+                         MOE_TRACE_STAGES entries.  Zero it before the call.
+                         tcgen05 GEMM (many rows per expert), per pipeline stage: row 0
+                         producer got a free stage, 1 producer issued its copies, 2 dequant
+                         warp 0 saw the stage land, 3 dequant warp 0 released it, 4 MMA lane
+                         saw it ready, 5 MMA issued and committed it; per work item: row 6
+                         epilogue start, row 7 its end.
+                         Decode GEMV (few rows per expert), per weight tile: row 0 producer got
+                         a free stage, 1 producer issued its copies, 2 consumer warp 0 found it
+                         landed, 3 consumer warp 0 released it; per work item: row 4 producer
+                         loaded the following item, 6 consumers started it, 7 finished it. */
 } moe_debug;
 
 #define MOE_TRACE_EVENTS 8

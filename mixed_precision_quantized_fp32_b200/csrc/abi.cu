@@ -48,14 +48,16 @@ struct Plan {
   bool tc;         // tcgen05 expert GEMMs (many rows per expert) or warp-MMA (few rows per expert)
 };
 
-// Few rows per expert (decode): chunks of 8 (or 16 when the batch averages more
-// than 8 rows per expert) on the register GEMV (warp MMA).  Many rows per expert
+// Few rows per expert (decode): chunks of 8 or 16 rows (by the average rows per
+// active expert) on the streaming GEMV (warp MMA).  Many rows per expert
 // (prefill): 256-row chunks on the tcgen05 kernel.
 Plan make_plan(int T, int k, int E) {
   Plan p;
   const long long R = (long long)T * k;
-  p.tc = R > 16LL * E && R >= 256;
-  p.chunk_rows = p.tc ? 256 : (R <= 8LL * E ? 8 : 16);
+  const long long active = R < E ? R : E;
+  const long long avg = active > 0 ? (R + active - 1) / active : 0;
+  p.tc = avg > 32 && R >= 256;
+  p.chunk_rows = p.tc ? 256 : (avg <= 3 ? 8 : 16);
   p.max_chunks = (int)(E + (R + p.chunk_rows - 1) / p.chunk_rows);
   return p;
 }
@@ -95,6 +97,18 @@ uint64_t carve(uint8_t* base, int T, int k, int E, int H, int F, bool fp4, const
     ws.sh = (float*)take(R * 4);
   }
   ws.o = (float*)take(R * H * 4);
+  if (!plan.tc) {
+    const int pg = gemv_split((long long)R, E, F, H, 2), pd = gemv_split((long long)R, E, H, F, 1);
+    const uint64_t part_g = pg > 1 ? (uint64_t)pg * R * 2 * F : 0, part_d = pd > 1 ? (uint64_t)pd * R * H : 0;
+    const uint64_t part = part_g > part_d ? part_g : part_d;
+    if (part) ws.part = (float*)take(part * 4);
+    ws.counter_len = 2;  // work counters of the gate/up and down GEMVs
+    ws.counters = (int32_t*)take((uint64_t)ws.counter_len * 4);
+    if (!fp4) {
+      ws.xsum = (float*)take(R * (H / 32) * 4);
+      ws.hsum = (float*)take(R * (F / 32) * 4);
+    }
+  }
   if (w) *w = ws;
   return pos;
 }
@@ -178,7 +192,9 @@ extern "C" moe_status moe_layer_forward(const void* x, int32_t T, const float* r
   int32_t* status = d.status ? d.status : wsp.status;
   auto gemm = [&](bool gateup) -> cudaError_t {
     return plan.tc ? launch_expert_gemm_tc(packed, E, H, F, T, k, fp4, gateup, wsp, status, d.trace, stream)
-                   : launch_expert_gemv(packed, E, H, F, k, fp4, gateup, plan.max_chunks, plan.chunk_rows, wsp, stream);
+                   : launch_expert_gemv(packed, w->packed_bytes, w->fmt, E, H, F, T * k, k, fp4, gateup,
+                                        plan.max_chunks, plan.chunk_rows, wsp, status, gateup ? d.trace : nullptr,
+                                        stream);
   };
   if (gemm(true) != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(4)) return MOE_ERR_CUDA;

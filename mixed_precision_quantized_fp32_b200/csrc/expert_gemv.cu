@@ -1,55 +1,135 @@
 // Dequant-fused grouped expert GEMV for batches with few token rows per expert
-// (decode: 1-16 rows), bound by streaming the active experts' packed weights
-// from HBM (the pages' observation that only the active experts' weights are
-// read, and the packed-linear operator of the MoE mixed-precision page, sec.
-// 2.3 / 3.5).
+// (decode: up to 16 rows per chunk), bound by streaming the active experts'
+// packed weights from HBM.  It follows the pages' observation that a token only
+// needs its active experts' weights, and implements the packed-linear operator
+// of the MoE mixed-precision page (sec. 2.3 / 3.5).
 //
-// Work item: (chunk of <= 16 expert-sorted rows of one expert, 32 weight rows).
-// A persistent CTA of kWarps warps walks its work items; every warp owns a
-// fixed 1/kWarps of the inputs of each item (split-K inside the CTA, summed
-// through shared memory when the item ends).  Per group of 32 inputs a thread
-// (g = lane/4, c = lane%4) needs word c of four consecutive weight rows of each
-// matrix, their scales and eight activations per token tile; it copies them
-// with cp.async straight into its own slots of a shared-memory ring that runs
-// kStages groups ahead, across item boundaries, so each SM keeps well over
-// 100 KB of weight loads in flight without spending registers on them.
+// Work item: (chunk of <= 8*NT8 expert-sorted token rows of one expert, block
+// of 128 weight rows, part p of P along K).  Persistent CTAs take items from a
+// global counter, so uneven items balance across SMs.  Warp 4 streams each
+// 128-input tile of the block through a ring of shared-memory stages:
+//   * the packed codes: two 3D TMA loads per matrix, with a 128-byte swizzle so
+//     the 16-byte code reads below are bank-conflict free;
+//   * the group scales: one bulk copy;
+//   * the token rows and their per-group sums: 2D TMA loads.
+// None is multicast.  Warps 0-3 own 32 weight rows each.
 //
-// Compute per group: the codes 8c..8c+7 of a row become four fp16 pairs
-// (exponent-bias unpack: code u OR'ed into the mantissa of 1024.0 gives 1024+u
-// exactly, minus 1024+offset exactly) that are the A fragments of two
-// mma.sync m16n8k16 per 16-row tile.  The input order inside an MMA is permuted
-// consistently for both operands: thread c supplies inputs 8c..8c+7 of the
-// group for A and the same eight activations for B.  Integer groups are scaled
-// after their MMAs (one fp32 FMA per output); NVFP4 codes are multiplied by
-// their e4m3 block scale before (exact in fp16).
+// Per group of 32 inputs, lane (g, c) holds word(s) of rows 4g..4g+3 covering
+// inputs 8c..8c+7.  It turns each pair of codes into one fp16x2 A-fragment
+// register with one AND (INT3: three ALU ops that merge the high-bit plane):
+//   * the masked field is read as an fp16 subnormal: a code u in a field of
+//     power-of-two weight f (bit position 2j or 4j of a half-word) is exactly
+//     u * f * 2^-24;
+//   * the matching activation is prescaled by 1/f (exact), so each product is
+//     x * u * 2^-24;
+//   * the code offset 2^(b-1) is removed through the MMA's C input:
+//     -offset * 2^-24 * (sum of the group's activations), precomputed per token
+//     row and group when the activations are written.
+// Each group's fp32 MMA result is scaled by its fp16 group scale, and 2^24 is
+// restored at the end.  NVFP4 codes become exact fp16 with cvt.e2m1x2 times
+// their e4m3 block scale and accumulate directly.
+//
+// Split-K (P > 1, for batches with too few blocks to fill the GPU) writes
+// per-part fp32 partials; a small follow-up kernel sums the parts in a fixed
+// order and runs the epilogue.  There are no atomics or fences between CTAs and
+// results do not depend on timing.  Every mbarrier wait is bounded; a wait that
+// gives up sets MOE_ERR_TIMEOUT in the status word.
+#include <cudaTypedefs.h>
+
 #include "moe_common.cuh"
 #include "kernels.cuh"
+#include "tc_ptx.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kRowsPerCta = 32;
-constexpr int kWarps = 4;          // K-split warps per CTA
-constexpr int kTokMax = 16;        // token rows per chunk
-constexpr int kStages = 4;         // ring stages per warp (kStages-1 groups in flight)
-constexpr int kPartStride = kTokMax + 1;
+constexpr int kBlockRows = 128;                 // weight rows per work item (one packed tile row)
+constexpr int kConsumers = 4;                   // consumer warps, 32 weight rows each
+constexpr int kProducer = kConsumers;           // warp index of the TMA warp
+constexpr int kGemvThreads = 32 * (kConsumers + 1);
+constexpr long long kGemvWait = 2000000000LL;   // clock cycles, ~1 s
+constexpr int kMaxSplit = 16;
+constexpr int kMaxStages = 32;
+constexpr int kCtrlBytes = 3072;                // barriers, item descriptors and flags after the ring
 
-__device__ __forceinline__ uint32_t h2sub_u(uint32_t a, uint32_t b) {
-  __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
-  return *reinterpret_cast<uint32_t*>(&r);
+// Shared-memory stage (sizes fixed per launch from the layer's widest formats):
+//   [matrix m: code box 0 | code box 1] [scales m] ... [token rows x 128 fp16]
+//   [token rows x 4 group sums fp32]
+// A code box holds 4 groups x wpg words x 2 row slices x 128 bytes (1024 * wpg).
+struct StageLayout {
+  int box[2];        // bytes of one code box of matrix 0 / 1
+  int code_off[2];   // offset of matrix m's first box
+  int scale_off[2];  // offset of matrix m's scales (1024 bytes)
+  int x_off;         // offset of the token rows
+  int sum_off;       // offset of the group sums (integer layers)
+  int bytes;         // stage size (multiple of 1024)
+  int stages;        // ring depth
+};
+
+struct GemvArgs {
+  const uint8_t* packed;
+  int E, H, F;
+  int N, K;               // weight rows and inputs of this projection
+  int proj;               // 0: gate+up with the SwiGLU epilogue; 2: down
+  int topk;
+  int P;                  // K parts
+  int R;                  // expert rows in the batch (T*k)
+  const int32_t* chunks;  // (expert, first row, rows)
+  const int32_t* chunk_count;
+  const float* row_scale; // NVFP4: gate/up -> per-token sx, down -> per-row sh; null for integer layers
+  const int32_t* perm;
+  bool sums;              // integer layer: activation group sums are loaded with the tiles
+  void* out;              // gate/up: h [R][F] (fp16, or fp32 for NVFP4); down: o fp32 [R][H]
+  float* out_sum;         // gate/up, integer layers: group sums of h [R][F/32]
+  float* part;            // [P][R][NMAT][N] partial sums (P > 1)
+  int32_t* work;          // next work item (zero before the launch)
+  int32_t* status;
+  unsigned long long* trace;  // diagnostics: clock64 stamps of CTA 0 (or null)
+  StageLayout st;
+};
+
+// Stamp event `ev` of index `i` (CTA 0 only, first MOE_TRACE_STAGES indices).
+__device__ __forceinline__ void gtrace(unsigned long long* tr, int ev, int i) {
+  if (tr && blockIdx.x == 0 && i < MOE_TRACE_STAGES) tr[ev * MOE_TRACE_STAGES + i] = (unsigned long long)clock64();
 }
-__device__ __forceinline__ uint32_t h2mul_u(uint32_t a, uint32_t b) {
+
+__device__ __forceinline__ const CUtensorMap* map_of(int wpg, const CUtensorMap* m2, const CUtensorMap* m3,
+                                                     const CUtensorMap* m4) {
+  return wpg == 2 ? m2 : wpg == 3 ? m3 : m4;
+}
+
+// ------------------------------------------------------------------ small PTX helpers
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          ptx::smem_u32(dst)),
+      "l"((uint64_t)map), "r"(x), "r"(y), "r"(z), "r"(ptx::smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ uint2 lds64(const uint8_t* p) { return *reinterpret_cast<const uint2*>(p); }
+__device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
+__device__ __forceinline__ float ldsf(const uint8_t* p) { return *reinterpret_cast<const float*>(p); }
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsumers) : "memory"); }
+
+// Bounded wait that ignores the abort flag (used to drain copies before exit).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!ptx::mbar_try_wait(bar, parity) && clock64() - t0 < kGemvWait / 4) {
+  }
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
   __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
   return *reinterpret_cast<uint32_t*>(&r);
 }
-__device__ __forceinline__ void e2m1x8_to_f16_v(uint32_t w, uint32_t* o) {
+__device__ __forceinline__ void e2m1x8_to_f16(uint32_t w, uint32_t* o) {
   asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
       "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
       "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
       : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
       : "r"(w));
 }
-
 __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1, const float* c) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -58,392 +138,529 @@ __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]),
         "f"(c[3]));
 }
+__device__ __forceinline__ float half_lo(uint32_t v) { return __half2float(__ushort_as_half((uint16_t)(v & 0xFFFFu))); }
+__device__ __forceinline__ float half_hi(uint32_t v) { return __half2float(__ushort_as_half((uint16_t)(v >> 16))); }
 
-// ---------------------------------------------------------------- cp.async
-__device__ __forceinline__ void cp16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-               "l"(src)
-               : "memory");
-}
-// 16-byte copy that reads src_bytes (0 or 16) and zero-fills the rest.
-__device__ __forceinline__ void cp16z(void* dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-               "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp8(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+constexpr uint32_t h2c(uint32_t h) { return h | (h << 16); }
 
-struct GemvArgs {
-  const uint8_t* packed;
-  int E, H, F;
-  int N, K;
-  int proj;                 // 0: gate+up (SwiGLU), 2: down
-  const __half* act;        // [rows][K] fp16 activations, sorted rows
-  const int32_t* chunks;
-  const int32_t* chunk_count;
-  const float* row_scale;   // NVFP4 only (sx per token for gate/up, sh per row for down)
-  const int32_t* perm;
-  int topk;
-  void* out;
-};
-
-// Where one work item's data lives; shared by the copy and compute sides.
-struct ItemView {
-  int e, row0, rows, slice;
-  int f0, f1;
-  const uint32_t* codes0;
-  const uint8_t* scales0;
-  const uint32_t* codes1;
-  const uint8_t* scales1;
-};
-
-template <int NMAT>
-__device__ __forceinline__ ItemView item_view(const GemvArgs& a, int item, int slices) {
-  ItemView v;
-  const int chunk = item / slices;
-  v.slice = item % slices;
-  v.e = a.chunks[3 * chunk];
-  v.row0 = a.chunks[3 * chunk + 1];
-  v.rows = a.chunks[3 * chunk + 2];
-  const uint8_t* fmt = a.packed + kOffFmt;
-  const uint64_t* co = reinterpret_cast<const uint64_t*>(a.packed + kOffCode);
-  const uint64_t* so = reinterpret_cast<const uint64_t*>(a.packed + kOffScale);
-  const int i0 = v.e * 3 + a.proj, i1 = i0 + NMAT - 1;
-  v.f0 = fmt[i0];
-  v.f1 = fmt[i1];
-  v.codes0 = reinterpret_cast<const uint32_t*>(a.packed + co[i0]);
-  v.scales0 = a.packed + so[i0];
-  v.codes1 = reinterpret_cast<const uint32_t*>(a.packed + co[i1]);
-  v.scales1 = a.packed + so[i1];
-  return v;
+// Activation multiplier 1/f_j (fp16x2) for pair j (j = 0..3) of a lane's eight
+// inputs, whose codes sit in a field of weight f_j: INT4 1, 16, 1, 16 (fields at
+// bits 0 and 4; pairs 2, 3 after >> 8); INT2 and INT3 4^j (fields at bits 2j).
+__host__ __device__ constexpr uint32_t act_mul(int fmt, int j) {
+  return fmt == MOE_FMT_NVFP4 ? h2c(0x3C00u)
+         : fmt == MOE_FMT_INT4 ? ((j & 1) ? h2c(0x2C00u) : h2c(0x3C00u))   // 1, 1/16
+         : (j == 0 ? h2c(0x3C00u) : j == 1 ? h2c(0x3400u) : j == 2 ? h2c(0x2C00u) : h2c(0x2400u));  // 4^-j
+}
+// -offset * 2^-24: times the group sum of the activations, the MMA's C input.
+__host__ __device__ constexpr float offset_term(int fmt) {
+  return fmt == MOE_FMT_INT4 ? -8.0f / 16777216.0f : fmt == MOE_FMT_INT3 ? -4.0f / 16777216.0f : -2.0f / 16777216.0f;
 }
 
-// Slot layout of one group (16-byte slots, [slot][lane] so 128-bit shared
-// accesses are conflict-free): 2m, 2m+1 words of matrix m (the second: 3-bit
-// high bits), 2*NMAT scales (matrix 0 in .xy, matrix 1 in .zw), 2*NMAT+1+nt
-// activations of token tile nt.
-template <int NMAT, int NT8>
-struct Slots {
-  static constexpr int kItems = 2 * NMAT + 1 + NT8;
-  static constexpr int kScale = 2 * NMAT;
-  static constexpr int kAct = 2 * NMAT + 1;
-};
-template <int NMAT, int NT8>
-__device__ __forceinline__ uint4* slot_ptr(uint4* ring, int stage, int slot, int lane) {
-  return ring + (stage * Slots<NMAT, NT8>::kItems + slot) * 32 + lane;
+// Address of the 16-byte chunk of rows 4g..4g+3 in word-row z of a code box
+// (lines of 128 bytes: line = 2z + slice; 128-byte swizzle: chunk ^= line % 8).
+__device__ __forceinline__ const uint8_t* code_chunk(const uint8_t* box, int z, int y, int g) {
+  const int line = 2 * z + y;
+  return box + line * 128 + ((g ^ (line & 7)) << 4);
 }
 
-// Copy side.  A cursor walks this warp's stream of (item, group) elements; its
-// per-thread source pointers advance by a fixed stride per group and are
-// recomputed only when the stream moves to the next work item.
-template <int NMAT, int NT8>
-struct Cursor {
-  int j, g, n_items, g0, g1, slices;
-  int fm[NMAT];
-  const uint32_t* cw[NMAT];   // word (4-bit / NVFP4: word c; 2-, 3-bit: low word c/2) of the thread's 4 rows
-  const uint32_t* ch[NMAT];   // 3-bit: high-bit word
-  const uint8_t* cs[NMAT];    // scales of the thread's 4 rows
-  int wstride[NMAT];          // words per group
-  const __half* cx[NT8];      // 8 activations of token gl (+8)
-  uint32_t xbytes[NT8];       // 16, or 0 beyond the chunk (zero fill)
-};
-
-template <int NMAT, int NT8>
-__device__ __forceinline__ void cursor_item(Cursor<NMAT, NT8>& cu, const GemvArgs& a, int lane) {
-  const ItemView v = item_view<NMAT>(a, blockIdx.x + cu.j * gridDim.x, cu.slices);
-  const int gl = lane >> 2, c = lane & 3;
-  const int nb4 = v.slice * kRowsPerCta + 4 * gl;
-#pragma unroll
-  for (int m = 0; m < NMAT; ++m) {
-    const int f = m == 0 ? v.f0 : v.f1;
-    const uint32_t* codes = m == 0 ? v.codes0 : v.codes1;
-    const uint8_t* scales = m == 0 ? v.scales0 : v.scales1;
-    const int wpg = fmt_words(f);
-    const int wsel = (f == MOE_FMT_INT4 || f == MOE_FMT_NVFP4) ? c : (c >> 1);
-    cu.fm[m] = f;
-    cu.wstride[m] = wpg * 128;
-    cu.cw[m] = codes + word_index(nb4, cu.g0 * 32, a.K, wpg, wsel);
-    cu.ch[m] = codes + word_index(nb4, cu.g0 * 32, a.K, wpg, 2);
-    cu.cs[m] = f == MOE_FMT_NVFP4 ? scales + scale_index(nb4, 2 * cu.g0 + (c >> 1), a.K / 16)
-                                  : scales + 2 * scale_index(nb4, cu.g0, a.K / 32);
-  }
-#pragma unroll
-  for (int nt = 0; nt < NT8; ++nt) {
-    const int tok = nt * 8 + gl;
-    const bool ok = tok < v.rows;
-    cu.cx[nt] = a.act + (size_t)(v.row0 + (ok ? tok : 0)) * a.K + cu.g0 * 32 + 8 * c;
-    cu.xbytes[nt] = ok ? 16u : 0u;
-  }
-}
-
-// Issue the cursor's element into ring stage `stage` and advance the cursor.
-template <int NMAT, int NT8>
-__device__ __forceinline__ void cursor_issue(Cursor<NMAT, NT8>& cu, const GemvArgs& a, uint4* ring, int stage,
-                                             int lane) {
-  if (cu.j >= cu.n_items) return;
-#pragma unroll
-  for (int m = 0; m < NMAT; ++m) {
-    cp16(slot_ptr<NMAT, NT8>(ring, stage, 2 * m, lane), cu.cw[m]);
-    if (cu.fm[m] == MOE_FMT_INT3) cp16(slot_ptr<NMAT, NT8>(ring, stage, 2 * m + 1, lane), cu.ch[m]);
-    uint8_t* sdst = reinterpret_cast<uint8_t*>(slot_ptr<NMAT, NT8>(ring, stage, Slots<NMAT, NT8>::kScale, lane)) + 8 * m;
-    if (cu.fm[m] == MOE_FMT_NVFP4) cp4(sdst, cu.cs[m]);
-    else cp8(sdst, cu.cs[m]);
-    cu.cw[m] += cu.wstride[m];
-    cu.ch[m] += cu.wstride[m];
-    cu.cs[m] += 256;  // 128 fp16 scales, or 2 x 128 e4m3 block scales, per group
-  }
-#pragma unroll
-  for (int nt = 0; nt < NT8; ++nt) {
-    cp16z(slot_ptr<NMAT, NT8>(ring, stage, Slots<NMAT, NT8>::kAct + nt, lane), cu.cx[nt], cu.xbytes[nt]);
-    cu.cx[nt] += 32;
-  }
-  if (++cu.g == cu.g1) {
-    cu.g = cu.g0;
-    if (++cu.j < cu.n_items) cursor_item(cu, a, lane);
-  }
-}
-
-__device__ __forceinline__ uint32_t h2fma_u(uint32_t a, uint32_t b, uint32_t c) {
-  __half2 r = __hfma2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b), *reinterpret_cast<__half2*>(&c));
-  return *reinterpret_cast<uint32_t*>(&r);
-}
-__device__ __forceinline__ uint32_t lop_or(uint32_t a, uint32_t mask, uint32_t c) { return (a & mask) | c; }
-
-// fp16 pair constants (both halves equal)
-constexpr uint32_t kMagic = 0x64006400u;  // 1024.0
-__host__ __device__ constexpr uint32_t h2c(uint32_t h) { return h | (h << 16); }
-
-// The four fp16 pairs (inputs 8c..8c+7 of the group) of row i (0..3) of the
-// thread, as the signed code q = u - offset (NVFP4: e2m1 value times block scale).
-// Unpack: masking bits [b, b+w) of both half-words and OR'ing 1024.0 gives
-// 1024 + 2^b * u exactly (b + w <= 10); one FMA with 2^-b and -(1024/2^b + offset)
-// then gives u - offset exactly (the exact result is representable).
-template <int FMT>
-__device__ __forceinline__ void unpack_row(uint4 w0, uint4 w1, uint32_t sc, int i, int c, uint32_t* p) {
-  const uint32_t w = i == 0 ? w0.x : i == 1 ? w0.y : i == 2 ? w0.z : w0.w;
+// One group (kg) of one matrix: unpack the lane's rows, run the MMAs for every
+// token tile and accumulate.  box: this warp's code box; sc: the matrix's scale
+// tile; xs: the lane's 16 activation bytes of the group in token tile 0 (token
+// tiles follow at 8 rows x 256 bytes); gs: the group sum of token 2c in token
+// tile 0 (token 2c+1 follows at +16 bytes, tile nt at nt * 128 bytes).
+template <int FMT, int NT8>
+__device__ __forceinline__ void group_mma(const uint8_t* box, const uint8_t* sc, int kg, int y, int s, int g, int c,
+                                          const uint8_t* xs, const uint8_t* gs, float (&acc)[2][NT8][4]) {
+  uint32_t p[4][4];   // [row i][pair j]
   if (FMT == MOE_FMT_NVFP4) {
-    e2m1x8_to_f16_v(w, p);
-    const __half2 s2 = __float2half2_rn(e4m3_value((sc >> (8 * i)) & 255u));
-    const uint32_t sp = *reinterpret_cast<const uint32_t*>(&s2);
+    const uint4 w = lds128(code_chunk(box, 4 * kg + c, y, g));
+    const uint32_t bs = lds32(sc + (2 * kg + (c >> 1)) * 128 + 32 * s + 4 * g);  // e4m3 block scales of rows 4g..
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) p[j] = h2mul_u(p[j], sp);  // exact: <= 6 significant bits
-  } else if (FMT == MOE_FMT_INT4) {
-    // pairs 0,1 at bits 0-3 / 4-7; pairs 2,3 at bits 8-11 / 12-15 (after >> 8)
-    const uint32_t w8 = w >> 8;
-    p[0] = h2fma_u(lop_or(w, 0x000F000Fu, kMagic), h2c(0x3C00u), h2c(0xE408u));    // x*1 - 1032
-    p[1] = h2fma_u(lop_or(w, 0x00F000F0u, kMagic), h2c(0x2C00u), h2c(0xD480u));    // x/16 - 72
-    p[2] = h2fma_u(lop_or(w8, 0x000F000Fu, kMagic), h2c(0x3C00u), h2c(0xE408u));
-    p[3] = h2fma_u(lop_or(w8, 0x00F000F0u, kMagic), h2c(0x2C00u), h2c(0xD480u));
-  } else if (FMT == MOE_FMT_INT2) {
-    const uint32_t ws = w >> (8 * (c & 1));  // the 4 pairs of inputs 8c..8c+7 at bits 0-7 / 16-23
-    p[0] = h2fma_u(lop_or(ws, 0x00030003u, kMagic), h2c(0x3C00u), h2c(0xE402u));   // x - 1026
-    p[1] = h2fma_u(lop_or(ws, 0x000C000Cu, kMagic), h2c(0x3400u), h2c(0xDC08u));   // x/4 - 258
-    p[2] = h2fma_u(lop_or(ws, 0x00300030u, kMagic), h2c(0x2C00u), h2c(0xD420u));   // x/16 - 66
-    p[3] = h2fma_u(lop_or(ws, 0x00C000C0u, kMagic), h2c(0x2400u), h2c(0xCC80u));   // x/64 - 18
-  } else {  // INT3: low bits as INT2; bit 2 of pair J at bits J and 16+J of the high word
-    const uint32_t lo = w >> (8 * (c & 1));
-    const uint32_t hw = i == 0 ? w1.x : i == 1 ? w1.y : i == 2 ? w1.z : w1.w;
-    const uint32_t hi = hw >> (4 * c);  // pair j's high bits at bits j, 16+j
-    // pair j's 3-bit code at bits [2j, 2j+3): low bits from lo, high bit = (hi << (j+2)) at 2j+2
-    p[0] = h2fma_u((lop_or(lo, 0x00030003u, kMagic) | ((hi << 2) & 0x00040004u)), h2c(0x3C00u), h2c(0xE404u));  // - 1028
-    p[1] = h2fma_u((lop_or(lo, 0x000C000Cu, kMagic) | ((hi << 3) & 0x00100010u)), h2c(0x3400u), h2c(0xDC10u));  // /4 - 260
-    p[2] = h2fma_u((lop_or(lo, 0x00300030u, kMagic) | ((hi << 4) & 0x00400040u)), h2c(0x2C00u), h2c(0xD440u));  // /16 - 68
-    p[3] = h2fma_u((lop_or(lo, 0x00C000C0u, kMagic) | ((hi << 5) & 0x01000100u)), h2c(0x2400u), h2c(0xCD00u));  // /64 - 20
-  }
-}
-
-__device__ __forceinline__ float half_at(uint32_t lohi, int hi) {
-  return __half2float(__ushort_as_half((uint16_t)(hi ? (lohi >> 16) : (lohi & 0xFFFFu))));
-}
-
-// Compute side for one group held in ring stage `stage`; formats F0/F1 known at
-// compile time.  acc[m][t][nt][4]: matrix m, 16-row tile t (rows 2t, 2t+1 of the
-// thread's four), token tile nt, mma accumulator element.
-template <int NMAT, int F0, int F1, int NT8>
-__device__ __forceinline__ void compute_group(uint4* ring, int stage, int lane, float (&acc)[NMAT][2][NT8][4]) {
-  const int c = lane & 3;
-  const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
-  const uint4 sc = *slot_ptr<NMAT, NT8>(ring, stage, Slots<NMAT, NT8>::kScale, lane);
-  uint4 x[NT8];
+    for (int i = 0; i < 4; ++i) {
+      e2m1x8_to_f16(wv[i], p[i]);
+      const __half2 s2 = __float2half2_rn(e4m3_value((bs >> (8 * i)) & 255u));
+      const uint32_t sp = *reinterpret_cast<const uint32_t*>(&s2);
 #pragma unroll
-  for (int nt = 0; nt < NT8; ++nt) x[nt] = *slot_ptr<NMAT, NT8>(ring, stage, Slots<NMAT, NT8>::kAct + nt, lane);
+      for (int j = 0; j < 4; ++j) p[i][j] = hmul2(p[i][j], sp);  // exact: <= 6 significant bits
+    }
 #pragma unroll
-  for (int m = 0; m < NMAT; ++m) {
-    constexpr int kF[2] = {F0, F1};
-    const int FMT = kF[m];
-    const uint4 w0 = *slot_ptr<NMAT, NT8>(ring, stage, 2 * m, lane);
-    const uint4 w1 = FMT == MOE_FMT_INT3 ? *slot_ptr<NMAT, NT8>(ring, stage, 2 * m + 1, lane) : make_uint4(0, 0, 0, 0);
-    const uint32_t s_lo = m == 0 ? sc.x : sc.z, s_hi = m == 0 ? sc.y : sc.w;  // 4 fp16 scales or 4 e4m3 bytes in s_lo
+    for (int nt = 0; nt < NT8; ++nt) {
+      const uint4 xr = lds128(xs + nt * 2048);
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      uint32_t pa[4], pb[4];  // rows 2t (MMA row g) and 2t+1 (MMA row g+8)
-      if (m == 0) {
-        unpack_row<F0>(w0, w1, s_lo, 2 * t, c, pa);
-        unpack_row<F0>(w0, w1, s_lo, 2 * t + 1, c, pb);
-      } else {
-        unpack_row<F1>(w0, w1, s_lo, 2 * t, c, pa);
-        unpack_row<F1>(w0, w1, s_lo, 2 * t + 1, c, pb);
-      }
-      const uint32_t A1[4] = {pa[0], pb[0], pa[1], pb[1]};
-      const uint32_t A2[4] = {pa[2], pb[2], pa[3], pb[3]};
-#pragma unroll
-      for (int nt = 0; nt < NT8; ++nt) {
-        if (FMT == MOE_FMT_NVFP4) {  // codes already carry their block scale: accumulate directly
-          mma16816(acc[m][t][nt], A1, x[nt].x, x[nt].y, acc[m][t][nt]);
-          mma16816(acc[m][t][nt], A2, x[nt].z, x[nt].w, acc[m][t][nt]);
-        } else {  // the group's raw sum, then one fp32 FMA per output with the row's scale
-          float d[4];
-          mma16816(d, A1, x[nt].x, x[nt].y, zero4);
-          mma16816(d, A2, x[nt].z, x[nt].w, d);
-          const uint32_t sw = t == 0 ? s_lo : s_hi;  // rows 2t, 2t+1 -> halves of one scale word
-          const float sa = half_at(sw, 0), sb = half_at(sw, 1);
-          acc[m][t][nt][0] = fmaf(sa, d[0], acc[m][t][nt][0]);
-          acc[m][t][nt][1] = fmaf(sa, d[1], acc[m][t][nt][1]);
-          acc[m][t][nt][2] = fmaf(sb, d[2], acc[m][t][nt][2]);
-          acc[m][t][nt][3] = fmaf(sb, d[3], acc[m][t][nt][3]);
-        }
+      for (int t = 0; t < 2; ++t) {
+        const uint32_t A1[4] = {p[2 * t][0], p[2 * t + 1][0], p[2 * t][1], p[2 * t + 1][1]};
+        const uint32_t A2[4] = {p[2 * t][2], p[2 * t + 1][2], p[2 * t][3], p[2 * t + 1][3]};
+        mma16816(acc[t][nt], A1, xr.x, xr.y, acc[t][nt]);
+        mma16816(acc[t][nt], A2, xr.z, xr.w, acc[t][nt]);
       }
     }
+    return;
   }
-}
-
-// Consume the ng groups of one item from the ring (formats F0/F1), keeping the
-// ring kStages-1 groups ahead: each consumed group frees its stage, which is
-// refilled with stream element s+kStages-1 (possibly of a later item).  The
-// warp's partial sums go to shared memory at the end.
-template <int NMAT, int F0, int F1, int NT8>
-__device__ __forceinline__ void consume_item(const GemvArgs& a, uint4* ring, float* part, int ng, int& s,
-                                          Cursor<NMAT, NT8>& cu, int warp, int lane) {
-  float acc[NMAT][2][NT8][4];
+  if (FMT == MOE_FMT_INT4) {
+    const uint4 w = lds128(code_chunk(box, 4 * kg + c, y, g));
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-  for (int m = 0; m < NMAT; ++m)
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t w8 = wv[i] >> 8;
+      p[i][0] = wv[i] & 0x000F000Fu;
+      p[i][1] = wv[i] & 0x00F000F0u;
+      p[i][2] = w8 & 0x000F000Fu;
+      p[i][3] = w8 & 0x00F000F0u;
+    }
+  } else {
+    const int wpg = FMT == MOE_FMT_INT3 ? 3 : 2;
+    const uint4 w = lds128(code_chunk(box, wpg * kg + (c >> 1), y, g));
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+    const int sh = 8 * (c & 1);
+    if (FMT == MOE_FMT_INT2) {
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t ws = wv[i] >> sh;
 #pragma unroll
-      for (int nt = 0; nt < NT8; ++nt)
+        for (int j = 0; j < 4; ++j) p[i][j] = ws & (0x00030003u << (2 * j));
+      }
+    } else {
+      // INT3: bit 2 of code 2m / 2m+1 sits at bit m / 16+m of word 2 (m = 0..15).
+      // The lane's pairs m = 4c+j rotate to bits j+2; shifted left by j they land
+      // on bit 2j+2, right above the pair's two low bits.
+      const uint4 hw = lds128(code_chunk(box, 3 * kg + 2, y, g));
+      const uint32_t hv[4] = {hw.x, hw.y, hw.z, hw.w};
+      const uint32_t rot = (uint32_t)(4 * c + 30) & 31u;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[m][t][nt][j] = 0.0f;
-  for (int i = 0; i < ng; ++i) {
-    cp_wait<kStages - 2>();  // this element has landed (the thread's own copies)
-    compute_group<NMAT, F0, F1, NT8>(ring, s, lane, acc);
-    // refill the stage consumed one element ago with the element kStages-1 ahead
-    cursor_issue(cu, a, ring, s == 0 ? kStages - 1 : s - 1, lane);
-    cp_commit();  // one (possibly empty) group per element keeps the wait count fixed
-    if (++s == kStages) s = 0;
-  }
-  const int gl = lane >> 2, c = lane & 3;
-#pragma unroll
-  for (int m = 0; m < NMAT; ++m)
-#pragma unroll
-    for (int t = 0; t < 2; ++t)
-#pragma unroll
-      for (int nt = 0; nt < NT8; ++nt)
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t ws = wv[i] >> sh;
+        const uint32_t hh = __funnelshift_r(hv[i], hv[i], rot);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          part[((warp * NMAT + m) * kRowsPerCta + 4 * gl + 2 * t + (j >> 1)) * kPartStride + nt * 8 + 2 * c + (j & 1)] =
-              acc[m][t][nt][j];
-}
-
-template <int NMAT, int F0, int NT8>
-__device__ __forceinline__ void consume_f1(int f1, const GemvArgs& a, uint4* ring, float* part, int ng, int& s,
-                                           Cursor<NMAT, NT8>& cu, int warp, int lane) {
-  if (NMAT == 1) return consume_item<NMAT, F0, F0, NT8>(a, ring, part, ng, s, cu, warp, lane);
-  switch (f1) {
-    case MOE_FMT_INT2: return consume_item<NMAT, F0, MOE_FMT_INT2, NT8>(a, ring, part, ng, s, cu, warp, lane);
-    case MOE_FMT_INT3: return consume_item<NMAT, F0, MOE_FMT_INT3, NT8>(a, ring, part, ng, s, cu, warp, lane);
-    case MOE_FMT_INT4: return consume_item<NMAT, F0, MOE_FMT_INT4, NT8>(a, ring, part, ng, s, cu, warp, lane);
-    default: return consume_item<NMAT, F0, MOE_FMT_NVFP4, NT8>(a, ring, part, ng, s, cu, warp, lane);
-  }
-}
-
-template <int NMAT, int NT8>
-__global__ void __launch_bounds__(32 * kWarps) expert_gemv_kernel(GemvArgs a) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  constexpr int kItems = Slots<NMAT, NT8>::kItems;
-  uint4* ring_all = reinterpret_cast<uint4*>(smem_raw);                                // [kWarps][kStages][kItems][32]
-  float* part = reinterpret_cast<float*>(ring_all + kWarps * kStages * kItems * 32);  // [kWarps][NMAT][32][17]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint4* ring = ring_all + warp * kStages * kItems * 32;
-
-  const int slices = a.N / kRowsPerCta;
-  const int total = *a.chunk_count * slices;
-  const int n_items = total > (int)blockIdx.x ? (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
-  const int G = a.K / 32;
-  const int g0 = (G * warp) / kWarps, g1 = (G * (warp + 1)) / kWarps, ng = g1 - g0;
-  // this warp's stream: (item, group) elements in item order, issued kStages-1 ahead
-  Cursor<NMAT, NT8> cu;
-  cu.j = 0;
-  cu.g = g0;
-  cu.n_items = n_items;
-  cu.g0 = g0;
-  cu.g1 = g1;
-  cu.slices = slices;
-  if (n_items > 0) cursor_item(cu, a, lane);
-  for (int st = 0; st < kStages - 1; ++st) {
-    cursor_issue(cu, a, ring, st, lane);
-    cp_commit();
-  }
-
-  int s = 0;  // ring stage of the next element to consume
-  for (int j = 0; j < n_items; ++j) {
-    const ItemView v = item_view<NMAT>(a, blockIdx.x + j * gridDim.x, slices);
-    switch (v.f0) {
-      case MOE_FMT_INT2: consume_f1<NMAT, MOE_FMT_INT2, NT8>(v.f1, a, ring, part, ng, s, cu, warp, lane); break;
-      case MOE_FMT_INT3: consume_f1<NMAT, MOE_FMT_INT3, NT8>(v.f1, a, ring, part, ng, s, cu, warp, lane); break;
-      case MOE_FMT_INT4: consume_f1<NMAT, MOE_FMT_INT4, NT8>(v.f1, a, ring, part, ng, s, cu, warp, lane); break;
-      default: consume_f1<NMAT, MOE_FMT_NVFP4, NT8>(v.f1, a, ring, part, ng, s, cu, warp, lane); break;
+          p[i][j] = (ws & (0x00030003u << (2 * j))) | ((hh << j) & (0x00040004u << (2 * j)));
+      }
     }
-    __syncthreads();
-    // reduce the K-split partials and run the epilogue of this item
-    const LayerHdr L = hdr_view(a.packed, a.E, a.H, a.F);
-    const float ts0 = v.f0 == MOE_FMT_NVFP4 ? L.tscale[v.e * 3 + a.proj] : 1.0f;
-    const float ts1 = v.f1 == MOE_FMT_NVFP4 ? L.tscale[v.e * 3 + a.proj + NMAT - 1] : 1.0f;
-    for (int idx = threadIdx.x; idx < kRowsPerCta * NT8 * 8; idx += blockDim.x) {
-      const int rl = idx % kRowsPerCta, tok = idx / kRowsPerCta;
-      if (tok >= v.rows) continue;
-      const int n = v.slice * kRowsPerCta + rl, r = v.row0 + tok;
-      float s0 = 0.0f, s1 = 0.0f;
+  }
+  const uint2 s4 = lds64(sc + kg * 256 + (32 * s + 4 * g) * 2);  // fp16 scales of rows 4g..4g+3
+  const float sr[4] = {half_lo(s4.x), half_hi(s4.x), half_lo(s4.y), half_hi(s4.y)};
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        s0 += part[((w * NMAT + 0) * kRowsPerCta + rl) * kPartStride + tok];
-        if (NMAT == 2) s1 += part[((w * NMAT + NMAT - 1) * kRowsPerCta + rl) * kPartStride + tok];
-      }
-      if (NMAT == 2) {
-        if (a.row_scale) {
-          const float sx = a.row_scale[a.perm[r] / a.topk];
-          s0 *= sx * ts0;
-          s1 *= sx * ts1;
-          reinterpret_cast<float*>(a.out)[(size_t)r * a.N + n] = s0 / (1.0f + __expf(-s0)) * s1;
-        } else {
-          reinterpret_cast<__half*>(a.out)[(size_t)r * a.N + n] = __float2half_rn(s0 / (1.0f + __expf(-s0)) * s1);
-        }
-      } else {
-        if (a.row_scale) s0 *= a.row_scale[r] * ts0;
-        reinterpret_cast<float*>(a.out)[(size_t)r * a.N + n] = s0;
+  for (int nt = 0; nt < NT8; ++nt) {
+    const uint4 xr = lds128(xs + nt * 2048);
+    const uint32_t b0 = xr.x, b1 = hmul2(xr.y, act_mul(FMT, 1));
+    const uint32_t b2 = FMT == MOE_FMT_INT4 ? xr.z : hmul2(xr.z, act_mul(FMT, 2));
+    const uint32_t b3 = hmul2(xr.w, act_mul(FMT, 3));
+    const float d0 = offset_term(FMT) * ldsf(gs + nt * 128), d1 = offset_term(FMT) * ldsf(gs + nt * 128 + 16);
+    const float D[4] = {d0, d1, d0, d1};  // -offset * sum(x) * 2^-24 for tokens 2c, 2c+1
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const uint32_t A1[4] = {p[2 * t][0], p[2 * t + 1][0], p[2 * t][1], p[2 * t + 1][1]};
+      const uint32_t A2[4] = {p[2 * t][2], p[2 * t + 1][2], p[2 * t][3], p[2 * t + 1][3]};
+      float d[4];
+      mma16816(d, A1, b0, b1, D);
+      mma16816(d, A2, b2, b3, d);
+      acc[t][nt][0] = fmaf(sr[2 * t], d[0], acc[t][nt][0]);
+      acc[t][nt][1] = fmaf(sr[2 * t], d[1], acc[t][nt][1]);
+      acc[t][nt][2] = fmaf(sr[2 * t + 1], d[2], acc[t][nt][2]);
+      acc[t][nt][3] = fmaf(sr[2 * t + 1], d[3], acc[t][nt][3]);
+    }
+  }
+}
+
+// Consume the k-tiles of one work item (formats F0, F1 of the first and second
+// matrix) from the ring; the first tile's stage has already been waited for.
+// Waits that give up clear `ok`; the loop still runs to the end (without waiting
+// or computing) so all consumer warps stay in step.
+template <int NMAT, int NT8, int F0, int F1>
+__device__ __forceinline__ void consume_tiles(const StageLayout& L, uint8_t* smem, uint64_t* full, uint64_t* empty,
+                                              volatile int* abort_flag, int ntiles, int& stage, uint32_t& phase,
+                                              bool& ok, float (&acc)[NMAT][2][NT8][4], unsigned long long* tr,
+                                              int& gtile) {
+  const int s = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  for (int kt = 0; kt < ntiles; ++kt) {
+    if (kt > 0 && ok && !__all_sync(0xffffffffu, ptx::mbar_wait(&full[stage], phase, abort_flag, kGemvWait)))
+      ok = false;
+    if (threadIdx.x == 0) gtrace(tr, 2, gtile);
+    if (ok) {
+      const uint8_t* sb = smem + stage * L.bytes;
+#pragma unroll
+      for (int kg = 0; kg < 4; ++kg) {
+        const uint8_t* xs = sb + L.x_off + g * 256 + (32 * kg + 8 * c) * 2;
+        const uint8_t* gs = sb + L.sum_off + (2 * c) * 16 + kg * 4;
+        group_mma<F0, NT8>(sb + L.code_off[0] + (s >> 1) * L.box[0], sb + L.scale_off[0], kg, s & 1, s, g, c, xs,
+                           gs, acc[0]);
+        if (NMAT == 2)
+          group_mma<F1, NT8>(sb + L.code_off[1] + (s >> 1) * L.box[1], sb + L.scale_off[1], kg, s & 1, s, g, c, xs,
+                             gs, acc[NMAT - 1]);
       }
     }
-    __syncthreads();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&empty[stage]);
+    if (threadIdx.x == 0) gtrace(tr, 3, gtile);
+    ++gtile;
+    if (++stage == L.stages) {
+      stage = 0;
+      phase ^= 1u;
+    }
   }
-  cp_wait<0>();  // no copy may still be landing when the CTA exits
+}
+
+template <int NMAT, int NT8, int F0>
+__device__ __forceinline__ void consume_f1(int f1, const StageLayout& L, uint8_t* smem, uint64_t* full,
+                                           uint64_t* empty, volatile int* abort_flag, int ntiles, int& stage,
+                                           uint32_t& phase, bool& ok, float (&acc)[NMAT][2][NT8][4],
+                                           unsigned long long* tr, int& gtile) {
+  if (NMAT == 1 || F0 == MOE_FMT_NVFP4)
+    return consume_tiles<NMAT, NT8, F0, F0>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile);
+  switch (f1) {
+    case MOE_FMT_INT2: return consume_tiles<NMAT, NT8, F0, MOE_FMT_INT2>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile);
+    case MOE_FMT_INT3: return consume_tiles<NMAT, NT8, F0, MOE_FMT_INT3>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile);
+    default: return consume_tiles<NMAT, NT8, F0, MOE_FMT_INT4>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile);
+  }
+}
+
+// Work item `it` -> (chunk, weight block, K part): block-major, so the chunks of
+// one expert (adjacent in the chunk list) read the same weight tiles close in
+// time and the second read hits L2.
+struct Item {
+  int chunk, nb, p;
+};
+__device__ __forceinline__ Item item_of(int it, int P, int nchunks) {
+  Item r;
+  r.p = it % P;
+  const int rest = it / P;
+  r.chunk = rest % nchunks;
+  r.nb = rest / nchunks;
+  return r;
+}
+
+// What the consumers need about an item, written by the producer into the
+// shared-memory slot of the item's first stage (it < 0 ends the stream).
+struct ItemDesc {
+  int it, chunk, nb, p, row0, rows, ntiles, f0, f1;
+  float ts0, ts1;
+  int pad;
+};
+static_assert(sizeof(ItemDesc) == 48, "descriptor size");
+
+// Producer-side view of an item: descriptor plus the copy sources.
+template <int NMAT>
+struct ItemSrc {
+  ItemDesc d;
+  int kt0;
+  int z0[NMAT], wpg[NMAT];
+  const uint8_t* sptr[NMAT];
+  uint32_t bytes;
+};
+
+template <int NMAT, int NT8>
+__device__ __forceinline__ void load_item(ItemSrc<NMAT>& s, int it, int total, int nchunks, const GemvArgs& a,
+                                          const LayerHdr& L, int KT) {
+  s.d.it = it < total ? it : -1;
+  s.bytes = (uint32_t)(8 * NT8 * 256) + (a.sums ? (uint32_t)(8 * NT8 * 16) : 0u);
+  if (it >= total) return;
+  const Item w = item_of(it, a.P, nchunks);
+  const int e = a.chunks[3 * w.chunk];
+  s.d.chunk = w.chunk;
+  s.d.nb = w.nb;
+  s.d.p = w.p;
+  s.d.row0 = a.chunks[3 * w.chunk + 1];
+  s.d.rows = a.chunks[3 * w.chunk + 2];
+  s.kt0 = w.p * KT / a.P;
+  s.d.ntiles = (w.p + 1) * KT / a.P - s.kt0;
+#pragma unroll
+  for (int m = 0; m < NMAT; ++m) {
+    const int i = e * 3 + a.proj + m;
+    const int f = L.fmt[i];
+    if (m == 0) {
+      s.d.f0 = f;
+      s.d.ts0 = f == MOE_FMT_NVFP4 ? L.tscale[i] : 1.0f;
+    }
+    if (m == NMAT - 1) {
+      s.d.f1 = f;
+      s.d.ts1 = f == MOE_FMT_NVFP4 ? L.tscale[i] : 1.0f;
+    }
+    s.wpg[m] = fmt_words(f);
+    s.z0[m] = (int)(L.code_off[i] >> 9) + (w.nb * KT) * 4 * s.wpg[m];
+    s.sptr[m] = L.base + L.scale_off[i] + (size_t)w.nb * KT * 1024u;
+    s.bytes += 2u * 1024u * (uint32_t)s.wpg[m] + 1024u;
+  }
+}
+
+// Epilogue of one output (row r, weight row n) from the matrices' sums v[m]
+// (integer formats: already multiplied by 2^24).  Gate/up returns h as stored
+// (fp16-rounded for integer layers), for the group sums of the down GEMV.
+template <int NMAT>
+__device__ __forceinline__ float store_output(const GemvArgs& a, int r, int n, const float* v, const float* ts) {
+  if (NMAT == 2) {
+    float gv = v[0], uv = v[1];
+    if (a.row_scale) {
+      const float sx = a.row_scale[a.perm[r] / a.topk];
+      gv *= sx * ts[0];
+      uv *= sx * ts[1];
+      const float h = gv / (1.0f + __expf(-gv)) * uv;
+      reinterpret_cast<float*>(a.out)[(size_t)r * a.N + n] = h;
+      return h;
+    }
+    const __half h = __float2half_rn(gv / (1.0f + __expf(-gv)) * uv);
+    reinterpret_cast<__half*>(a.out)[(size_t)r * a.N + n] = h;
+    return __half2float(h);
+  }
+  float o = v[0];
+  if (a.row_scale) o *= a.row_scale[r] * ts[0];
+  reinterpret_cast<float*>(a.out)[(size_t)r * a.N + n] = o;
+  return o;
 }
 
 template <int NMAT, int NT8>
-constexpr size_t smem_bytes() {
-  return (size_t)kWarps * kStages * Slots<NMAT, NT8>::kItems * 32 * 16 +
-         (size_t)kWarps * NMAT * kRowsPerCta * kPartStride * 4;
+__global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? 3 : 2) expert_gemv_kernel(const __grid_constant__ CUtensorMap tm_w2,
+                                                                   const __grid_constant__ CUtensorMap tm_w3,
+                                                                   const __grid_constant__ CUtensorMap tm_w4,
+                                                                   const __grid_constant__ CUtensorMap tm_x,
+                                                                   const __grid_constant__ CUtensorMap tm_s,
+                                                                   const GemvArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const StageLayout& SL = a.st;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SL.stages * SL.bytes);
+  uint64_t* empty = full + kMaxStages;
+  ItemDesc* slot = reinterpret_cast<ItemDesc*>(empty + kMaxStages);  // item starting at a stage
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(slot + kMaxStages);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < SL.stages; ++st) {
+      ptx::mbar_init(&full[st], 1);
+      ptx::mbar_init(&empty[st], kConsumers);
+    }
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == kProducer && lane == 0) {
+    ptx::prefetch_tmap(&tm_w2);
+    ptx::prefetch_tmap(&tm_w3);
+    ptx::prefetch_tmap(&tm_w4);
+    ptx::prefetch_tmap(&tm_x);
+    if (a.sums) ptx::prefetch_tmap(&tm_s);
+  }
+  __syncthreads();
+
+  const int NB = a.N / kBlockRows, KT = a.K / 128;
+  const int nchunks = *a.chunk_count;
+  const int total = nchunks * NB * a.P;
+  const LayerHdr L = hdr_view(a.packed, a.E, a.H, a.F);
+  bool ok = true;
+
+  if (warp == kProducer) {
+    // Items are taken from a global counter (dynamic balance), one item ahead:
+    // the next item's index and sources load while this item's tiles are issued.
+    int stage = 0;
+    uint32_t phase = 0, armed = 0, armed_par = 0;
+    int nxt = 0, gtile = 0, gitem = 0;
+    if (lane == 0) nxt = atomicAdd(a.work, 1);
+    nxt = __shfl_sync(0xffffffffu, nxt, 0);
+    ItemSrc<NMAT> cur, ahead;
+    load_item<NMAT, NT8>(ahead, nxt, total, nchunks, a, L, KT);
+    while (ok) {
+      cur = ahead;
+      const bool done = cur.d.it < 0;
+      if (!done) {
+        if (lane == 0) nxt = atomicAdd(a.work, 1);
+        nxt = __shfl_sync(0xffffffffu, nxt, 0);
+      }
+      const int ntiles = done ? 1 : cur.d.ntiles;
+      for (int kt = 0; kt < ntiles; ++kt) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kGemvWait))) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) gtrace(a.trace, 0, gtile);
+        if (lane == 0) {
+          uint8_t* sb = smem + stage * SL.bytes;
+          if (kt == 0) slot[stage] = cur.d;
+          if (done) {
+            ptx::mbar_arrive(&full[stage]);
+          } else {
+            ptx::mbar_arrive_expect_tx(&full[stage], cur.bytes);
+            const int k = cur.kt0 + kt;
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m) {
+              const int z = cur.z0[m] + k * 4 * cur.wpg[m];
+              const CUtensorMap* map = map_of(cur.wpg[m], &tm_w2, &tm_w3, &tm_w4);
+              tma_load_3d(sb + SL.code_off[m], map, 0, 0, z, &full[stage]);
+              tma_load_3d(sb + SL.code_off[m] + SL.box[m], map, 0, 2, z, &full[stage]);
+              ptx::bulk_load(sb + SL.scale_off[m], cur.sptr[m] + (size_t)k * 1024u, 1024u, &full[stage]);
+            }
+            ptx::tma_load_2d(sb + SL.x_off, &tm_x, k * 128, cur.d.row0, &full[stage]);
+            if (a.sums) ptx::tma_load_2d(sb + SL.sum_off, &tm_s, k * 4, cur.d.row0, &full[stage]);
+          }
+          gtrace(a.trace, 1, gtile);
+        }
+        ++gtile;
+        __syncwarp();
+        if (!done) {
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+        } else {
+          armed &= ~(1u << stage);  // released by the consumers: its last copy has landed
+        }
+        if (++stage == SL.stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        if (kt == 0 && !done) {
+          load_item<NMAT, NT8>(ahead, nxt, total, nchunks, a, L, KT);
+          if (lane == 0) gtrace(a.trace, 4, gitem);
+        }
+      }
+      ++gitem;
+      if (done) break;
+    }
+    // No copy may still be landing when the CTA exits.  Without an abort every
+    // armed stage was consumed; after one, consumers skip their waits, so wait here.
+    if (lane == 0 && (!ok || *abort_flag))
+      for (int st = 0; st < SL.stages; ++st)
+        if (armed & (1u << st)) mbar_drain(&full[st], (armed_par >> st) & 1u);
+    __syncwarp();
+  } else {
+    const int s = warp, g = lane >> 2, c = lane & 3;
+    int stage = 0, gtile = 0, gitem = 0;
+    uint32_t phase = 0;
+    while (true) {
+      // first stage of the next item (or the end marker); all consumer warps agree
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&full[stage], phase, abort_flag, kGemvWait))) *abort_flag = 1;
+      consumer_sync();
+      if (*abort_flag) {
+        ok = false;
+        break;
+      }
+      const ItemDesc w = slot[stage];
+      if (w.it < 0) break;
+      if (threadIdx.x == 0) gtrace(a.trace, 6, gitem);
+      const int row0 = w.row0, rows = w.rows, ntiles = w.ntiles;
+      const int fm[2] = {w.f0, w.f1};
+      const float ts[2] = {w.ts0, w.ts1};
+      float fscale[2];
+#pragma unroll
+      for (int m = 0; m < 2; ++m) fscale[m] = fm[m] == MOE_FMT_NVFP4 ? 1.0f : 16777216.0f;  // integer sums carry 2^-24
+      float acc[NMAT][2][NT8][4];
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int nt = 0; nt < NT8; ++nt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[m][t][nt][j] = 0.0f;
+      switch (fm[0]) {
+        case MOE_FMT_INT2: consume_f1<NMAT, NT8, MOE_FMT_INT2>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile); break;
+        case MOE_FMT_INT3: consume_f1<NMAT, NT8, MOE_FMT_INT3>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile); break;
+        case MOE_FMT_INT4: consume_f1<NMAT, NT8, MOE_FMT_INT4>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile); break;
+        default: consume_f1<NMAT, NT8, MOE_FMT_NVFP4>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile); break;
+      }
+      // lane outputs: weight row nl = 32s + 4g + 2t + (j >> 1), token row nt*8 + 2c + (j & 1)
+      if (ok && a.P == 1) {
+#pragma unroll
+        for (int nt = 0; nt < NT8; ++nt) {
+          float hs[2] = {0.0f, 0.0f};  // this lane's part of the group sums of h for tokens 2c, 2c+1
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int tk = nt * 8 + 2 * c + (j & 1);
+              if (tk < rows) {
+                float v[NMAT];
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m) v[m] = acc[m][t][nt][j] * fscale[m];
+                hs[j & 1] += store_output<NMAT>(a, row0 + tk, w.nb * kBlockRows + 32 * s + 4 * g + 2 * t + (j >> 1),
+                                                v, ts);
+              }
+            }
+          if (a.out_sum) {  // warp s owns the 32 weight rows of one down-projection input group
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+              hs[0] += __shfl_xor_sync(0xffffffffu, hs[0], o);
+              hs[1] += __shfl_xor_sync(0xffffffffu, hs[1], o);
+            }
+            const int grp = (w.nb * kBlockRows + 32 * s) / 32, G = a.N / 32;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int tk = nt * 8 + 2 * c + u;
+              if (g == 0 && tk < rows) a.out_sum[(size_t)(row0 + tk) * G + grp] = hs[u];
+            }
+          }
+        }
+      } else if (ok) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int nt = 0; nt < NT8; ++nt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int tk = nt * 8 + 2 * c + (j & 1);
+              if (tk < rows) {
+                const int n = w.nb * kBlockRows + 32 * s + 4 * g + 2 * t + (j >> 1);
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m)
+                  a.part[(((size_t)w.p * a.R + row0 + tk) * NMAT + m) * a.N + n] = acc[m][t][nt][j] * fscale[m];
+              }
+            }
+      }
+      if (threadIdx.x == 0) gtrace(a.trace, 7, gitem);
+      ++gitem;
+    }
+  }
+
+  if (!ok) {
+    *abort_flag = 1;
+    if (a.status) atomicExch(a.status, (int32_t)MOE_ERR_TIMEOUT);
+  }
+  __syncthreads();
 }
 
-int sm_count_gemv() {
+// Split-K epilogue: block (r, b) sums the P parts of outputs 256b..256b+255 of
+// expert row r in order, then applies SwiGLU (gate/up) or writes o (down).
+// Gate/up of integer layers also writes the group sums of h for the down GEMV.
+template <int NMAT>
+__global__ void __launch_bounds__(256) gemv_fixup_kernel(GemvArgs a, const int32_t* idx) {
+  const int r = blockIdx.x;
+  const int e = idx[a.perm[r]];
+  const LayerHdr L = hdr_view(a.packed, a.E, a.H, a.F);
+  float ts[2];
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    const int i = e * 3 + a.proj + (m < NMAT ? m : 0);
+    ts[m] = L.fmt[i] == MOE_FMT_NVFP4 ? L.tscale[i] : 1.0f;
+  }
+  const int lane = threadIdx.x & 31;
+  const int n0 = blockIdx.y * 256 + threadIdx.x - lane;  // warp-uniform: 32 outputs = one group
+  if (n0 < a.N) {
+    const int n = n0 + lane;
+    float v[NMAT];
+#pragma unroll
+    for (int m = 0; m < NMAT; ++m) {
+      float sum = 0.0f;
+      for (int q = 0; q < a.P; ++q) sum += a.part[(((size_t)q * a.R + r) * NMAT + m) * a.N + n];
+      v[m] = sum;
+    }
+    float h = store_output<NMAT>(a, r, n, v, ts);
+    if (a.out_sum) {
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) h += __shfl_xor_sync(0xffffffffu, h, o);
+      if (lane == 0) a.out_sum[(size_t)r * (a.N / 32) + n0 / 32] = h;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 gemv_tmap_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+int gemv_sm_count() {
   static int n[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
@@ -455,52 +672,171 @@ int sm_count_gemv() {
   return n[dev];
 }
 
+// The packed buffer as 3D tensor of u32: x = 32 words (128 bytes), y = 4 such
+// lines per 512-byte word row, z = word rows.  Box: 32 x 2 x (4 groups * wpg).
+bool encode_code_map(CUtensorMap* map, const uint8_t* packed, uint64_t packed_bytes, int wpg) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = gemv_tmap_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {32u, 4u, (cuuint64_t)(packed_bytes / 512u)};
+  const cuuint64_t strides[2] = {128u, 512u};
+  const cuuint32_t box[3] = {32u, 2u, (cuuint32_t)(4 * wpg)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t*>(packed), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A row-major [rows][cols] matrix of 2- or 4-byte elements; box of box_cols x box_rows.
+bool encode_rows_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize, int rows, int cols,
+                     int box_cols, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = gemv_tmap_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * (cuuint64_t)esize};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Stage layout for the widest formats of the layer at each matrix position.
+// Shared memory is budgeted for three CTAs per SM with one token tile and two
+// with two (whose registers allow no more).
+StageLayout stage_layout(int nmat, int nt8, const int* wmax) {
+  StageLayout L{};
+  int off = 0;
+  for (int m = 0; m < nmat; ++m) {
+    L.box[m] = 1024 * wmax[m];
+    L.code_off[m] = off;
+    off += 2 * L.box[m];
+  }
+  for (int m = 0; m < nmat; ++m) {
+    L.scale_off[m] = off;
+    off += 1024;
+  }
+  L.x_off = off;
+  off += nt8 * 8 * 256;
+  L.sum_off = off;
+  off += nt8 * 8 * 16;
+  L.bytes = (off + 1023) / 1024 * 1024;
+  const int cta_per_sm = nt8 == 1 ? 3 : 2;
+  const int budget = 227 * 1024 / cta_per_sm - 1024 - kCtrlBytes - 1024;  // minus alignment, control, per-CTA reserve
+  L.stages = budget / L.bytes;
+  if (L.stages > kMaxStages) L.stages = kMaxStages;
+  if (L.stages < 2) L.stages = 2;
+  return L;
+}
+
 template <int NMAT, int NT8>
-cudaError_t launch_n(const GemvArgs& g, int max_chunks, cudaStream_t stream) {
+cudaError_t launch_n(GemvArgs g, const uint8_t* packed, uint64_t packed_bytes, const void* act, const float* sums,
+                     const int* wmax, int max_chunks, cudaStream_t stream) {
+  CUtensorMap m2, m3, m4, mx, ms;
+  if (!encode_code_map(&m2, packed, packed_bytes, 2) || !encode_code_map(&m3, packed, packed_bytes, 3) ||
+      !encode_code_map(&m4, packed, packed_bytes, 4) ||
+      !encode_rows_map(&mx, act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, g.R, g.K, 128, 8 * NT8))
+    return cudaErrorInvalidValue;
+  g.sums = sums != nullptr;
+  if (g.sums) {
+    if (!encode_rows_map(&ms, sums, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, g.R, g.K / 32, 4, 8 * NT8))
+      return cudaErrorInvalidValue;
+  } else {
+    ms = mx;  // unused
+  }
+  g.st = stage_layout(NMAT, NT8, wmax);
+  const int smem = g.st.stages * g.st.bytes + 1024 + kCtrlBytes;
   auto kern = expert_gemv_kernel<NMAT, NT8>;
-  constexpr size_t kSmemBytes = smem_bytes<NMAT, NT8>();
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   int per_sm = 0;
-  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32 * kWarps, kSmemBytes);
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGemvThreads, smem);
   if (err != cudaSuccess) return err;
-  const long long items = (long long)max_chunks * (g.N / kRowsPerCta);
-  long long grid = (long long)sm_count_gemv() * (per_sm > 0 ? per_sm : 1);
+  const long long items = (long long)max_chunks * (g.N / kBlockRows) * g.P;
+  long long grid = (long long)gemv_sm_count() * (per_sm > 0 ? per_sm : 1);
   if (grid > items) grid = items;
-  kern<<<(unsigned)grid, 32 * kWarps, kSmemBytes, stream>>>(g);
+  if (grid < 1) grid = 1;
+  kern<<<(unsigned)grid, kGemvThreads, smem, stream>>>(m2, m3, m4, mx, ms, g);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_expert_gemv(const uint8_t* packed, int E, int H, int F, int k, bool fp4, bool gateup,
-                               int max_chunks, int chunk_rows, const Workspace& ws, cudaStream_t stream) {
+int gemv_split(long long R, int E, int N, int K, int nmat) {
+  const long long chunks = R < E ? R : E;  // active experts at most
+  long long base = chunks * (N / kBlockRows);
+  if (base < 1) base = 1;
+  const long long target = 4LL * 3 * 148;  // about four items per CTA at three CTAs per SM
+  long long P = (target + base - 1) / base;
+  const long long per_part = R * (long long)N * nmat * 4;
+  const long long mem_cap = (8LL << 20) / (per_part > 0 ? per_part : 1);
+  const int kt = K / 128;
+  long long cap = kt / 4 > 1 ? kt / 4 : 1;  // parts of at least four tiles
+  if (cap > kMaxSplit) cap = kMaxSplit;
+  if (P > cap) P = cap;
+  if (P > mem_cap) P = mem_cap;
+  return P < 1 ? 1 : (int)P;
+}
+
+cudaError_t launch_expert_gemv(const uint8_t* packed, uint64_t packed_bytes, const uint8_t* fmt_host, int E, int H,
+                               int F, int R, int k, bool fp4, bool gateup, int max_chunks, int chunk_rows,
+                               const Workspace& ws, int32_t* status, uint64_t* trace, cudaStream_t stream) {
   GemvArgs g{};
+  g.trace = reinterpret_cast<unsigned long long*>(trace);
   g.packed = packed;
   g.E = E;
   g.H = H;
   g.F = F;
+  g.topk = k;
+  g.R = R;
   g.chunks = ws.chunks;
   g.chunk_count = ws.chunk_count;
   g.perm = ws.perm;
-  g.topk = k;
-  const bool two = chunk_rows > 8;
+  g.part = ws.part;
+  g.work = ws.counters + (gateup ? 0 : 1);
+  g.status = status;
+  const void* act;
+  const float* sums;
+  int wmax[2] = {2, 2};
+  for (int e = 0; e < E; ++e)
+    for (int m = 0; m < (gateup ? 2 : 1); ++m) {
+      const int w = fmt_words(fmt_host[e * 3 + (gateup ? m : 2)]);
+      if (w > wmax[m]) wmax[m] = w;
+    }
   if (gateup) {
     g.N = F;
     g.K = H;
     g.proj = 0;
-    g.act = reinterpret_cast<const __half*>(ws.xs);
+    act = ws.xs;
+    sums = fp4 ? nullptr : ws.xsum;
     g.row_scale = fp4 ? ws.sx : nullptr;
     g.out = ws.h;
-    return two ? launch_n<2, 2>(g, max_chunks, stream) : launch_n<2, 1>(g, max_chunks, stream);
+    g.out_sum = fp4 ? nullptr : ws.hsum;
+  } else {
+    g.N = H;
+    g.K = F;
+    g.proj = 2;
+    act = fp4 ? ws.hb : ws.h;
+    sums = fp4 ? nullptr : ws.hsum;
+    g.row_scale = fp4 ? ws.sh : nullptr;
+    g.out = ws.o;
+    g.out_sum = nullptr;
   }
-  g.N = H;
-  g.K = F;
-  g.proj = 2;
-  g.act = reinterpret_cast<const __half*>(fp4 ? ws.hb : ws.h);
-  g.row_scale = fp4 ? ws.sh : nullptr;
-  g.out = ws.o;
-  return two ? launch_n<1, 2>(g, max_chunks, stream) : launch_n<1, 1>(g, max_chunks, stream);
+  const int nmat = gateup ? 2 : 1;
+  g.P = gemv_split(R, E, g.N, g.K, nmat);
+  const bool two = chunk_rows > 8;
+  cudaError_t err;
+  if (gateup)
+    err = two ? launch_n<2, 2>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream)
+              : launch_n<2, 1>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream);
+  else
+    err = two ? launch_n<1, 2>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream)
+              : launch_n<1, 1>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream);
+  if (err != cudaSuccess || g.P == 1) return err;
+  if (gateup)
+    gemv_fixup_kernel<2><<<dim3(R, (g.N + 255) / 256), 256, 0, stream>>>(g, ws.idx);
+  else
+    gemv_fixup_kernel<1><<<dim3(R, (g.N + 255) / 256), 256, 0, stream>>>(g, ws.idx);
+  return cudaGetLastError();
 }
 
 }  // namespace moe

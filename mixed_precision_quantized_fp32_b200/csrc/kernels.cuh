@@ -24,8 +24,13 @@ cudaError_t launch_act_quant_h(int R, int F, const Workspace& ws, uint8_t* dbg_h
 cudaError_t launch_expert_gemm_tc(const uint8_t* packed, int E, int H, int F, int T, int k, bool fp4, bool gateup,
                                   const Workspace& ws, int32_t* status, uint64_t* trace, cudaStream_t stream);
 
-cudaError_t launch_expert_gemv(const uint8_t* packed, int E, int H, int F, int k, bool fp4, bool gateup,
-                               int max_chunks, int chunk_rows, const Workspace& ws, cudaStream_t stream);
+// K parts of the decode GEMV for R expert rows on an N x K projection (nmat
+// matrices); the workspace holds P*R*N*nmat fp32 partials when P > 1.
+int gemv_split(long long R, int E, int N, int K, int nmat);
+
+cudaError_t launch_expert_gemv(const uint8_t* packed, uint64_t packed_bytes, const uint8_t* fmt_host, int E, int H,
+                               int F, int R, int k, bool fp4, bool gateup, int max_chunks, int chunk_rows,
+                               const Workspace& ws, int32_t* status, uint64_t* trace, cudaStream_t stream);
 
 cudaError_t launch_combine(int T, int k, int H, const Workspace& ws, __nv_bfloat16* y, cudaStream_t stream);
 

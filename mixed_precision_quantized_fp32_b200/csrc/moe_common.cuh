@@ -134,6 +134,11 @@ struct Workspace {
   float* sh;           // [T*k]
   float* o;            // [T*k*H] fp32 expert outputs, sorted rows
   int32_t* status;     // [1]
+  float* part;         // decode GEMV split-K partial sums (null when not split)
+  int32_t* counters;   // [counter_len] decode GEMV work counters (gate/up, down)
+  int counter_len;
+  float* xsum;         // [T*k][H/32] group sums of the gathered fp16 activations (integer layers)
+  float* hsum;         // [T*k][F/32] group sums of the fp16 SwiGLU outputs (integer layers)
 };
 
 }  // namespace moe

@@ -108,9 +108,19 @@ __global__ void __launch_bounds__(kPermBlock) perm_scatter_kernel(const int32_t*
   if (dbg_inv) dbg_inv[i] = row;
 }
 
-// Gather x rows into expert-sorted order as fp16 (integer-format layers).
+// Zero the decode GEMV's work counters (the workspace starts undefined).
+__device__ __forceinline__ void zero_counters(int32_t* counters, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) counters[i] = 0;
+}
+
+// Gather x rows into expert-sorted order as fp16 (integer-format layers), with
+// the sum of every group of 32 fp16 values (fp32) for the decode GEMV's code
+// offset term (xsum may be null).  blockDim.x is a multiple of 32 and H of 128,
+// so the four threads of a group sit in one warp at every step.
 __global__ void gather_f16_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm,
-                                  int R, int H, int k, __half* __restrict__ xs) {
+                                  int R, int H, int k, __half* __restrict__ xs, float* __restrict__ xsum,
+                                  int32_t* counters, int n_counters) {
+  zero_counters(counters, n_counters);
   const int r = blockIdx.x;
   const int t = perm[r] / k;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
@@ -120,9 +130,17 @@ __global__ void gather_f16_kernel(const __nv_bfloat16* __restrict__ x, const int
     const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v);
     uint4 o;
     __half2* h2 = reinterpret_cast<__half2*>(&o);
+    float sum = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) h2[i] = __float22half2_rn(__bfloat1622float2(b2[i]));
+    for (int i = 0; i < 4; ++i) {
+      h2[i] = __float22half2_rn(__bfloat1622float2(b2[i]));
+      const float2 f = __half22float2(h2[i]);
+      sum += f.x + f.y;
+    }
     dst[c] = o;
+    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+    if (xsum && (c & 3) == 0) xsum[(size_t)r * (H / 32) + c / 4] = sum;
   }
 }
 
@@ -168,7 +186,8 @@ __global__ void act_quant_x_kernel(const __nv_bfloat16* __restrict__ x, int H, u
 
 // Gather e4m3 activation codes into sorted rows as exact fp16 values.
 __global__ void gather_fp8_kernel(const uint8_t* __restrict__ xq, const int32_t* __restrict__ perm, int R,
-                                  int H, int k, __half* __restrict__ xs) {
+                                  int H, int k, __half* __restrict__ xs, int32_t* counters, int n_counters) {
+  zero_counters(counters, n_counters);
   const int r = blockIdx.x;
   const int t = perm[r] / k;
   const uint2* src = reinterpret_cast<const uint2*>(xq + (size_t)t * H);
@@ -226,9 +245,11 @@ cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4,
   const int R = T * k;
   if (fp4) {
     act_quant_x_kernel<<<T, 256, 0, stream>>>(x, H, ws.xq, ws.sx, dbg_xq, dbg_sx);
-    gather_fp8_kernel<<<R, 128, 0, stream>>>(ws.xq, ws.perm, R, H, k, (__half*)ws.xs);
+    gather_fp8_kernel<<<R, 128, 0, stream>>>(ws.xq, ws.perm, R, H, k, (__half*)ws.xs, ws.counters,
+                                             ws.counter_len);
   } else {
-    gather_f16_kernel<<<R, 128, 0, stream>>>(x, ws.perm, R, H, k, (__half*)ws.xs);
+    gather_f16_kernel<<<R, 128, 0, stream>>>(x, ws.perm, R, H, k, (__half*)ws.xs, ws.xsum, ws.counters,
+                                             ws.counter_len);
   }
   return cudaGetLastError();
 }
