@@ -72,6 +72,8 @@ struct TcArgs {
   int E, H, F;
   int N, K;                // output rows (weight rows) and inputs of this GEMM
   int proj;                // 0: gate+up with SwiGLU epilogue; 2: down
+  int pair;                // down with NMAT == 2: the two "matrices" are weight tiles 2p, 2p+1 of one
+                           // matrix, sharing each activation tile (half the activation reads per FLOP)
   const int32_t* chunks;   // (expert, first row, rows) triples
   const int32_t* chunk_count;
   const float* row_scale;  // NVFP4: gate/up -> per-token sx, down -> per-row sh; null for integer layers
@@ -87,8 +89,8 @@ __device__ __forceinline__ void trace_stamp(unsigned long long* tr, int ev, int 
   if (tr && blockIdx.x == 0 && i < MOE_TRACE_STAGES) tr[ev * MOE_TRACE_STAGES + i] = (unsigned long long)clock64();
 }
 
-__device__ __forceinline__ uint32_t h2sub(uint32_t a, uint32_t b) {
-  __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+__device__ __forceinline__ uint32_t h2fma(uint32_t a, uint32_t b, uint32_t c) {
+  __half2 r = __hfma2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b), *reinterpret_cast<__half2*>(&c));
   return *reinterpret_cast<uint32_t*>(&r);
 }
 __device__ __forceinline__ uint32_t h2mul(uint32_t a, uint32_t b) {
@@ -120,25 +122,32 @@ __device__ __forceinline__ uint4 dequant_chunk(const uint32_t* __restrict__ code
 #pragma unroll
     for (int b = 0; b < 4; ++b) v[b] = h2mul(v[b], p);  // exact: <= 6 significant bits
   } else {
+    // A field u of weight f (bit position log2 f of both half-words) OR'ed into
+    // the mantissa of 1024.0 reads as 1024 + f*u; one FMA with 1/f and
+    // -(1024/f + offset) gives q = u - offset exactly, then one multiply by the
+    // group scale rounds s*q once.
     const uint32_t s = reinterpret_cast<const uint16_t*>(scales)[n];
     const uint32_t s2 = s | (s << 16);
+    constexpr uint32_t kMagic = 0x64006400u;
     if (FMT == MOE_FMT_INT4) {
-      const uint32_t w = codes[c * 128 + n];
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        v[j] = h2mul(h2sub(((w >> (4 * j)) & 0x000F000Fu) | 0x64006400u, 0x64086408u), s2);
-    } else if (FMT == MOE_FMT_INT2) {
-      const uint32_t w = codes[(c >> 1) * 128 + n] >> (8 * (c & 1));
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        v[j] = h2mul(h2sub(((w >> (2 * j)) & 0x00030003u) | 0x64006400u, 0x64026402u), s2);
-    } else {  // INT3: low bits as INT2, bit 2 of pair J at bits J and 16+J of word 2
+      const uint32_t w = codes[c * 128 + n], w8 = w >> 8;
+      v[0] = h2mul(h2fma((w & 0x000F000Fu) | kMagic, 0x3C003C00u, 0xE408E408u), s2);   // u - 8
+      v[1] = h2mul(h2fma((w & 0x00F000F0u) | kMagic, 0x2C002C00u, 0xD480D480u), s2);   // 16u / 16 + 64 - 72
+      v[2] = h2mul(h2fma((w8 & 0x000F000Fu) | kMagic, 0x3C003C00u, 0xE408E408u), s2);
+      v[3] = h2mul(h2fma((w8 & 0x00F000F0u) | kMagic, 0x2C002C00u, 0xD480D480u), s2);
+    } else {
+      // fields of pair j at bits 2j (weight 4^j); INT3 adds bit 2 of the pair's
+      // codes from word 2 (pair m at bits m, 16+m), moved to bit 2j+2
+      constexpr uint32_t kMul[4] = {0x3C003C00u, 0x34003400u, 0x2C002C00u, 0x24002400u};        // 4^-j
+      constexpr uint32_t kSub2[4] = {0xE402E402u, 0xDC08DC08u, 0xD420D420u, 0xCC80CC80u};       // -(1024/4^j + 2)
+      constexpr uint32_t kSub3[4] = {0xE404E404u, 0xDC10DC10u, 0xD440D440u, 0xCD00CD00u};       // -(1024/4^j + 4)
       const uint32_t lo = codes[(c >> 1) * 128 + n] >> (8 * (c & 1));
-      const uint32_t hi = codes[2 * 128 + n] >> (4 * c);
+      const uint32_t hh = FMT == MOE_FMT_INT3 ? codes[2 * 128 + n] >> (4 * c) : 0u;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint32_t u = ((lo >> (2 * j)) & 0x00030003u) | (((hi >> j) & 0x00010001u) << 2);
-        v[j] = h2mul(h2sub(u | 0x64006400u, 0x64046404u), s2);
+        uint32_t raw = (lo & (0x00030003u << (2 * j))) | kMagic;
+        if (FMT == MOE_FMT_INT3) raw |= (hh << (j + 2)) & (0x00040004u << (2 * j));
+        v[j] = h2mul(h2fma(raw, kMul[j], FMT == MOE_FMT_INT3 ? kSub3[j] : kSub2[j]), s2);
       }
     }
   }
@@ -279,7 +288,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int m_tiles = a.N / kTcBM;
+  const int m_tiles = a.N / kTcBM / (a.pair ? 2 : 1);  // work items per chunk
   const int total = *a.chunk_count * m_tiles;
   const int ksteps = a.K / kTcBK;
   const LayerHdr L = hdr_view(a.packed, a.E, a.H, a.F);
@@ -307,11 +316,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t bytes = C::kBBytes;
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) {
-        const int i = e * 3 + a.proj + m;
+        const int i = e * 3 + a.proj + (a.pair ? 0 : m);
+        const int mtm = a.pair ? 2 * mt + m : mt;
         const int f = L.fmt[i];
         cbytes[m] = (uint32_t)(fmt_words(f) * 512 * kGroups);
-        cptr[m] = L.base + L.code_off[i] + code_stage_offset(mt, 0, a.K, fmt_words(f));
-        sptr[m] = L.base + L.scale_off[i] + scale_stage_offset(mt, 0, a.K, f);
+        cptr[m] = L.base + L.code_off[i] + code_stage_offset(mtm, 0, a.K, fmt_words(f));
+        sptr[m] = L.base + L.scale_off[i] + scale_stage_offset(mtm, 0, a.K, f);
         bytes += cbytes[m] + (uint32_t)C::kScaleBytes;
       }
       for (int ks = 0; ks < ksteps; ++ks) {
@@ -424,7 +434,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       float tsc[NMAT];
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) {
-        const int i = e * 3 + a.proj + m;
+        const int i = e * 3 + a.proj + (a.pair ? 0 : m);
         fmt[m] = L.fmt[i];
         tsc[m] = fmt[m] == MOE_FMT_NVFP4 ? L.tscale[i] : 1.0f;
       }
@@ -441,7 +451,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       acc_phase ^= 1u;
       if (threadIdx.x == 0) trace_stamp(a.trace, 6, item);
       ptx::tc_fence_after();
-      const int nrow = mt * kTcBM + q * 32 + lane;
+      const int nrow = (a.pair ? 2 * mt : mt) * kTcBM + q * 32 + lane;
       const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
       for (int cb = cq * kColsPerWarp; cb < cq * kColsPerWarp + kColsPerWarp && cb < rows; cb += 16) {
         uint32_t r0[16], r1[16];
@@ -453,7 +463,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int tok = cb + j;
           if (tok >= rows) break;
           const int r = row0 + tok;
-          if (NMAT == 2) {
+          if (NMAT == 2 && a.pair) {  // two weight tiles of the down matrix: rows nrow and nrow + 128
+            float o0 = __uint_as_float(r0[j]), o1 = __uint_as_float(r1[j]);
+            if (a.row_scale) {
+              const float sc = a.row_scale[r] * tsc[0];
+              o0 *= sc;
+              o1 *= sc;
+            }
+            reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = o0;
+            reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow + kTcBM] = o1;
+          } else if (NMAT == 2) {
             float g = __uint_as_float(r0[j]), u = __uint_as_float(r1[j]);
             if (a.row_scale) {
               const float sx = a.row_scale[a.perm[r] / a.topk];
@@ -563,6 +582,10 @@ cudaError_t launch_expert_gemm_tc(const uint8_t* packed, int E, int H, int F, in
   a.proj = 2;
   a.row_scale = fp4 ? ws.sh : nullptr;
   a.out = ws.o;
+  if ((H / kTcBM) % 2 == 0) {  // pairs of weight tiles share each activation tile
+    a.pair = 1;
+    return launch_tc<2>(a, fp4 ? ws.hb : ws.h, R, stream);
+  }
   return launch_tc<1>(a, fp4 ? ws.hb : ws.h, R, stream);
 }
 
