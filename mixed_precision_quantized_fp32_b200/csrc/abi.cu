@@ -73,7 +73,9 @@ uint64_t carve(uint8_t* base, int T, int k, int E, int H, int F, bool fp4, const
     return p;
   };
   Workspace ws{};
-  ws.logits = (float*)take((uint64_t)T * E * 4);
+  const int rparts = router_parts(T, H, E);
+  ws.logits = (float*)take((uint64_t)(rparts > 1 ? rparts : 1) * T * E * 4);
+  if (rparts > 0) ws.wsplit = (__nv_bfloat16*)take((uint64_t)3 * E * H * 2);
   ws.idx = (int32_t*)take(R * 4);
   ws.wts = (float*)take(R * 4);
   ws.counts = (int32_t*)take((uint64_t)E * 4);

@@ -8,6 +8,9 @@ cudaError_t launch_pack(const float* W, int e0, int ne, int E, int H, int F, con
                         uint8_t* out, const uint64_t* code_off, const uint64_t* scale_off,
                         cudaStream_t stream);
 
+// Router K parts (0: warp kernel, no parts); the workspace holds max(1, parts) logit planes.
+int router_parts(long long T, int H, int E);
+
 cudaError_t launch_router_topk(const __nv_bfloat16* x, const float* Wr, const float* b, int T, int H,
                                int E, int k, const Workspace& ws, int32_t* dbg_idx, float* dbg_w,
                                cudaStream_t stream);

@@ -114,7 +114,8 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {
 
 // Workspace layout shared by the host ABI and the kernels.
 struct Workspace {
-  float* logits;       // [T*E]
+  float* logits;       // [parts][T*E] (parts: router K parts, at least 1)
+  __nv_bfloat16* wsplit;  // [3][E*H] bf16 terms of the router weights (router GEMM only)
   int32_t* idx;        // [T*k]
   float* wts;          // [T*k]
   int32_t* counts;     // [E]

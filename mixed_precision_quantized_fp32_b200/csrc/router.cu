@@ -38,103 +38,166 @@ __global__ void router_warp_kernel(const __nv_bfloat16* __restrict__ x, const fl
 }
 
 // ---------------------------------------------------------------- router, many tokens
-// Tiled fp32 GEMM: block tile 64 tokens x TE experts, k-tile 32; 256 threads,
-// each computing 4 tokens x TE/16 experts.  Each k-tile is summed on its own and
-// the tile sums are added with Kahan compensation, so the rounding error stays
-// near that of a pairwise sum even for H = 12288.
-template <int TE>
-__global__ void __launch_bounds__(256) router_tile_kernel(const __nv_bfloat16* __restrict__ x,
-                                                          const float* __restrict__ Wr,
-                                                          const float* __restrict__ b, int T, int H,
-                                                          int E, float* __restrict__ logits) {
-  constexpr int TT = 64, BK = 32, PE = TE / 16;
-  __shared__ float xs[BK][TT + 4];
-  __shared__ float ws[BK][TE + 4];
-  const int tid = threadIdx.x;
-  const int t0 = blockIdx.x * TT, e0 = blockIdx.y * TE;
-  const int ty = tid >> 4, tx = tid & 15;
-  float acc[4][PE], comp[4][PE];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < PE; ++j) acc[i][j] = comp[i][j] = 0.0f;
+// The fp32 router weights are split exactly into three bf16 terms
+// (w = hi + mid + lo up to the last bit of lo), so with bf16 x every product
+// x * term is exact and bf16 tensor-core MMAs with fp32 accumulation compute
+// the fp32 dot product.  The MMAs accumulate chunks of 64 inputs in
+// registers; chunk sums are added with Kahan compensation, so the rounding
+// error stays near that of a pairwise sum even for H = 12288.
 
-  for (int k0 = 0; k0 < H; k0 += BK) {
-    {  // x tile: 64 tokens x 32 h = 256 chunks of 8 bf16
-      const int tt = tid >> 2, hh = (tid & 3) * 8;
-      const int t = t0 + tt;
-      float v[8];
-      if (t < T) {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + k0 + hh));
-        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+// Wr fp32 [E][H] -> Wb bf16 [3][E][H] (hi, mid, lo).
+__global__ void router_split_kernel(const float* __restrict__ Wr, long long n, __nv_bfloat16* __restrict__ Wb) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float w = Wr[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = __fsub_rn(w, __bfloat162float(hi));
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = __fsub_rn(r1, __bfloat162float(mid));
+    Wb[i] = hi;
+    Wb[n + i] = mid;
+    Wb[2 * n + i] = __float2bfloat16_rn(r2);
+  }
+}
+
+constexpr int kRT = 128, kRE = 64, kRK = 32, kRStages = 3, kRChunk = 64;
+constexpr int kRRow = kRK + 8;  // bf16 per smem row: 80 bytes, conflict-free ldmatrix
+constexpr int kRStageA = kRT * kRRow, kRStageB = 3 * kRE * kRRow;  // bf16 elements
+constexpr int kRSmem = kRStages * (kRStageA + kRStageB) * 2;
+
+__device__ __forceinline__ void cp16z(void* dst, const void* src, bool ok) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(ok ? 16u : 0u)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t* r, const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
+__device__ __forceinline__ void mma_bf16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Block tile 128 tokens x 64 experts, 8 warps of 32 x 32; k-stages of 32 inputs
+// (cp.async, three in flight).  blockIdx.z selects a part of the inputs
+// (split-K for grids smaller than the GPU); each part writes its own logit
+// plane, which the top-k kernel adds in double precision.  The bias goes into
+// plane 0.
+__global__ void __launch_bounds__(256, 2) router_mma_kernel(const __nv_bfloat16* __restrict__ x,
+                                                         const __nv_bfloat16* __restrict__ Wb,
+                                                         const float* __restrict__ b, int T, int H, int E,
+                                                         float* __restrict__ logits) {
+  extern __shared__ __align__(16) __nv_bfloat16 rsm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wm = warp & 3, wn = warp >> 2;
+  const int t0 = blockIdx.x * kRT, e0 = blockIdx.y * kRE;
+  const int nk = H / kRK;
+  const int kb = blockIdx.z * nk / gridDim.z, ke = (blockIdx.z + 1) * nk / gridDim.z;  // k-steps of this part
+  logits += (size_t)blockIdx.z * T * E;
+  if (blockIdx.z > 0) b = nullptr;
+  const size_t plane = (size_t)E * H;
+
+  auto load = [&](int ks, int st) {
+    __nv_bfloat16* A = rsm + st * (kRStageA + kRStageB);
+    __nv_bfloat16* B = A + kRStageA;
+    const int k0 = ks * kRK;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          v[2 * i] = __low2float(p2[i]);
-          v[2 * i + 1] = __high2float(p2[i]);
+    for (int u = 0; u < 2; ++u) {  // A: 128 rows x 4 chunks of 16 bytes
+      const int c = tid + 256 * u, r = c >> 2, q = c & 3;
+      const bool ok = t0 + r < T;
+      cp16z(A + r * kRRow + q * 8, x + (size_t)(ok ? t0 + r : 0) * H + k0 + q * 8, ok);
+    }
+#pragma unroll
+    for (int u = 0; u < 3; ++u) {  // B: 3 planes x 64 rows x 4 chunks
+      const int c = tid + 256 * u, p = c >> 8, r = (c >> 2) & 63, q = c & 3;
+      const bool ok = e0 + r < E;
+      cp16z(B + (p * kRE + r) * kRRow + q * 8, Wb + p * plane + (size_t)(ok ? e0 + r : 0) * H + k0 + q * 8, ok);
+    }
+  };
+
+  float tot[2][4][4], comp[2][4][4], acc[2][4][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) tot[i][j][v] = comp[i][j][v] = acc[i][j][v] = 0.0f;
+
+#pragma unroll
+  for (int st = 0; st < kRStages - 1; ++st) {
+    if (kb + st < ke) load(kb + st, st);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  for (int ks = kb; ks < ke; ++ks) {
+    asm volatile("cp.async.wait_group %0;" ::"n"(kRStages - 2) : "memory");
+    __syncthreads();
+    {  // refill the stage consumed one step ago
+      const int kn = ks + kRStages - 1;
+      if (kn < ke) load(kn, (kn - kb) % kRStages);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    const __nv_bfloat16* A = rsm + ((ks - kb) % kRStages) * (kRStageA + kRStageB);
+    const __nv_bfloat16* B = A + kRStageA;
+#pragma unroll
+    for (int kk = 0; kk < kRK; kk += 16) {
+      uint32_t af[2][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+        ldsm_x4(af[mt], A + (wm * 32 + mt * 16 + (lane & 15)) * kRRow + kk + (lane >> 4) * 8);
+#pragma unroll
+      for (int p = 0; p < 3; ++p) {
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {  // n8 tiles 2np, 2np+1
+          uint32_t bf[4];
+          ldsm_x4(bf, B + (p * kRE + wn * 32 + np * 16 + (lane & 7) + ((lane >> 4) << 3)) * kRRow + kk +
+                          ((lane >> 3) & 1) * 8);
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            mma_bf16(acc[mt][2 * np], af[mt], bf[0], bf[1]);
+            mma_bf16(acc[mt][2 * np + 1], af[mt], bf[2], bf[3]);
+          }
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) xs[hh + i][tt] = v[i];
     }
-    for (int c = tid; c < TE * (BK / 4); c += 256) {  // Wr tile: TE experts x 32 h
-      const int ee = c / (BK / 4), hh = (c % (BK / 4)) * 4;
-      const int e = e0 + ee;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e < E) v = __ldg(reinterpret_cast<const float4*>(Wr + (size_t)e * H + k0 + hh));
-      ws[hh][ee] = v.x;
-      ws[hh + 1][ee] = v.y;
-      ws[hh + 2][ee] = v.z;
-      ws[hh + 3][ee] = v.w;
-    }
-    __syncthreads();
-    float part[4][PE];
+    if ((ks - kb + 1) % (kRChunk / kRK) == 0 || ks + 1 == ke) {  // chunk done: Kahan-add into the totals
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int j = 0; j < PE; ++j) part[i][j] = 0.0f;
-#pragma unroll 8
-    for (int kk = 0; kk < BK; ++kk) {
-      float a[4], w[PE];
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = xs[kk][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < PE; ++j) w[j] = ws[kk][tx * PE + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < PE; ++j) part[i][j] = fmaf(a[i], w[j], part[i][j]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < PE; ++j) {  // Kahan: acc += part
-        const float y = __fsub_rn(part[i][j], comp[i][j]);
-        const float t = __fadd_rn(acc[i][j], y);
-        comp[i][j] = __fsub_rn(__fsub_rn(t, acc[i][j]), y);
-        acc[i][j] = t;
-      }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = t0 + ty * 4 + i;
-    if (t >= T) continue;
-#pragma unroll
-    for (int j = 0; j < PE; ++j) {
-      const int e = e0 + tx * PE + j;
-      if (e < E) logits[(size_t)t * E + e] = b ? acc[i][j] + b[e] : acc[i][j];
+          for (int v = 0; v < 4; ++v) {
+            const float y = __fsub_rn(acc[i][j][v], comp[i][j][v]);
+            const float t = __fadd_rn(tot[i][j][v], y);
+            comp[i][j][v] = __fsub_rn(__fsub_rn(t, tot[i][j][v]), y);
+            tot[i][j][v] = t;
+            acc[i][j][v] = 0.0f;
+          }
     }
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  // accumulator element v of tile (mt, nt): token wm*32 + mt*16 + lane/4 + 8*(v >> 1),
+  // expert wn*32 + nt*8 + 2*(lane%4) + (v & 1)
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int t = t0 + wm * 32 + mt * 16 + (lane >> 2) + 8 * (v >> 1);
+        const int e = e0 + wn * 32 + nt * 8 + 2 * (lane & 3) + (v & 1);
+        if (t < T && e < E) logits[(size_t)t * E + e] = b ? tot[mt][nt][v] + b[e] : tot[mt][nt][v];
+      }
 }
 
 // ---------------------------------------------------------------- top-k + softmax
 // One warp per token.  Expert e lives in lane e%32, slot e/32.  k passes of a
 // warp-wide arg-max over the experts not chosen yet; ties go to the lower
 // expert index; NaN ranks below every number.
-__global__ void topk_softmax_kernel(const float* __restrict__ logits, int T, int E, int k,
+__global__ void topk_softmax_kernel(const float* __restrict__ logits, int nparts, int T, int E, int k,
                                     int32_t* __restrict__ idx, float* __restrict__ wts,
                                     int32_t* __restrict__ dbg_idx, float* __restrict__ dbg_w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -144,7 +207,16 @@ __global__ void topk_softmax_kernel(const float* __restrict__ logits, int T, int
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int e = lane + 32 * i;
-    float l = (e < E) ? logits[(size_t)t * E + e] : -INFINITY;
+    float l = -INFINITY;
+    if (e < E) {
+      if (nparts == 1) {
+        l = logits[(size_t)t * E + e];
+      } else {  // split-K planes of the router GEMM
+        double sum = 0.0;
+        for (int z = 0; z < nparts; ++z) sum += (double)logits[((size_t)z * T + t) * E + e];
+        l = (float)sum;
+      }
+    }
     v[i] = (l != l) ? -INFINITY : l;
   }
   uint32_t taken = 0;
@@ -194,19 +266,37 @@ __global__ void topk_softmax_kernel(const float* __restrict__ logits, int T, int
   }
 }
 
+// 0: warp-per-dot-product router; otherwise the GEMM with this many K parts
+// (enough tiles for two per SM on 148 SMs, parts of at least 512 inputs).
+int router_parts(long long T, int H, int E) {
+  if (T <= 64 || E <= 32) return 0;
+  const long long tiles = ((T + kRT - 1) / kRT) * ((E + kRE - 1) / kRE);
+  long long p = (2 * 148 + tiles - 1) / tiles;
+  const long long pmax = H / 512 > 1 ? H / 512 : 1;
+  if (p > pmax) p = pmax;
+  if (p > 8) p = 8;
+  return p < 1 ? 1 : (int)p;
+}
+
 cudaError_t launch_router_topk(const __nv_bfloat16* x, const float* Wr, const float* b, int T, int H,
                                int E, int k, const Workspace& ws, int32_t* dbg_idx, float* dbg_w,
                                cudaStream_t stream) {
-  if (T <= 64 || E <= 32) {  // one warp per dot product: plenty of parallelism when E is small
+  const int parts = router_parts(T, H, E);
+  if (parts == 0) {  // one warp per dot product: plenty of parallelism when E is small
     dim3 grid(T, (E + 7) / 8);
     router_warp_kernel<<<grid, 256, 0, stream>>>(x, Wr, b, T, H, E, ws.logits);
   } else {
-    dim3 grid((T + 63) / 64, (E + 63) / 64);
-    router_tile_kernel<64><<<grid, 256, 0, stream>>>(x, Wr, b, T, H, E, ws.logits);
+    const long long n = (long long)E * H;
+    router_split_kernel<<<(int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0, stream>>>(Wr, n, ws.wsplit);
+    cudaError_t aerr = cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRSmem);
+    if (aerr != cudaSuccess) return aerr;
+    dim3 grid((T + kRT - 1) / kRT, (E + kRE - 1) / kRE, parts);
+    router_mma_kernel<<<grid, 256, kRSmem, stream>>>(x, ws.wsplit, b, T, H, E, ws.logits);
   }
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  topk_softmax_kernel<<<(T + 7) / 8, 256, 0, stream>>>(ws.logits, T, E, k, ws.idx, ws.wts, dbg_idx, dbg_w);
+  topk_softmax_kernel<<<(T + 7) / 8, 256, 0, stream>>>(ws.logits, parts > 1 ? parts : 1, T, E, k, ws.idx, ws.wts,
+                                                        dbg_idx, dbg_w);
   return cudaGetLastError();
 }
 
