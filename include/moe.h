@@ -194,7 +194,10 @@ typedef struct {
  *   size needed for (T, k, weights) and nothing runs.
  * Steps (all on `stream`):
  *   1. logits[t][e] = sum_h x[t][h]*Wr[e][h] (+ b[e]) accumulated in fp32
- *      (the router stays unquantized: MoE mixed-precision page sec. 2.1);
+ *      (the router stays unquantized: MoE mixed-precision page sec. 2.1); for
+ *      many tokens each fp32 weight is split exactly into three bf16 terms so
+ *      the tensor cores form exact products, summed in fp32 chunks of 64
+ *      inputs with Kahan-compensated chunk sums;
  *   2. top-k (ties to the lower expert index; NaN ranks lowest), then
  *      w = softmax over the k chosen logits (expert-routing section of the
  *      quantized-MoE-inference page);
