@@ -478,9 +478,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const float sx = a.row_scale[a.perm[r] / a.topk];
               g *= sx * tsc[0];
               u *= sx * tsc[1];
-              reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = g / (1.0f + __expf(-g)) * u;
+              reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = __fdividef(g, 1.0f + __expf(-g)) * u;
             } else {
-              reinterpret_cast<__half*>(a.out)[(size_t)r * a.N + nrow] = __float2half_rn(g / (1.0f + __expf(-g)) * u);
+              reinterpret_cast<__half*>(a.out)[(size_t)r * a.N + nrow] = __float2half_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
             }
           } else {
             float o = __uint_as_float(r0[j]);

@@ -393,11 +393,11 @@ __device__ __forceinline__ float store_output(const GemvArgs& a, int r, int n, c
       const float sx = a.row_scale[a.perm[r] / a.topk];
       gv *= sx * ts[0];
       uv *= sx * ts[1];
-      const float h = gv / (1.0f + __expf(-gv)) * uv;
+      const float h = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
       reinterpret_cast<float*>(a.out)[(size_t)r * a.N + n] = h;
       return h;
     }
-    const __half h = __float2half_rn(gv / (1.0f + __expf(-gv)) * uv);
+    const __half h = __float2half_rn(__fdividef(gv, 1.0f + __expf(-gv)) * uv);
     reinterpret_cast<__half*>(a.out)[(size_t)r * a.N + n] = h;
     return __half2float(h);
   }

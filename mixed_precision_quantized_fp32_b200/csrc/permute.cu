@@ -144,85 +144,98 @@ __global__ void gather_f16_kernel(const __nv_bfloat16* __restrict__ x, const int
   }
 }
 
-__device__ __forceinline__ float block_max(float v, float* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    v = (lane < (int)(blockDim.x >> 5)) ? red[lane] : 0.0f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if (lane == 0) red[0] = v;
-  }
-  __syncthreads();
-  v = red[0];
-  __syncthreads();
-  return v;
-}
-
-// Per-token e4m3 codes of x: s = amax/448 (1 if amax == 0); q = e4m3(x/s), RNE, saturating.
-__global__ void act_quant_x_kernel(const __nv_bfloat16* __restrict__ x, int H, uint8_t* __restrict__ xq,
+// Per-token e4m3 codes of x: s = amax/448 (1 if amax == 0); q = e4m3(x/s), RNE,
+// saturating.  One warp per token; H is a multiple of 128.
+__global__ void act_quant_x_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, uint8_t* __restrict__ xq,
                                    float* __restrict__ sx, uint8_t* __restrict__ dbg_xq,
                                    float* __restrict__ dbg_sx) {
-  __shared__ float red[32];
-  const int t = blockIdx.x;
-  const __nv_bfloat16* xr = x + (size_t)t * H;
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const uint2* xr = reinterpret_cast<const uint2*>(x + (size_t)t * H);  // 4 bf16 per load
   float m = 0.0f;
-  for (int h = threadIdx.x; h < H; h += blockDim.x) m = fmaxf(m, fabsf(__bfloat162float(xr[h])));
-  const float amax = block_max(m, red);
-  const float s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-  for (int h = threadIdx.x; h < H; h += blockDim.x) {
-    const uint8_t c = __nv_cvt_float_to_fp8(__fdiv_rn(__bfloat162float(xr[h]), s), __NV_SATFINITE, __NV_E4M3);
-    xq[(size_t)t * H + h] = c;
-    if (dbg_xq) dbg_xq[(size_t)t * H + h] = c;
+  for (int c = lane; c < H / 4; c += 32) {
+    const uint2 v = __ldg(xr + c);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v.x), b = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(__low2float(a)), fabsf(__high2float(a))), fmaxf(fabsf(__low2float(b)), fabsf(__high2float(b)))));
   }
-  if (threadIdx.x == 0) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const float s = (m == 0.0f) ? 1.0f : __fdiv_rn(m, 448.0f);
+  for (int c = lane; c < H / 4; c += 32) {
+    const uint2 v = __ldg(xr + c);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v.x), b = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+    const float f[4] = {__low2float(a), __high2float(a), __low2float(b), __high2float(b)};
+    uint32_t q = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      q |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(f[i], s), __NV_SATFINITE, __NV_E4M3) << (8 * i);
+    reinterpret_cast<uint32_t*>(xq + (size_t)t * H)[c] = q;
+    if (dbg_xq) reinterpret_cast<uint32_t*>(dbg_xq + (size_t)t * H)[c] = q;
+  }
+  if (lane == 0) {
     sx[t] = s;
     if (dbg_sx) dbg_sx[t] = s;
   }
 }
 
-// Gather e4m3 activation codes into sorted rows as exact fp16 values.
+// Gather e4m3 activation codes into sorted rows as exact fp16 values: one
+// thread per 16 codes (hardware e4m3x2 -> f16x2 conversion).
 __global__ void gather_fp8_kernel(const uint8_t* __restrict__ xq, const int32_t* __restrict__ perm, int R,
                                   int H, int k, __half* __restrict__ xs, int32_t* counters, int n_counters) {
   zero_counters(counters, n_counters);
-  const int r = blockIdx.x;
+  const int per_row = H / 16;
+  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (i >= (long long)R * per_row) return;
+  const int r = (int)(i / per_row), c = (int)(i % per_row);
   const int t = perm[r] / k;
-  const uint2* src = reinterpret_cast<const uint2*>(xq + (size_t)t * H);
-  uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)r * H);
-  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
-    const uint2 v = __ldg(src + c);
-    uint4 o;
-    __half* ob = reinterpret_cast<__half*>(&o);
+  const uint4 v = __ldg(reinterpret_cast<const uint4*>(xq + (size_t)t * H) + c);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      ob[i] = __float2half_rn(e4m3_value((v.x >> (8 * i)) & 255u));
-      ob[4 + i] = __float2half_rn(e4m3_value((v.y >> (8 * i)) & 255u));
-    }
-    dst[c] = o;
+  for (int j = 0; j < 4; ++j) {
+    const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[j] & 0xFFFFu), __NV_E4M3);
+    const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[j] >> 16), __NV_E4M3);
+    o[2 * j] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
+    o[2 * j + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
   }
+  uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)r * H) + 2 * c;
+  dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+  dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// Per-row e4m3 codes of the SwiGLU output (NVFP4 layers) and their exact fp16 values.
-__global__ void act_quant_h_kernel(const float* __restrict__ h, int F, uint8_t* __restrict__ hq,
+// Per-row e4m3 codes of the SwiGLU output (NVFP4 layers) and their exact fp16
+// values.  One warp per row; F is a multiple of 128.
+__global__ void act_quant_h_kernel(const float* __restrict__ h, int R, int F, uint8_t* __restrict__ hq,
                                    float* __restrict__ sh, __half* __restrict__ hb,
                                    uint8_t* __restrict__ dbg_hq, float* __restrict__ dbg_sh) {
-  __shared__ float red[32];
-  const int r = blockIdx.x;
-  const float* hr = h + (size_t)r * F;
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= R) return;
+  const float4* hr = reinterpret_cast<const float4*>(h + (size_t)r * F);
   float m = 0.0f;
-  for (int i = threadIdx.x; i < F; i += blockDim.x) m = fmaxf(m, fabsf(hr[i]));
-  const float amax = block_max(m, red);
-  const float s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-  for (int i = threadIdx.x; i < F; i += blockDim.x) {
-    const uint8_t c = __nv_cvt_float_to_fp8(__fdiv_rn(hr[i], s), __NV_SATFINITE, __NV_E4M3);
-    hq[(size_t)r * F + i] = c;
-    hb[(size_t)r * F + i] = __float2half_rn(e4m3_value(c));
-    if (dbg_hq) dbg_hq[(size_t)r * F + i] = c;
+  for (int c = lane; c < F / 4; c += 32) {
+    const float4 v = __ldg(hr + c);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
   }
-  if (threadIdx.x == 0) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const float s = (m == 0.0f) ? 1.0f : __fdiv_rn(m, 448.0f);
+  for (int c = lane; c < F / 4; c += 32) {
+    const float4 v = __ldg(hr + c);
+    const float f[4] = {v.x, v.y, v.z, v.w};
+    uint32_t q = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      q |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(f[i], s), __NV_SATFINITE, __NV_E4M3) << (8 * i);
+    reinterpret_cast<uint32_t*>(hq + (size_t)r * F)[c] = q;
+    if (dbg_hq) reinterpret_cast<uint32_t*>(dbg_hq + (size_t)r * F)[c] = q;
+    const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(q & 0xFFFFu), __NV_E4M3);
+    const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(q >> 16), __NV_E4M3);
+    reinterpret_cast<uint2*>(hb + (size_t)r * F)[c] =
+        make_uint2((uint32_t)lo.x | ((uint32_t)lo.y << 16), (uint32_t)hi.x | ((uint32_t)hi.y << 16));
+  }
+  if (lane == 0) {
     sh[r] = s;
     if (dbg_sh) dbg_sh[r] = s;
   }
@@ -244,9 +257,10 @@ cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4,
                           uint8_t* dbg_xq, float* dbg_sx, cudaStream_t stream) {
   const int R = T * k;
   if (fp4) {
-    act_quant_x_kernel<<<T, 256, 0, stream>>>(x, H, ws.xq, ws.sx, dbg_xq, dbg_sx);
-    gather_fp8_kernel<<<R, 128, 0, stream>>>(ws.xq, ws.perm, R, H, k, (__half*)ws.xs, ws.counters,
-                                             ws.counter_len);
+    act_quant_x_kernel<<<(T + 7) / 8, 256, 0, stream>>>(x, T, H, ws.xq, ws.sx, dbg_xq, dbg_sx);
+    const long long n = (long long)R * (H / 16);
+    gather_fp8_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(ws.xq, ws.perm, R, H, k, (__half*)ws.xs,
+                                                                     ws.counters, ws.counter_len);
   } else {
     gather_f16_kernel<<<R, 128, 0, stream>>>(x, ws.perm, R, H, k, (__half*)ws.xs, ws.xsum, ws.counters,
                                              ws.counter_len);
@@ -256,8 +270,8 @@ cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4,
 
 cudaError_t launch_act_quant_h(int R, int F, const Workspace& ws, uint8_t* dbg_hq, float* dbg_sh,
                                cudaStream_t stream) {
-  act_quant_h_kernel<<<R, 256, 0, stream>>>((const float*)ws.h, F, ws.hq, ws.sh, (__half*)ws.hb,
-                                            dbg_hq, dbg_sh);
+  act_quant_h_kernel<<<(R + 7) / 8, 256, 0, stream>>>((const float*)ws.h, R, F, ws.hq, ws.sh, (__half*)ws.hb,
+                                                      dbg_hq, dbg_sh);
   return cudaGetLastError();
 }
 
