@@ -408,7 +408,7 @@ __device__ __forceinline__ float store_output(const GemvArgs& a, int r, int n, c
 }
 
 template <int NMAT, int NT8>
-__global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? 3 : 2) expert_gemv_kernel(const __grid_constant__ CUtensorMap tm_w2,
+__global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) : 2) expert_gemv_kernel(const __grid_constant__ CUtensorMap tm_w2,
                                                                    const __grid_constant__ CUtensorMap tm_w3,
                                                                    const __grid_constant__ CUtensorMap tm_w4,
                                                                    const __grid_constant__ CUtensorMap tm_x,
@@ -701,8 +701,9 @@ bool encode_rows_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt,
 }
 
 // Stage layout for the widest formats of the layer at each matrix position.
-// Shared memory is budgeted for three CTAs per SM with one token tile and two
-// with two (whose registers allow no more).
+// Shared memory is budgeted for the CTAs per SM that the registers allow: four
+// (one matrix, one token tile), three (two matrices, one token tile) or two
+// (two token tiles).
 StageLayout stage_layout(int nmat, int nt8, const int* wmax) {
   StageLayout L{};
   int off = 0;
@@ -720,7 +721,7 @@ StageLayout stage_layout(int nmat, int nt8, const int* wmax) {
   L.sum_off = off;
   off += nt8 * 8 * 16;
   L.bytes = (off + 1023) / 1024 * 1024;
-  const int cta_per_sm = nt8 == 1 ? 3 : 2;
+  const int cta_per_sm = nt8 == 1 ? (nmat == 1 ? 4 : 3) : 2;
   const int budget = 227 * 1024 / cta_per_sm - 1024 - kCtrlBytes - 1024;  // minus alignment, control, per-CTA reserve
   L.stages = budget / L.bytes;
   if (L.stages > kMaxStages) L.stages = kMaxStages;
