@@ -97,6 +97,35 @@ def job_tokens_per_s(tokens_per_rank: int, steps: int, world: int, max_ms: float
     return world * tokens_per_rank * steps / (max_ms / 1e3)
 
 
+# ------------------------------------------------------------------ CUDA-graph replay
+def graph_step_ms(forward, flush, n: int) -> float:
+    """Median device time of one forward replayed from a CUDA graph (no host launch
+    cost), with L2 flushed before each replay (outside the timed interval)."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        forward()  # first call outside the capture (sets kernel attributes)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        forward()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(n + 2):
+        if flush is not None:
+            flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    del g
+    return float(np.median(ts[2:]))
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     def __init__(self, device_index: int):
@@ -283,8 +312,11 @@ def run_ours(args, rank, world, local_rank):
             stp = np.array([evd[s][0].elapsed_time(evd[s][-1]) for s in range(nd)])
             gu = float(st[:, 3].mean())
             by = float(eb[active].sum())
+            yd = torch.empty_like(xd)
+            gms = graph_step_ms(lambda: moe.moe_layer_forward(xd, Wr, b, layer, L.k, y=yd, ws=wsd), flush, nd)
             runs.append({"workload": workload_desc(L, Td, "decode"), "tokens_per_s": round(Td / (stp.mean() / 1e3), 1),
                          "ms_per_step": round(float(stp.mean()), 4),
+                         "graph_tokens_per_s": round(Td / (gms / 1e3), 1), "graph_ms_per_step": round(gms, 4),
                          "active_experts": int(active.sum()),
                          "gateup": {"bound": "hbm", "achieved": round(by / (gu / 1e3) / 1e9, 1),
                                     "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -363,6 +395,10 @@ def run_suite(args):
                    "stages_ms": dict(zip(["router_topk", "permute", "gather", "gateup", "h_quant", "down", "combine"],
                                          [round(float(v), 4) for v in st]))}
             if decode:
+                yg = torch.empty_like(x)
+                gms = graph_step_ms(lambda: moe.moe_layer_forward(x, Wr, b, layer, L.k, y=yg, ws=ws), flush, n)
+                out["graph_tokens_per_s"] = round(T / gms * 1e3, 1)
+                out["graph_ms_per_step"] = round(gms, 4)
                 bg = sum(matrix_bytes(L, int(e), 0) + matrix_bytes(L, int(e), 1) for e in active)
                 bd = sum(matrix_bytes(L, int(e), 2) for e in active)
                 out["gateup"] = {"GB/s": round(bg / gu / 1e6, 1), "frac_hbm": round(bg / gu / 1e6 / pk["hbm_gbs"], 4)}

@@ -287,6 +287,32 @@ def test_forward_deterministic_and_empty_batch():
     assert y0.shape == (0, L.H)
 
 
+@pytest.mark.parametrize("name,T", [("mixtral", 1), ("mixtral", 8), ("tiny", 512)])
+def test_forward_replays_from_cuda_graph(name, T):
+    """The forward captures into a CUDA graph (no host sync or allocation inside)
+    and every replay gives the eager result bit for bit: split-K decode (Mixtral
+    T=1, 8) and the tcgen05 path (T=512 of the small layer)."""
+    L = W.layer(name)
+    layer = hp.gpu_pack_cached(L) if name != "tiny" else hp.gpu_pack(L)
+    x = W.device_x(T, L.H)
+    Wr, b = W.device_router(L)
+    ws = moe.alloc_packed(moe.workspace_bytes(layer, T, L.k))
+    y_eager = moe.moe_layer_forward(x, Wr, b, layer, L.k, ws=ws).clone()
+    y = torch.empty_like(x)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        moe.moe_layer_forward(x, Wr, b, layer, L.k, y=y, ws=ws)
+    for _ in range(3):
+        y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y_eager.view(torch.int16))
+    del g
+
+
 def test_stage_events_record():
     L = W.layer("tiny")
     layer = hp.gpu_pack(L)
