@@ -48,8 +48,9 @@ struct Plan {
   bool tc;         // tcgen05 expert GEMMs (many rows per expert) or warp-MMA (few rows per expert)
 };
 
-// Few rows per expert (decode): chunks of 8 or 16 rows (by the average rows per
-// active expert) on the streaming GEMV (warp MMA).  Many rows per expert
+// Few rows per expert (decode): chunks of 8 rows on the streaming GEMV (warp
+// MMA); an expert with more rows gets several chunks, which read the same weight
+// tiles close in time (the second read hits L2).  Many rows per expert
 // (prefill): 256-row chunks on the tcgen05 kernel.
 Plan make_plan(int T, int k, int E) {
   Plan p;
@@ -57,7 +58,7 @@ Plan make_plan(int T, int k, int E) {
   const long long active = R < E ? R : E;
   const long long avg = active > 0 ? (R + active - 1) / active : 0;
   p.tc = avg > 32 && R >= 256;
-  p.chunk_rows = p.tc ? 256 : (avg <= 3 ? 8 : 16);
+  p.chunk_rows = p.tc ? 256 : 8;
   p.max_chunks = (int)(E + (R + p.chunk_rows - 1) / p.chunk_rows);
   return p;
 }

@@ -1,5 +1,5 @@
 // Dequant-fused grouped expert GEMV for batches with few token rows per expert
-// (decode: up to 16 rows per chunk), bound by streaming the active experts'
+// (decode: chunks of up to 8 rows), bound by streaming the active experts'
 // packed weights from HBM.  It follows the pages' observation that a token only
 // needs its active experts' weights, and implements the packed-linear operator
 // of the MoE mixed-precision page (sec. 2.3 / 3.5).
@@ -824,14 +824,9 @@ cudaError_t launch_expert_gemv(const uint8_t* packed, uint64_t packed_bytes, con
   }
   const int nmat = gateup ? 2 : 1;
   g.P = gemv_split(R, E, g.N, g.K, nmat);
-  const bool two = chunk_rows > 8;
-  cudaError_t err;
-  if (gateup)
-    err = two ? launch_n<2, 2>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream)
-              : launch_n<2, 1>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream);
-  else
-    err = two ? launch_n<1, 2>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream)
-              : launch_n<1, 1>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream);
+  if (chunk_rows != 8) return cudaErrorInvalidValue;  // the host plans 8-row chunks (one token tile)
+  cudaError_t err = gateup ? launch_n<2, 1>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream)
+                           : launch_n<1, 1>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream);
   if (err != cudaSuccess || g.P == 1) return err;
   if (gateup)
     gemv_fixup_kernel<2><<<dim3(R, (g.N + 255) / 256), 256, 0, stream>>>(g, ws.idx);
