@@ -246,25 +246,52 @@ def run_ours(args, rank, world, local_rank):
     total_ms = max_over_ranks(float(sum(step_ms)), world, dev)
     value = job_tokens_per_s(T, args.steps, world, total_ms)
 
-    # ---- end to end through the public API with host buffers (pinned)
-    x_host = x.cpu().pin_memory()
-    y_host = torch.empty_like(x_host).pin_memory()
-    x_dev = torch.empty_like(x)
-    for _ in range(args.warmup):
-        x_dev.copy_(x_host, non_blocking=True)
-        forward(xx=x_dev)
-        y_host.copy_(y, non_blocking=True)
+    # ---- end to end through the public API with host buffers (pinned).  Every step
+    # copies its own input in and its result out; copy streams (one per direction)
+    # overlap step i+1's input copy and step i's output copy with compute, through
+    # two device buffers (the usual double-buffered serving loop).
+    x_host = [x.cpu().pin_memory(), x.cpu().pin_memory()]
+    y_host = [torch.empty_like(x_host[0]).pin_memory(), torch.empty_like(x_host[0]).pin_memory()]
+    x_dev = [torch.empty_like(x), torch.empty_like(x)]
+    y_dev = [torch.empty_like(x), torch.empty_like(x)]
+    h2d, d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+
+    def e2e_steps(n):
+        done = [None, None]   # compute of the step that last used buffer i
+        out_done = [None, None]  # output copy of that step
+        for i in range(n):
+            j = i % 2
+            with torch.cuda.stream(h2d):
+                if done[j] is not None:
+                    h2d.wait_event(done[j])  # buffer j's previous step has finished reading x
+                x_dev[j].copy_(x_host[j], non_blocking=True)
+                x_in = torch.cuda.Event()
+                x_in.record(h2d)
+            stream.wait_event(x_in)
+            if out_done[j] is not None:
+                stream.wait_event(out_done[j])  # y_dev[j] was copied out before it is overwritten
+            forward(xx=x_dev[j], yy=y_dev[j])
+            done[j] = torch.cuda.Event()
+            done[j].record(stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(done[j])
+                y_host[j].copy_(y_dev[j], non_blocking=True)
+                out_done[j] = torch.cuda.Event()
+                out_done[j].record(d2h)
+        for ev in out_done:
+            if ev is not None:
+                stream.wait_event(ev)
+
+    e2e_steps(args.warmup)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        forward(xx=x_dev)
-        y_host.copy_(y, non_blocking=True)
-    e1.record(stream)
+    e2e_steps(args.steps)
+    e1.record(stream)  # after the last output copy (the compute stream waited for it)
     torch.cuda.synchronize()
+    assert torch.equal(y_host[(args.steps - 1) % 2].view(torch.int16), y.cpu().view(torch.int16))
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = job_tokens_per_s(T, args.steps, world, e2e_ms)
 
@@ -335,7 +362,9 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "inputs larger than L2 (617 MB packed weights streamed per step)"},
         "roofline": roofline,
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2)},
+                "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2),
+                "overlap": "double-buffered: copy streams move step i+1's input and step i-1's output while "
+                           "step i computes"},
         "gpu_launches": KERNELS_PER_FORWARD_INT * args.steps,
         "clocks": clk, "stages_ms": stages, "runs": runs,
     }
