@@ -16,7 +16,7 @@ __global__ void combine_kernel(const float* __restrict__ o, const float* __restr
     rows[j] = inv[t * k + j];
     w[j] = wts[t * k + j];
   }
-  for (int c = threadIdx.x; c < H / 4; c += blockDim.x) {
+  for (int c = blockIdx.y * blockDim.x + threadIdx.x; c < H / 4; c += gridDim.y * blockDim.x) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
       const float4 v = __ldg(reinterpret_cast<const float4*>(o + (size_t)rows[j] * H) + c);
@@ -35,7 +35,8 @@ __global__ void combine_kernel(const float* __restrict__ o, const float* __restr
 }
 
 cudaError_t launch_combine(int T, int k, int H, const Workspace& ws, __nv_bfloat16* y, cudaStream_t stream) {
-  combine_kernel<<<T, 256, 0, stream>>>(ws.o, ws.wts, ws.inv, k, H, y);
+  const int ny = (H / 4 + 255) / 256 < 8 ? (H / 4 + 255) / 256 : 8;  // column blocks: more parallelism for few tokens
+  combine_kernel<<<dim3(T, ny), 256, 0, stream>>>(ws.o, ws.wts, ws.inv, k, H, y);
   return cudaGetLastError();
 }
 

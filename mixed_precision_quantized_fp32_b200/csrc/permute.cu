@@ -108,9 +108,76 @@ __global__ void __launch_bounds__(kPermBlock) perm_scatter_kernel(const int32_t*
   if (dbg_inv) dbg_inv[i] = row;
 }
 
-// Zero the decode GEMV's work counters (the workspace starts undefined).
+// All of the permutation in one block when T*k <= 1024 (decode batches): the
+// histogram and stable ranks of pass 1, the scan and chunk list of pass 2 and
+// the scatter of pass 3, with the same results.
+__global__ void __launch_bounds__(kPermBlock) perm_small_kernel(const int32_t* __restrict__ idx, int R, int E,
+                                                                int chunk_rows, int32_t* __restrict__ counts,
+                                                                int32_t* __restrict__ offsets,
+                                                                int32_t* __restrict__ chunks,
+                                                                int32_t* __restrict__ chunk_count,
+                                                                int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                                int32_t* __restrict__ dbg_counts,
+                                                                int32_t* __restrict__ dbg_perm,
+                                                                int32_t* __restrict__ dbg_inv) {
+  __shared__ int32_t wcnt[kPermBlock / 32][kMaxE];
+  __shared__ int32_t s_off[kMaxE + 1], s_cstart[kMaxE + 1], s_cnt[kMaxE];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < (kPermBlock / 32) * kMaxE; i += kPermBlock) (&wcnt[0][0])[i] = 0;
+  __syncthreads();
+  const bool valid = tid < R;
+  const int e = valid ? idx[tid] : -1;
+  const unsigned same = __match_any_sync(0xffffffffu, e);
+  const int rw = __popc(same & ((1u << lane) - 1u));
+  if (valid && rw == 0) wcnt[warp][e] = __popc(same);
+  __syncthreads();
+  int rank = rw;
+  if (valid)
+    for (int w = 0; w < warp; ++w) rank += wcnt[w][e];
+  for (int ee = tid; ee < E; ee += kPermBlock) {
+    int total = 0;
+    for (int w = 0; w < kPermBlock / 32; ++w) total += wcnt[w][ee];
+    s_cnt[ee] = total;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0, crun = 0;
+    for (int j = 0; j < E; ++j) {
+      s_off[j] = run;
+      run += s_cnt[j];
+      s_cstart[j] = crun;
+      crun += (s_cnt[j] + chunk_rows - 1) / chunk_rows;
+    }
+    s_off[E] = run;
+    *chunk_count = crun;
+    offsets[E] = run;
+  }
+  __syncthreads();
+  for (int ee = tid; ee < E; ee += kPermBlock) {
+    const int total = s_cnt[ee];
+    counts[ee] = total;
+    offsets[ee] = s_off[ee];
+    if (dbg_counts) dbg_counts[ee] = total;
+    for (int c = 0; c * chunk_rows < total; ++c) {
+      int32_t* ch = chunks + 3 * (size_t)(s_cstart[ee] + c);
+      ch[0] = ee;
+      ch[1] = s_off[ee] + c * chunk_rows;
+      ch[2] = min(chunk_rows, total - c * chunk_rows);
+    }
+  }
+  if (valid) {
+    const int row = s_off[e] + rank;
+    perm[row] = tid;
+    inv[tid] = row;
+    if (dbg_perm) dbg_perm[row] = tid;
+    if (dbg_inv) dbg_inv[tid] = row;
+  }
+}
+
+// Zero the decode GEMV's work counters (the workspace starts undefined); called
+// by one block.
 __device__ __forceinline__ void zero_counters(int32_t* counters, int n) {
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) counters[i] = 0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) counters[i] = 0;
 }
 
 // Gather x rows into expert-sorted order as fp16 (integer-format layers), with
@@ -120,12 +187,12 @@ __device__ __forceinline__ void zero_counters(int32_t* counters, int n) {
 __global__ void gather_f16_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm,
                                   int R, int H, int k, __half* __restrict__ xs, float* __restrict__ xsum,
                                   int32_t* counters, int n_counters) {
-  zero_counters(counters, n_counters);
+  if (blockIdx.x == 0 && blockIdx.y == 0) zero_counters(counters, n_counters);
   const int r = blockIdx.x;
   const int t = perm[r] / k;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
   uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)r * H);
-  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
+  for (int c = blockIdx.y * blockDim.x + threadIdx.x; c < H / 8; c += gridDim.y * blockDim.x) {
     const uint4 v = __ldg(src + c);
     const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v);
     uint4 o;
@@ -138,8 +205,9 @@ __global__ void gather_f16_kernel(const __nv_bfloat16* __restrict__ x, const int
       sum += f.x + f.y;
     }
     dst[c] = o;
-    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+    const unsigned act = __activemask();  // whole groups of four lanes (H/8 is a multiple of 16)
+    sum += __shfl_xor_sync(act, sum, 1);
+    sum += __shfl_xor_sync(act, sum, 2);
     if (xsum && (c & 3) == 0) xsum[(size_t)r * (H / 32) + c / 4] = sum;
   }
 }
@@ -183,7 +251,7 @@ __global__ void act_quant_x_kernel(const __nv_bfloat16* __restrict__ x, int T, i
 // thread per 16 codes (hardware e4m3x2 -> f16x2 conversion).
 __global__ void gather_fp8_kernel(const uint8_t* __restrict__ xq, const int32_t* __restrict__ perm, int R,
                                   int H, int k, __half* __restrict__ xs, int32_t* counters, int n_counters) {
-  zero_counters(counters, n_counters);
+  if (blockIdx.x == 0) zero_counters(counters, n_counters);
   const int per_row = H / 16;
   const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (i >= (long long)R * per_row) return;
@@ -245,6 +313,11 @@ cudaError_t launch_permute(int T, int k, int E, int chunk_rows, const Workspace&
                            int32_t* dbg_perm, int32_t* dbg_inv, cudaStream_t stream) {
   const int R = T * k;
   const int nblk = (R + kPermBlock - 1) / kPermBlock;
+  if (nblk == 1) {
+    perm_small_kernel<<<1, kPermBlock, 0, stream>>>(ws.idx, R, E, chunk_rows, ws.counts, ws.offsets, ws.chunks,
+                                                    ws.chunk_count, ws.perm, ws.inv, dbg_counts, dbg_perm, dbg_inv);
+    return cudaGetLastError();
+  }
   perm_count_kernel<<<nblk, kPermBlock, 0, stream>>>(ws.idx, R, E, ws.blk_hist, ws.rank);
   perm_scan_kernel<<<1, 256, 0, stream>>>(ws.blk_hist, nblk, E, R, chunk_rows, ws.counts, ws.offsets,
                                           ws.chunks, ws.chunk_count, dbg_counts);
@@ -262,8 +335,9 @@ cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4,
     gather_fp8_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(ws.xq, ws.perm, R, H, k, (__half*)ws.xs,
                                                                      ws.counters, ws.counter_len);
   } else {
-    gather_f16_kernel<<<R, 128, 0, stream>>>(x, ws.perm, R, H, k, (__half*)ws.xs, ws.xsum, ws.counters,
-                                             ws.counter_len);
+    const int ny = (H / 8 + 127) / 128 < 8 ? (H / 8 + 127) / 128 : 8;  // column blocks: more parallelism for few rows
+    gather_f16_kernel<<<dim3(R, ny), 128, 0, stream>>>(x, ws.perm, R, H, k, (__half*)ws.xs, ws.xsum, ws.counters,
+                                                       ws.counter_len);
   }
   return cudaGetLastError();
 }

@@ -37,6 +37,38 @@ __global__ void router_warp_kernel(const __nv_bfloat16* __restrict__ x, const fl
   if (lane == 0) logits[(size_t)t * E + e] = b ? acc + b[e] : acc;
 }
 
+// One block of 128 threads per (token, expert) dot product: each thread sums its
+// share of H (8-byte bf16 and 16-byte fp32 loads, several in flight), then the
+// block adds the 128 partial sums.  Used for decode-sized batches.
+__global__ void __launch_bounds__(128) router_dot_kernel(const __nv_bfloat16* __restrict__ x,
+                                                         const float* __restrict__ Wr, const float* __restrict__ b,
+                                                         int T, int H, int E, float* __restrict__ logits) {
+  __shared__ float red[4];
+  const int t = blockIdx.x, e = blockIdx.y;
+  const __nv_bfloat16* xr = x + (size_t)t * H;
+  const float* wr = Wr + (size_t)e * H;
+  float acc = 0.0f;
+#pragma unroll 4
+  for (int h = threadIdx.x * 4; h < H; h += 512) {
+    const uint2 xv = __ldg(reinterpret_cast<const uint2*>(xr + h));
+    const float4 wv = __ldg(reinterpret_cast<const float4*>(wr + h));
+    const __nv_bfloat162 x01 = *reinterpret_cast<const __nv_bfloat162*>(&xv.x);
+    const __nv_bfloat162 x23 = *reinterpret_cast<const __nv_bfloat162*>(&xv.y);
+    acc = fmaf(__low2float(x01), wv.x, acc);
+    acc = fmaf(__high2float(x01), wv.y, acc);
+    acc = fmaf(__low2float(x23), wv.z, acc);
+    acc = fmaf(__high2float(x23), wv.w, acc);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const float v = (red[0] + red[1]) + (red[2] + red[3]);
+    logits[(size_t)t * E + e] = b ? v + b[e] : v;
+  }
+}
+
 // ---------------------------------------------------------------- router, many tokens
 // The fp32 router weights are split exactly into three bf16 terms
 // (w = hi + mid + lo up to the last bit of lo), so with bf16 x every product
@@ -282,7 +314,9 @@ cudaError_t launch_router_topk(const __nv_bfloat16* x, const float* Wr, const fl
                                int E, int k, const Workspace& ws, int32_t* dbg_idx, float* dbg_w,
                                cudaStream_t stream) {
   const int parts = router_parts(T, H, E);
-  if (parts == 0) {  // one warp per dot product: plenty of parallelism when E is small
+  if (parts == 0 && T <= 64) {  // decode: one block per dot product
+    router_dot_kernel<<<dim3(T, E), 128, 0, stream>>>(x, Wr, b, T, H, E, ws.logits);
+  } else if (parts == 0) {  // many tokens, few experts: one warp per dot product
     dim3 grid(T, (E + 7) / 8);
     router_warp_kernel<<<grid, 256, 0, stream>>>(x, Wr, b, T, H, E, ws.logits);
   } else {
