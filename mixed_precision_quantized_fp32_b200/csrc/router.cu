@@ -314,7 +314,7 @@ cudaError_t launch_router_topk(const __nv_bfloat16* x, const float* Wr, const fl
                                int E, int k, const Workspace& ws, int32_t* dbg_idx, float* dbg_w,
                                cudaStream_t stream) {
   const int parts = router_parts(T, H, E);
-  if (parts == 0 && T <= 64) {  // decode: one block per dot product
+  if (parts == 0 && T <= 64 && E <= 32) {  // decode, few experts: one block per dot product
     router_dot_kernel<<<dim3(T, E), 128, 0, stream>>>(x, Wr, b, T, H, E, ws.logits);
   } else if (parts == 0) {  // many tokens, few experts: one warp per dot product
     dim3 grid(T, (E + 7) / 8);
