@@ -21,6 +21,7 @@
 // Every mbarrier wait is bounded; a wait that gives up raises an abort flag so
 // every role leaves its loop, writes MOE_ERR_TIMEOUT to the status word and
 // the CTA frees its TMEM before returning.
+#include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
 #include "moe_common.cuh"
@@ -116,8 +117,8 @@ __device__ __forceinline__ uint4 dequant_chunk(const uint32_t* __restrict__ code
                                               int n, int c) {
   uint32_t v[4];
   if (FMT == MOE_FMT_NVFP4) {
-    const __half2 s2 = __float2half2_rn(e4m3_value(scales[(c >> 1) * 128 + n]));
-    const uint32_t p = *reinterpret_cast<const uint32_t*>(&s2);
+    const __half_raw sr = __nv_cvt_fp8_to_halfraw(scales[(c >> 1) * 128 + n], __NV_E4M3);  // exact
+    const uint32_t p = (uint32_t)sr.x | ((uint32_t)sr.x << 16);
     e2m1x8_to_f16(codes[c * 128 + n], v);
 #pragma unroll
     for (int b = 0; b < 4; ++b) v[b] = h2mul(v[b], p);  // exact: <= 6 significant bits

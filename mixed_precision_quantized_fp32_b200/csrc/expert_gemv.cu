@@ -34,6 +34,7 @@
 // order and runs the epilogue.  There are no atomics or fences between CTAs and
 // results do not depend on timing.  Every mbarrier wait is bounded; a wait that
 // gives up sets MOE_ERR_TIMEOUT in the status word.
+#include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
 #include "moe_common.cuh"
@@ -176,13 +177,17 @@ __device__ __forceinline__ void group_mma(const uint8_t* box, const uint8_t* sc,
     const uint4 w = lds128(code_chunk(box, 4 * kg + c, y, g));
     const uint32_t bs = lds32(sc + (2 * kg + (c >> 1)) * 128 + 32 * s + 4 * g);  // e4m3 block scales of rows 4g..
     const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+    // e4m3 pairs -> f16 pairs (hardware conversion, exact), then each row's scale in both halves
+    const __half2_raw s01 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(bs & 0xFFFFu), __NV_E4M3);
+    const __half2_raw s23 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(bs >> 16), __NV_E4M3);
+    const uint32_t w01 = (uint32_t)s01.x | ((uint32_t)s01.y << 16), w23 = (uint32_t)s23.x | ((uint32_t)s23.y << 16);
+    const uint32_t sp[4] = {__byte_perm(w01, 0u, 0x1010u), __byte_perm(w01, 0u, 0x3232u), __byte_perm(w23, 0u, 0x1010u),
+                            __byte_perm(w23, 0u, 0x3232u)};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       e2m1x8_to_f16(wv[i], p[i]);
-      const __half2 s2 = __float2half2_rn(e4m3_value((bs >> (8 * i)) & 255u));
-      const uint32_t sp = *reinterpret_cast<const uint32_t*>(&s2);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) p[i][j] = hmul2(p[i][j], sp);  // exact: <= 6 significant bits
+      for (int j = 0; j < 4; ++j) p[i][j] = hmul2(p[i][j], sp[i]);  // exact: <= 6 significant bits
     }
 #pragma unroll
     for (int nt = 0; nt < NT8; ++nt) {
