@@ -113,7 +113,8 @@ enum {
  *   2-bit: codes 16w..16w+15 in word w; code 16w+2j at bits 2j..2j+1, code
  *          16w+2j+1 at bits 16+2j..17+2j (j = 0..7)
  *   3-bit: words 0-1 hold the low two bits of u as for 2-bit; word 2 holds
- *          bit 2 of u: code 2j at bit j, code 2j+1 at bit 16+j (j = 0..15)
+ *          bit 2 of u: of pair m = 4c+j (c, j = 0..3), code 2m at bit
+ *          P = 8*(c/2) + c%2 + 2j and code 2m+1 at bit 16+P
  *   NVFP4: codes 8w..8w+7 in word w, code 8w+i at bits 4i..4i+3.
  * Scale layout: [N/128][K/gs][128] (gs = 32 integer, 16 NVFP4).
  */

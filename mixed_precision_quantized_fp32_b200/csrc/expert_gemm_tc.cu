@@ -138,16 +138,21 @@ __device__ __forceinline__ uint4 dequant_chunk(const uint32_t* __restrict__ code
       v[3] = h2mul(h2fma((w8 & 0x00F000F0u) | kMagic, 0x2C002C00u, 0xD480D480u), s2);
     } else {
       // fields of pair j at bits 2j (weight 4^j); INT3 adds bit 2 of the pair's
-      // codes from word 2 (pair m at bits m, 16+m), moved to bit 2j+2
+      // codes from word 2 (pair m = 4c+j at bits 8*(c/2) + c%2 + 2j and 16 above),
+      // which one rotation moves to bit 2j+2
       constexpr uint32_t kMul[4] = {0x3C003C00u, 0x34003400u, 0x2C002C00u, 0x24002400u};        // 4^-j
       constexpr uint32_t kSub2[4] = {0xE402E402u, 0xDC08DC08u, 0xD420D420u, 0xCC80CC80u};       // -(1024/4^j + 2)
       constexpr uint32_t kSub3[4] = {0xE404E404u, 0xDC10DC10u, 0xD440D440u, 0xCD00CD00u};       // -(1024/4^j + 4)
       const uint32_t lo = codes[(c >> 1) * 128 + n] >> (8 * (c & 1));
-      const uint32_t hh = FMT == MOE_FMT_INT3 ? codes[2 * 128 + n] >> (4 * c) : 0u;
+      uint32_t hh = 0u;
+      if (FMT == MOE_FMT_INT3) {
+        const uint32_t hw = codes[2 * 128 + n];
+        hh = __funnelshift_r(hw, hw, (uint32_t)(8 * (c >> 1) + (c & 1) + 30) & 31u);
+      }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t raw = (lo & (0x00030003u << (2 * j))) | kMagic;
-        if (FMT == MOE_FMT_INT3) raw |= (hh << (j + 2)) & (0x00040004u << (2 * j));
+        if (FMT == MOE_FMT_INT3) raw |= hh & (0x00040004u << (2 * j));
         v[j] = h2mul(h2fma(raw, kMul[j], FMT == MOE_FMT_INT3 ? kSub3[j] : kSub2[j]), s2);
       }
     }

@@ -16,7 +16,7 @@
 //
 // Per group of 32 inputs, lane (g, c) holds word(s) of rows 4g..4g+3 covering
 // inputs 8c..8c+7.  It turns each pair of codes into one fp16x2 A-fragment
-// register with one AND (INT3: three ALU ops that merge the high-bit plane):
+// register with one AND (INT3: one more op per pair merges the high-bit plane):
 //   * the masked field is read as an fp16 subnormal: a code u in a field of
 //     power-of-two weight f (bit position 2j or 4j of a half-word) is exactly
 //     u * f * 2^-24;
@@ -226,19 +226,18 @@ __device__ __forceinline__ void group_mma(const uint8_t* box, const uint8_t* sc,
         for (int j = 0; j < 4; ++j) p[i][j] = ws & (0x00030003u << (2 * j));
       }
     } else {
-      // INT3: bit 2 of code 2m / 2m+1 sits at bit m / 16+m of word 2 (m = 0..15).
-      // The lane's pairs m = 4c+j rotate to bits j+2; shifted left by j they land
-      // on bit 2j+2, right above the pair's two low bits.
+      // INT3: bit 2 of pair m = 4c+j sits at bit 8*(c/2) + c%2 + 2j of word 2 (and
+      // 16 above for the odd code), so one rotation per row puts all four of the
+      // lane's high bits on bit 2j+2, right above each pair's two low bits.
       const uint4 hw = lds128(code_chunk(box, 3 * kg + 2, y, g));
       const uint32_t hv[4] = {hw.x, hw.y, hw.z, hw.w};
-      const uint32_t rot = (uint32_t)(4 * c + 30) & 31u;
+      const uint32_t rot = (uint32_t)(8 * (c >> 1) + (c & 1) + 30) & 31u;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint32_t ws = wv[i] >> sh;
         const uint32_t hh = __funnelshift_r(hv[i], hv[i], rot);
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          p[i][j] = (ws & (0x00030003u << (2 * j))) | ((hh << j) & (0x00040004u << (2 * j)));
+        for (int j = 0; j < 4; ++j) p[i][j] = (ws & (0x00030003u << (2 * j))) | (hh & (0x00040004u << (2 * j)));
       }
     }
   }

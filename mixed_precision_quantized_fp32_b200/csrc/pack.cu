@@ -123,10 +123,13 @@ __global__ void pack_int_kernel(const float* __restrict__ W, int N, int K, uint3
         v |= ((u[wd * 16 + 2 * j] & 3u) << (2 * j)) | ((u[wd * 16 + 2 * j + 1] & 3u) << (16 + 2 * j));
       codes[word_index(n, k0, K, BITS, wd)] = v;
     }
-    if (BITS == 3) {
+    if (BITS == 3) {  // bit 2 of pair m = 4c+j at bit 8*(c/2) + c%2 + 2j (low half: even code)
       uint32_t hi = 0;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) hi |= (((u[2 * j] >> 2) & 1u) << j) | (((u[2 * j + 1] >> 2) & 1u) << (16 + j));
+      for (int m = 0; m < 16; ++m) {
+        const int c = m >> 2, pos = 8 * (c >> 1) + (c & 1) + 2 * (m & 3);
+        hi |= (((u[2 * m] >> 2) & 1u) << pos) | (((u[2 * m + 1] >> 2) & 1u) << (16 + pos));
+      }
       codes[word_index(n, k0, K, 3, 2)] = hi;
     }
   }

@@ -237,7 +237,9 @@ ORC_EXPORT void orc_quant_nvfp4(const float* W, int N, int K, uint8_t* v, uint8_
 /*   b = 2: codes 16w..16w+15 in word w; code 16w+2j at bits 2j..2j+1, code  */
 /*          16w+2j+1 at bits 16+2j..17+2j (j = 0..7);                        */
 /*   b = 3: words 0-1 hold the low two bits of u exactly as b = 2; word 2     */
-/*          holds bit 2 of u: code 2j at bit j, code 2j+1 at bit 16+j.        */
+/*          holds bit 2 of u: of pair m = 4c+j (c, j = 0..3), code 2m at bit  */
+/*          P = 8*(c/2) + c%2 + 2j and code 2m+1 at bit 16+P, so the bits of  */
+/*          each run of four pairs sit at every other position.               */
 /*   NVFP4: codes 8w..8w+7 in word w, code 8w+i at bits 4i..4i+3.            */
 /* Scales: fp16 (int) or e4m3 bytes (NVFP4) in [N/128][K/gs][128] order,      */
 /* gs = 32 (int) or 16 (NVFP4).                                               */
@@ -254,6 +256,12 @@ static int pair_shift(int i, int width, int per_word) {
   return (c % 2) * 16 + (c / 2) * width;
 }
 
+/* bit of word 2 holding bit 2 of 3-bit code i (0..31 of its group) */
+static int int3_high_shift(int i) {
+  int m = i / 2, c = m / 4, j = m % 4;
+  return (i % 2) * 16 + 8 * (c / 2) + c % 2 + 2 * j;
+}
+
 /* code (already offset / e2m1, 0..15) of element (n, k) is placed into words */
 static void put_code(uint32_t* words, int n, int k, int K, int fmt, uint32_t u) {
   int i = k % 32;
@@ -265,7 +273,7 @@ static void put_code(uint32_t* words, int n, int k, int K, int fmt, uint32_t u) 
     words[word_index(n, k, K, 2, i / 16)] |= (u & 3u) << pair_shift(i, 2, 16);
   } else { /* INT3 */
     words[word_index(n, k, K, 3, i / 16)] |= (u & 3u) << pair_shift(i, 2, 16);
-    words[word_index(n, k, K, 3, 2)] |= ((u >> 2) & 1u) << pair_shift(i, 1, 32);
+    words[word_index(n, k, K, 3, 2)] |= ((u >> 2) & 1u) << int3_high_shift(i);
   }
 }
 
@@ -275,7 +283,7 @@ static uint32_t get_code(const uint32_t* words, int n, int k, int K, int fmt) {
   if (fmt == ORC_INT4) return (words[word_index(n, k, K, 4, i / 8)] >> pair_shift(i, 4, 8)) & 15u;
   if (fmt == ORC_INT2) return (words[word_index(n, k, K, 2, i / 16)] >> pair_shift(i, 2, 16)) & 3u;
   uint32_t lo = (words[word_index(n, k, K, 3, i / 16)] >> pair_shift(i, 2, 16)) & 3u;
-  uint32_t hi = (words[word_index(n, k, K, 3, 2)] >> pair_shift(i, 1, 32)) & 1u;
+  uint32_t hi = (words[word_index(n, k, K, 3, 2)] >> int3_high_shift(i)) & 1u;
   return lo | (hi << 2);
 }
 

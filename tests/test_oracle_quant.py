@@ -46,13 +46,14 @@ def test_hand_worked_groups(orc):
 def test_layout_positions_hand_computed(orc):
     # element (n=130, k=200) of a 256x256 matrix: n-block 1, k-block 1, group 2
     # inside the tile, position 8 inside the group (an even code: 4-bit nibble 0 of
-    # word 1; 2-bit field 4 of word 0; 3-bit field 4 of word 0 and bit 4 of word 2).
+    # word 1; 2-bit field 4 of word 0; 3-bit field 4 of word 0 and, pair m=4 being
+    # c=1, j=0, bit 8*0 + 1 + 0 = 1 of word 2).
     N = K = 256
     cases = {
         # bits: (code, [(byte offset, expected word), ...], base word)
         4: (5, [(29192, 0x8888888D)], 0x88888888),
         2: (-1, [(14344, 0xAAAAA9AA)], 0xAAAAAAAA),
-        3: (-3, [(21512, 0x00000100), (22536, 0xFFFFFFEF)], None),
+        3: (-3, [(21512, 0x00000100), (22536, 0xFFFFFFFD)], None),
     }
     for bits, (code, checks, base) in cases.items():
         q = np.zeros((N, K), np.int8)
