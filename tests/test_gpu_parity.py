@@ -188,6 +188,34 @@ def test_forward_prefill_chunks_and_tails():
     check_layer(L, 300)
 
 
+@pytest.mark.parametrize("T", [9, 300])
+def test_forward_single_tile_dims(T):
+    # H = F = 128: one 128-input tile per row block (no split-K), a gather row of 16
+    # chunks; decode (GEMV) and prefill (tcgen05) batch sizes
+    L = custom("tile1", T, 128, 128, 5, 2, [[3, 2, 4], [4, 4, 4], [2, 2, 2], [4, 3, 2], [2, 4, 3]])
+    check_layer(L, T)
+
+
+def test_forward_single_tile_dims_nvfp4():
+    L = custom("tile1fp4", 11, 128, 128, 4, 2, [[16, 16, 16]] * 4)
+    check_layer(L, 11)
+
+
+def test_forward_router_gemm_ragged_experts_bias():
+    # 72 experts (the last 64-expert tile ragged), split-K router planes, a bias
+    E = 72
+    L = custom("rgemm", 300, 1024, 256, E, 4, [[4, 2, 3]] * E)
+    bias = (np.random.default_rng(5).standard_normal(E) * 0.05).astype(np.float32)
+    check_layer(L, 300, bias=bias)
+
+
+def test_forward_permutation_block_edges():
+    # T*k = 1024 (the one-block permutation at its limit) and 1028 (the three-pass path)
+    L = custom("perm1k", 256, 256, 256, 16, 4, [[4, 4, 4], [2, 2, 2], [3, 2, 4], [4, 3, 2]] * 4)
+    check_layer(L, 256)
+    check_layer(L, 257)
+
+
 def test_forward_nvfp4_small():
     L = custom("fp4small", 23, 256, 384, 16, 6, [[16, 16, 16]] * 16)
     check_layer(L, 23)
