@@ -35,7 +35,8 @@ __global__ void combine_kernel(const float* __restrict__ o, const float* __restr
 }
 
 cudaError_t launch_combine(int T, int k, int H, const Workspace& ws, __nv_bfloat16* y, cudaStream_t stream) {
-  const int ny = (H / 4 + 255) / 256 < 8 ? (H / 4 + 255) / 256 : 8;  // column blocks: more parallelism for few tokens
+  int ny = T < 512 ? (H / 4 + 255) / 256 : 1;  // column blocks: more parallelism for few tokens
+  if (ny > 8) ny = 8;
   combine_kernel<<<dim3(T, ny), 256, 0, stream>>>(ws.o, ws.wts, ws.inv, k, H, y);
   return cudaGetLastError();
 }

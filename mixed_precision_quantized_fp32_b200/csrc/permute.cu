@@ -335,7 +335,8 @@ cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4,
     gather_fp8_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(ws.xq, ws.perm, R, H, k, (__half*)ws.xs,
                                                                      ws.counters, ws.counter_len);
   } else {
-    const int ny = (H / 8 + 127) / 128 < 8 ? (H / 8 + 127) / 128 : 8;  // column blocks: more parallelism for few rows
+    int ny = R < 512 ? (H / 8 + 127) / 128 : 1;  // column blocks: more parallelism for few rows
+    if (ny > 8) ny = 8;
     gather_f16_kernel<<<dim3(R, ny), 128, 0, stream>>>(x, ws.perm, R, H, k, (__half*)ws.xs, ws.xsum, ws.counters,
                                                        ws.counter_len);
   }
