@@ -2,6 +2,9 @@
 
   * hand-worked groups (tests/golden/int_group_examples.json): scale bits,
     codes (round-half-even ties) and packed words;
+  * a hand-worked NVFP4 block (tests/golden/nvfp4_group_example.json): tensor
+    scale, e4m3 block scale, e2m1 codes with ties to even, packed word and
+    the dequantized values;
   * hand-computed word / byte positions of single codes in multi-tile
     matrices for every format (the 128x128 tile layout);
   * an independent numpy implementation of the quantization rule built on
@@ -41,6 +44,26 @@ def test_hand_worked_groups(orc):
         for w_i, hexw in enumerate(e["words"]):
             assert _word(codes, 512 * w_i) == int(hexw, 16), (e["bits"], w_i)
         assert int(np.frombuffer(scales[:2].tobytes(), "<u2")[0]) == e["scale_bits"]
+
+
+def test_hand_worked_nvfp4_group(orc):
+    ex = json.load(open(os.path.join(GOLD, "nvfp4_group_example.json")))
+    N = K = 128
+    W = np.zeros((N, K), np.float32)
+    W[0, :8] = np.asarray(ex["w_block0"], np.float32)
+    v, sb, sT = orc.quant_nvfp4(W)
+    assert sT == ex["tensor_scale"]
+    assert int(sb[0, 0]) == ex["block0_scale_code"]
+    assert np.count_nonzero(sb) == 1
+    assert v[0, :8].tolist() == ex["codes_first8"]
+    assert np.count_nonzero(v) == np.count_nonzero(ex["codes_first8"])
+    codes, scales = orc.pack_nvfp4(v, sb)
+    assert _word(codes, 0) == int(ex["word0"], 16)
+    assert np.count_nonzero(codes) == 4  # the nonzero nibbles of word 0 fill four bytes
+    assert scales[0] == ex["block0_scale_code"] and np.count_nonzero(scales) == 1
+    deq = orc.decode_matrix(codes, scales, orc.FMT_NVFP4, N, K, sT)
+    np.testing.assert_array_equal(deq[0, :8], np.asarray(ex["dequant_first8"]))
+    assert np.count_nonzero(deq) == 7
 
 
 def test_layout_positions_hand_computed(orc):
