@@ -21,6 +21,7 @@
 // Every mbarrier wait is bounded; a wait that gives up raises an abort flag so
 // every role leaves its loop, writes MOE_ERR_TIMEOUT to the status word and
 // the CTA frees its TMEM before returning.
+#include <algorithm>
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
@@ -51,22 +52,44 @@ constexpr int kTcThreads = 32 * (kDeqWarps + 2);
 constexpr long long kWaitLimit = 4000000000LL;  // clock cycles, ~2 s
 constexpr int kPrefetchAhead = 4;                 // stages of packed codes warmed in L2 ahead of their copy
 
-template <int NMAT>
+// CG2: the work item runs on a pair of CTAs (one cluster) with cta_group::2
+// MMAs, each CTA holding half of the activation tile's token rows.
+// Stage layout: activation tile, NMAT dequantized weight tiles, NMAT code slots,
+// NMAT scale slots.  The code slot is sized for the widest format the launch
+// meets (Ring), so narrow layers get a deeper ring.
+template <int NMAT, bool CG2 = false>
 struct TcCfg {
-  static constexpr int kBBytes = kTcBN * kRowBytes;   // activation tile
+  static constexpr int kBRows = CG2 ? kTcBN / 2 : kTcBN;
+  static constexpr int kBBytes = kBRows * kRowBytes;  // activation tile (this CTA's rows)
   static constexpr int kABytes = kTcBM * kRowBytes;   // dequantized weight tile
-  static constexpr int kCodeBytes = kGroups * 2048;   // <= 4 words x 128 rows x 4 bytes per group
   static constexpr int kScaleBytes = kGroups * 256;   // one fp16 group or two e4m3 blocks x 128 rows
   static constexpr int kOffB = 0;
   static constexpr int kOffA = kBBytes;
   static constexpr int kOffCodes = kOffA + NMAT * kABytes;
-  static constexpr int kOffScales = kOffCodes + NMAT * kCodeBytes;
-  static constexpr int kStageBytes = (kOffScales + NMAT * kScaleBytes + 1023) / 1024 * 1024;
-  static constexpr int kBarBytes = 256;
-  static constexpr int kStages = (232448 - kBarBytes - 1024) / kStageBytes;  // as many as fit
-  static constexpr int kSmem = kStages * kStageBytes + kBarBytes + 1024;
 };
-static_assert(TcCfg<2>::kStages >= 3 && TcCfg<1>::kStages >= 4 && TcCfg<1>::kStages <= 8, "pipeline depth");
+constexpr int kMaxStages = 8;
+constexpr int kBarBytes = 256;                       // 3 barriers per stage + 2 + TMEM slot + flag
+constexpr int kSmemMax = 232448;                     // opt-in shared memory per CTA
+static_assert(3 * 8 * kMaxStages + 32 <= kBarBytes, "barrier area");
+
+struct Ring {
+  int stages;       // stages in the ring (<= kMaxStages)
+  int stage_bytes;  // one stage, a multiple of 1024
+  int code_bytes;   // one matrix's code slot: kGroups x 512 bytes per code word of the widest format
+  int off_scales;   // scale slots
+};
+
+template <int NMAT, bool CG2>
+Ring make_ring(int max_words) {
+  using C = TcCfg<NMAT, CG2>;
+  Ring r;
+  r.code_bytes = kGroups * 512 * max_words;
+  r.off_scales = C::kOffCodes + NMAT * r.code_bytes;
+  r.stage_bytes = (r.off_scales + NMAT * C::kScaleBytes + 1023) / 1024 * 1024;
+  r.stages = min(kMaxStages, (kSmemMax - kBarBytes - 1024) / r.stage_bytes);
+  return r;
+}
+inline int ring_smem(const Ring& r) { return r.stages * r.stage_bytes + kBarBytes + 1024; }
 
 struct TcArgs {
   const uint8_t* packed;
@@ -83,6 +106,7 @@ struct TcArgs {
   void* out;               // gate/up: h [rows][F] (fp16, or fp32 for NVFP4); down: o fp32 [rows][H]
   int32_t* status;
   unsigned long long* trace;  // diagnostics: per-stage clock64 stamps of CTA 0 (or null)
+  Ring ring;
 };
 
 // Stamp event `ev` of global stage counter `i` (CTA 0 only, first MOE_TRACE_STAGES stages).
@@ -187,11 +211,11 @@ __device__ __forceinline__ uint64_t scale_stage_offset(int mt, int g, int K, int
 // second): wait for the stage's codes, convert this thread's units, publish
 // them to the tensor core and release the stage to the MMA warp.  Returns
 // false if a bounded wait gave up.
-template <int NMAT, int F0, int F1>
-__device__ __noinline__ bool dequant_item(uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
+template <int NMAT, bool CG2, int F0, int F1>
+__device__ __noinline__ bool dequant_item(const Ring R, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
                                           volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
                                           uint32_t& phase, int& gstage, unsigned long long* trace) {
-  using C = TcCfg<NMAT>;
+  using C = TcCfg<NMAT, CG2>;
   constexpr int kUnits = NMAT * kGroups * 4 / kThreadsPerRow;
   static_assert(NMAT == 1 || kUnits % 2 == 0, "units must alternate matrices evenly");
   const int lane = threadIdx.x & 31;
@@ -199,17 +223,17 @@ __device__ __noinline__ bool dequant_item(uint8_t* smem, uint64_t* load_full, ui
   for (int ks = 0; ks < ksteps; ++ks) {
     if (!__all_sync(0xffffffffu, ptx::mbar_wait(&load_full[stage], phase, abort_flag, kWaitLimit))) return false;
     if (threadIdx.x == 0) trace_stamp(trace, 2, gstage);
-    uint8_t* sb = smem + stage * C::kStageBytes;
+    uint8_t* sb = smem + stage * R.stage_bytes;
     uint4 v[kUnits];
 #pragma unroll
     for (int i = 0; i < kUnits; ++i) {
       const int m = i % NMAT, cg = cg0 + i / NMAT, g = cg >> 2;
-      const uint8_t* scales = sb + C::kOffScales + m * C::kScaleBytes + g * 256;
+      const uint8_t* scales = sb + R.off_scales + m * C::kScaleBytes + g * 256;
       if (m == 0) {
         const uint32_t* codes = reinterpret_cast<const uint32_t*>(sb + C::kOffCodes) + g * fmt_words(F0) * 128;
         v[i] = dequant_chunk<F0>(codes, scales, n, cg & 3);
       } else {
-        const uint32_t* codes = reinterpret_cast<const uint32_t*>(sb + C::kOffCodes + C::kCodeBytes) +
+        const uint32_t* codes = reinterpret_cast<const uint32_t*>(sb + C::kOffCodes + R.code_bytes) +
                                 g * fmt_words(F1) * 128;
         v[i] = dequant_chunk<F1>(codes, scales, n, cg & 3);
       }
@@ -221,10 +245,15 @@ __device__ __noinline__ bool dequant_item(uint8_t* smem, uint64_t* load_full, ui
     }
     ptx::fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(&a_full[stage]);
+    if (lane == 0) {
+      if (CG2)
+        ptx::mbar_arrive_cluster(&a_full[stage], 0);  // the even CTA issues the pair's MMAs
+      else
+        ptx::mbar_arrive(&a_full[stage]);
+    }
     if (threadIdx.x == 0) trace_stamp(trace, 3, gstage);
     ++gstage;
-    if (++stage == C::kStages) {
+    if (++stage == R.stages) {
       stage = 0;
       phase ^= 1u;
     }
@@ -233,69 +262,86 @@ __device__ __noinline__ bool dequant_item(uint8_t* smem, uint64_t* load_full, ui
 }
 
 // Runtime format pair -> the matching dequant_item instantiation.
-template <int NMAT, int F0>
-__device__ __forceinline__ bool dequant_item_f1(int f1, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
+template <int NMAT, bool CG2, int F0>
+__device__ __forceinline__ bool dequant_item_f1(int f1, const Ring R, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
                                                 volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
                                                 uint32_t& phase, int& gstage, unsigned long long* trace) {
-  if (NMAT == 1) return dequant_item<NMAT, F0, F0>(smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+  if (NMAT == 1) return dequant_item<NMAT, CG2, F0, F0>(R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
   switch (f1) {
-    case MOE_FMT_INT2: return dequant_item<NMAT, F0, MOE_FMT_INT2>(smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    case MOE_FMT_INT3: return dequant_item<NMAT, F0, MOE_FMT_INT3>(smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    case MOE_FMT_INT4: return dequant_item<NMAT, F0, MOE_FMT_INT4>(smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    default: return dequant_item<NMAT, F0, MOE_FMT_NVFP4>(smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT2: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT2>(R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT3: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT3>(R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT4: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT4>(R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    default: return dequant_item<NMAT, CG2, F0, MOE_FMT_NVFP4>(R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
   }
 }
-template <int NMAT>
-__device__ __forceinline__ bool dequant_item_any(int f0, int f1, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
+template <int NMAT, bool CG2>
+__device__ __forceinline__ bool dequant_item_any(int f0, int f1, const Ring R, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
                                                  volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
                                                  uint32_t& phase, int& gstage, unsigned long long* trace) {
   switch (f0) {
-    case MOE_FMT_INT2: return dequant_item_f1<NMAT, MOE_FMT_INT2>(f1, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    case MOE_FMT_INT3: return dequant_item_f1<NMAT, MOE_FMT_INT3>(f1, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    case MOE_FMT_INT4: return dequant_item_f1<NMAT, MOE_FMT_INT4>(f1, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    default: return dequant_item_f1<NMAT, MOE_FMT_NVFP4>(f1, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT2: return dequant_item_f1<NMAT, CG2, MOE_FMT_INT2>(f1, R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT3: return dequant_item_f1<NMAT, CG2, MOE_FMT_INT3>(f1, R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT4: return dequant_item_f1<NMAT, CG2, MOE_FMT_INT4>(f1, R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    default: return dequant_item_f1<NMAT, CG2, MOE_FMT_NVFP4>(f1, R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
   }
 }
 
-template <int NMAT>
+template <int NMAT, bool CG2>
 __global__ void __launch_bounds__(kTcThreads, 1)
     expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
-  using C = TcCfg<NMAT>;
+  using C = TcCfg<NMAT, CG2>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  const Ring R = a.ring;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + R.stages * R.stage_bytes);
   uint64_t* load_full = bars;
-  uint64_t* a_full = bars + C::kStages;
-  uint64_t* stage_empty = bars + 2 * C::kStages;
-  uint64_t* acc_full = bars + 3 * C::kStages;
+  uint64_t* a_full = bars + R.stages;
+  uint64_t* stage_empty = bars + 2 * R.stages;
+  uint64_t* acc_full = bars + 3 * R.stages;
   uint64_t* acc_empty = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // CTA pairs: the even CTA (rank 0) issues the MMAs of both, so the dequant and
+  // epilogue warps of both CTAs arrive on its barriers (a plain remote arrive:
+  // release at CTA scope, as a cluster-scope release costs ~1600 cycles here);
+  // its commits reach both CTAs.
+  const uint32_t rank = CG2 ? ptx::cluster_ctarank() : 0u;
+  constexpr int kPairCtas = CG2 ? 2 : 1;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < R.stages; ++s) {
       ptx::mbar_init(&load_full[s], 1);
-      ptx::mbar_init(&a_full[s], kDeqWarps);  // one arrival per dequant warp
+      ptx::mbar_init(&a_full[s], kDeqWarps * kPairCtas);  // one arrival per dequant warp of the pair
       ptx::mbar_init(&stage_empty[s], 1);
     }
     ptx::mbar_init(acc_full, 1);
-    ptx::mbar_init(acc_empty, kDeqWarps);
+    ptx::mbar_init(acc_empty, kDeqWarps * kPairCtas);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
   if (warp == kMmaWarp) {
-    ptx::tmem_alloc(tmem_slot, 512);
-    ptx::tmem_relinquish();
+    if (CG2) {
+      ptx::tmem_alloc2(tmem_slot, 512);
+      ptx::tmem_relinquish2();
+    } else {
+      ptx::tmem_alloc(tmem_slot, 512);
+      ptx::tmem_relinquish();
+    }
   }
   if (warp == kTmaWarp && lane == 0) ptx::prefetch_tmap(&tmap_b);
   ptx::tc_fence_before();
   __syncthreads();
+  if (CG2) ptx::cluster_sync();  // the peer's barriers are initialised before any remote arrival
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int m_tiles = a.N / kTcBM / (a.pair ? 2 : 1);  // work items per chunk
+  // work items per chunk: 128-row weight tiles (pairs of them in pair mode), two
+  // per item on a CTA pair, the even CTA taking the first
+  const int m_tiles = a.N / kTcBM / (a.pair ? 2 : 1) / kPairCtas;
   const int total = *a.chunk_count * m_tiles;
+  const int first = CG2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int stride = CG2 ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int ksteps = a.K / kTcBK;
   const LayerHdr L = hdr_view(a.packed, a.E, a.H, a.F);
   bool ok = true;
@@ -311,9 +357,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int stage = 0, gstage = 0;
     uint32_t phase = 0;
     uint32_t issued = 0, issued_phase = 0;  // per stage: a load was armed, and its parity
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const int c = t / m_tiles, mt = t % m_tiles;
-      const int e = a.chunks[3 * c], row0 = a.chunks[3 * c + 1];
+    for (int t = first; t < total && ok; t += stride) {
+      const int c = t / m_tiles, mt = (t % m_tiles) * kPairCtas + (int)rank;
+      const int e = a.chunks[3 * c];
+      // this CTA's token rows of the MMA's N = nmma columns: the first or second half
+      const int nmma = min(kTcBN, (a.chunks[3 * c + 2] + 15) & ~15);
+      const int row0 = a.chunks[3 * c + 1] + (int)rank * (nmma / 2);
       // A weight tile's codes (and scales) are contiguous along K, so each stage's
       // slice is the tile base plus ks times a fixed stride.
       const uint8_t* cptr[NMAT];
@@ -342,14 +391,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         if (lane == 0) {
           trace_stamp(a.trace, 0, gstage);
-          uint8_t* sb = smem + stage * C::kStageBytes;
+          uint8_t* sb = smem + stage * R.stage_bytes;
           ptx::mbar_arrive_expect_tx(&load_full[stage], bytes);
           ptx::tma_load_2d(sb + C::kOffB, &tmap_b, ks * kTcBK, row0, &load_full[stage]);
 #pragma unroll
           for (int m = 0; m < NMAT; ++m) {
-            ptx::bulk_load(sb + C::kOffCodes + m * C::kCodeBytes, cptr[m] + (size_t)ks * cbytes[m], cbytes[m],
+            ptx::bulk_load(sb + C::kOffCodes + m * R.code_bytes, cptr[m] + (size_t)ks * cbytes[m], cbytes[m],
                            &load_full[stage]);
-            ptx::bulk_load(sb + C::kOffScales + m * C::kScaleBytes, sptr[m] + (size_t)ks * C::kScaleBytes,
+            ptx::bulk_load(sb + R.off_scales + m * C::kScaleBytes, sptr[m] + (size_t)ks * C::kScaleBytes,
                            (uint32_t)C::kScaleBytes, &load_full[stage]);
           }
           trace_stamp(a.trace, 1, gstage);
@@ -358,14 +407,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
         issued |= 1u << stage;
         issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-        if (++stage == C::kStages) {
+        if (++stage == R.stages) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
     // never leave while a copy may still be landing in shared memory
-    for (int s = 0; s < C::kStages; ++s)
+    for (int s = 0; s < R.stages; ++s)
       if (issued & (1u << s)) ptx::mbar_wait(&load_full[s], (issued_phase >> s) & 1u, abort_flag, kWaitLimit / 4);
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -373,11 +422,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t phase = 0, acc_phase = 0;
     const uint32_t sbase = ptx::smem_u32(smem);
     bool committed = false;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    for (int t = first; t < total && ok && rank == 0; t += stride) {
       const int c = t / m_tiles;
       const int rows = a.chunks[3 * c + 2];
       const int nmma = min(kTcBN, (rows + 15) & ~15);
-      const uint32_t idesc = ptx::idesc_f16_f32(kTcBM, nmma);
+      const uint32_t idesc = ptx::idesc_f16_f32(kTcBM * kPairCtas, nmma);
       if (!wait_all(acc_empty, acc_phase ^ 1u)) {
         ok = false;
         break;
@@ -392,30 +441,43 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ptx::tc_fence_after();
         if (lane == 0) trace_stamp(a.trace, 4, gstage);
         if (lane == 0) {
-          const uint32_t st = sbase + (uint32_t)(stage * C::kStageBytes);
+          const uint32_t st = sbase + (uint32_t)(stage * R.stage_bytes);
 #pragma unroll
           for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-            for (int k16 = 0; k16 < kTcBK / 16; ++k16)
-              ptx::mma_f16_ss(tmem + (uint32_t)(m * 256), tile_desc(st + C::kOffA + m * C::kABytes + k16 * 32),
-                              tile_desc(st + C::kOffB + k16 * 32), idesc, (ks | k16) != 0);
-          ptx::mma_commit(&stage_empty[stage]);
+            for (int k16 = 0; k16 < kTcBK / 16; ++k16) {
+              const uint64_t ad = tile_desc(st + C::kOffA + m * C::kABytes + k16 * 32);
+              const uint64_t bd = tile_desc(st + C::kOffB + k16 * 32);
+              if (CG2)
+                ptx::mma2_f16_ss(tmem + (uint32_t)(m * 256), ad, bd, idesc, (ks | k16) != 0);
+              else
+                ptx::mma_f16_ss(tmem + (uint32_t)(m * 256), ad, bd, idesc, (ks | k16) != 0);
+            }
+          if (CG2)
+            ptx::mma2_commit_mc(&stage_empty[stage], 0x3);
+          else
+            ptx::mma_commit(&stage_empty[stage]);
           trace_stamp(a.trace, 5, gstage);
         }
         ++gstage;
         __syncwarp();
         committed = true;
-        if (++stage == C::kStages) {
+        if (++stage == R.stages) {
           stage = 0;
           phase ^= 1u;
         }
       }
       if (!ok) break;
-      if (lane == 0) ptx::mma_commit(acc_full);
+      if (lane == 0) {
+        if (CG2)
+          ptx::mma2_commit_mc(acc_full, 0x3);
+        else
+          ptx::mma_commit(acc_full);
+      }
       __syncwarp();
     }
     if (committed) {  // the last commit lands once every MMA issued by this CTA has completed
-      const int last = (stage + C::kStages - 1) % C::kStages;
+      const int last = (stage + R.stages - 1) % R.stages;
       const uint32_t par = (stage == 0) ? (phase ^ 1u) : phase;
       ptx::mbar_wait(&stage_empty[last], par, abort_flag, kWaitLimit / 4);
     }
@@ -433,8 +495,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int u0 = sel * kUnits;
     int stage = 0, gstage = 0, item = 0;
     uint32_t phase = 0, acc_phase = 0;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++item) {
-      const int c = t / m_tiles, mt = t % m_tiles;
+    for (int t = first; t < total && ok; t += stride, ++item) {
+      const int c = t / m_tiles, mt = (t % m_tiles) * kPairCtas + (int)rank;
       const int e = a.chunks[3 * c], row0 = a.chunks[3 * c + 1], rows = a.chunks[3 * c + 2];
       int fmt[NMAT];
       float tsc[NMAT];
@@ -444,7 +506,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         fmt[m] = L.fmt[i];
         tsc[m] = fmt[m] == MOE_FMT_NVFP4 ? L.tscale[i] : 1.0f;
       }
-      if (!dequant_item_any<NMAT>(fmt[0], fmt[NMAT - 1], smem, load_full, a_full, abort_flag, ksteps, n, u0, stage,
+      if (!dequant_item_any<NMAT, CG2>(fmt[0], fmt[NMAT - 1], a.ring, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage,
                                   phase, gstage, a.trace)) {
         ok = false;
         break;
@@ -497,20 +559,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(acc_empty);
+      if (lane == 0) {
+        if (CG2)
+          ptx::mbar_arrive_cluster(acc_empty, 0);
+        else
+          ptx::mbar_arrive(acc_empty);
+      }
       if (threadIdx.x == 0) trace_stamp(a.trace, 7, item);
     }
   }
 
   if (!ok) {
     *abort_flag = 1;
+    if (CG2) ptx::st_cluster_u32(abort_flag, rank ^ 1u, 1);  // the peer's waits give up too
     if (a.status) atomicExch(a.status, (int32_t)MOE_ERR_TIMEOUT);
   }
   ptx::tc_fence_before();
   __syncthreads();
+  // a pair leaves together: the even CTA's MMAs read the odd CTA's shared memory
+  // and write its tensor memory, and the odd CTA arrives on the even one's barriers
+  if (CG2) ptx::cluster_sync();
   if (warp == kMmaWarp) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, 512);
+    if (CG2)
+      ptx::tmem_dealloc2(tmem, 512);
+    else
+      ptx::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -538,31 +612,62 @@ int sm_count() {
   return n[dev];
 }
 
-template <int NMAT>
-cudaError_t launch_tc(const TcArgs& a, const void* act, int rows_total, cudaStream_t stream) {
+template <int NMAT, bool CG2>
+cudaError_t launch_tc(TcArgs a, int max_words, const void* act, int rows_total, cudaStream_t stream) {
+  using C = TcCfg<NMAT, CG2>;
+  a.ring = make_ring<NMAT, CG2>(max_words);
+  if (a.ring.stages < 3) return cudaErrorInvalidConfiguration;
+  const int smem = ring_smem(a.ring);
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap map;
   const cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)rows_total};
   const cuuint64_t strides[1] = {(cuuint64_t)a.K * 2u};
-  const cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)kTcBN};
+  const cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)C::kBRows};
   const CUtensorMapSwizzle swz = kRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   const cuuint32_t estr[2] = {1u, 1u};
   if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(act), dims, strides, box, estr,
           CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  auto kern = expert_gemm_tc_kernel<NMAT>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<NMAT>::kSmem);
+  auto kern = expert_gemm_tc_kernel<NMAT, CG2>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
-  kern<<<sm_count(), kTcThreads, TcCfg<NMAT>::kSmem, stream>>>(map, a);
-  return cudaGetLastError();
+  if (!CG2) {
+    kern<<<sm_count(), kTcThreads, smem, stream>>>(map, a);
+    return cudaGetLastError();
+  }
+  // one persistent pair of CTAs per pair of SMs: as many clusters as can be
+  // resident at once (a GPC with an odd number of free SMs leaves one idle)
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3((unsigned)(sm_count() & ~1));
+  int clusters = 0;
+  err = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+  if (err != cudaSuccess) return err;
+  if (clusters < 1) return cudaErrorInvalidConfiguration;
+  cfg.gridDim = dim3((unsigned)(2 * min(clusters, sm_count() / 2)));
+  return cudaLaunchKernelEx(&cfg, kern, map, a);
 }
 
 }  // namespace
 
-cudaError_t launch_expert_gemm_tc(const uint8_t* packed, int E, int H, int F, int T, int k, bool fp4, bool gateup,
-                                  const Workspace& ws, int32_t* status, uint64_t* trace, cudaStream_t stream) {
+cudaError_t launch_expert_gemm_tc(const uint8_t* packed, const uint8_t* fmt_host, int E, int H, int F, int T, int k,
+                                  bool fp4, bool gateup, const Workspace& ws, int32_t* status, uint64_t* trace,
+                                  cudaStream_t stream) {
+  // widest code format of the projections this launch reads (sizes the code slots)
+  int max_words = 1;
+  for (int e = 0; e < E; ++e)
+    for (int p = gateup ? 0 : 2; p <= (gateup ? 1 : 2); ++p) max_words = std::max(max_words, fmt_words(fmt_host[e * 3 + p]));
   TcArgs a{};
   a.trace = gateup ? reinterpret_cast<unsigned long long*>(trace) : nullptr;
   a.packed = packed;
@@ -581,7 +686,8 @@ cudaError_t launch_expert_gemm_tc(const uint8_t* packed, int E, int H, int F, in
     a.proj = 0;
     a.row_scale = fp4 ? ws.sx : nullptr;
     a.out = ws.h;
-    return launch_tc<2>(a, ws.xs, R, stream);
+    if ((F / kTcBM) % 2 == 0) return launch_tc<2, true>(a, max_words, ws.xs, R, stream);  // weight tiles in pairs of CTAs
+    return launch_tc<2, false>(a, max_words, ws.xs, R, stream);
   }
   a.N = H;
   a.K = F;
@@ -590,9 +696,10 @@ cudaError_t launch_expert_gemm_tc(const uint8_t* packed, int E, int H, int F, in
   a.out = ws.o;
   if ((H / kTcBM) % 2 == 0) {  // pairs of weight tiles share each activation tile
     a.pair = 1;
-    return launch_tc<2>(a, fp4 ? ws.hb : ws.h, R, stream);
+    if ((H / kTcBM) % 4 == 0) return launch_tc<2, true>(a, max_words, fp4 ? ws.hb : ws.h, R, stream);
+    return launch_tc<2, false>(a, max_words, fp4 ? ws.hb : ws.h, R, stream);
   }
-  return launch_tc<1>(a, fp4 ? ws.hb : ws.h, R, stream);
+  return launch_tc<1, false>(a, max_words, fp4 ? ws.hb : ws.h, R, stream);
 }
 
 }  // namespace moe

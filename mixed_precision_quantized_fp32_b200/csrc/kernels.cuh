@@ -24,8 +24,9 @@ cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4,
 cudaError_t launch_act_quant_h(int R, int F, const Workspace& ws, uint8_t* dbg_hq, float* dbg_sh,
                                cudaStream_t stream);
 
-cudaError_t launch_expert_gemm_tc(const uint8_t* packed, int E, int H, int F, int T, int k, bool fp4, bool gateup,
-                                  const Workspace& ws, int32_t* status, uint64_t* trace, cudaStream_t stream);
+cudaError_t launch_expert_gemm_tc(const uint8_t* packed, const uint8_t* fmt_host, int E, int H, int F, int T, int k,
+                                  bool fp4, bool gateup, const Workspace& ws, int32_t* status, uint64_t* trace,
+                                  cudaStream_t stream);
 
 // K parts of the decode GEMV for R expert rows on an N x K projection (nmat
 // matrices); the workspace holds P*R*N*nmat fp32 partials when P > 1.
