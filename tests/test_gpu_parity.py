@@ -188,6 +188,14 @@ def test_forward_prefill_chunks_and_tails():
     check_layer(L, 300)
 
 
+def test_forward_cta_pairs_ragged_chunks():
+    # tcgen05 path on CTA pairs for both GEMMs: gate/up F/128 = 2 weight tiles, down H/128 = 4 (two
+    # pairs of tiles).  12 experts share 600 rows, a few dozen each, so every chunk's token count N
+    # (rounded up to 16) splits over the two CTAs at N/2 rows, well short of a full 128-row half.
+    L = custom("pairs", 300, 512, 256, 12, 2, [[3, 2, 4], [4, 4, 4], [2, 2, 2], [4, 3, 2]] * 3)
+    check_layer(L, 300)
+
+
 @pytest.mark.parametrize("T", [9, 300])
 def test_forward_single_tile_dims(T):
     # H = F = 128: one 128-input tile per row block (no split-K), a gather row of 16
