@@ -177,6 +177,13 @@ typedef struct {
                          a free stage, 1 producer issued its copies, 2 consumer warp 0 found it
                          landed, 3 consumer warp 0 released it; per work item: row 4 producer
                          loaded the following item, 6 consumers started it, 7 finished it. */
+  uint32_t test_withhold; /* test hook, 0 in normal use: nonzero makes the copy warps of the expert
+                             GEMMs issue no loads, so their consumers' bounded waits run out.  The
+                             call then writes MOE_ERR_TIMEOUT to *status; the outputs are undefined
+                             and the context stays usable. */
+  uint32_t wait_cycles;   /* budget of the expert GEMMs' waits on their pipelines, in clock cycles;
+                             0: the default (~1-2 s).  Waits for copies still in flight at exit keep
+                             the default. */
 } moe_debug;
 
 #define MOE_TRACE_EVENTS 8

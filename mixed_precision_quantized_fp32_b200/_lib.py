@@ -34,7 +34,8 @@ class MoeDebug(C.Structure):
     _fields_ = [("topk_idx", C.c_void_p), ("topk_w", C.c_void_p), ("perm", C.c_void_p),
                 ("inv", C.c_void_p), ("counts", C.c_void_p), ("xq", C.c_void_p), ("sx", C.c_void_p),
                 ("hq", C.c_void_p), ("sh", C.c_void_p), ("status", C.c_void_p),
-                ("stage_events", C.c_void_p), ("trace", C.c_void_p)]
+                ("stage_events", C.c_void_p), ("trace", C.c_void_p),
+                ("test_withhold", C.c_uint32), ("wait_cycles", C.c_uint32)]
 
 
 class MoeError(RuntimeError):

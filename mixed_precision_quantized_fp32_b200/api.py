@@ -92,6 +92,7 @@ def workspace_bytes(layer: PackedLayer, T: int, k: int) -> int:
 
 
 DEBUG_FIELDS = ("topk_idx", "topk_w", "perm", "inv", "counts", "xq", "sx", "hq", "sh", "status", "trace")
+DEBUG_INTS = ("test_withhold", "wait_cycles")  # plain integers, see moe_debug in moe.h
 
 
 def moe_layer_forward(x: torch.Tensor, router_w: torch.Tensor, router_b: torch.Tensor | None,
@@ -113,6 +114,9 @@ def moe_layer_forward(x: torch.Tensor, router_w: torch.Tensor, router_b: torch.T
     if debug or stage_events:
         dbg = MoeDebug()
         for name, t in (debug or {}).items():
+            if name in DEBUG_INTS:
+                setattr(dbg, name, int(t))
+                continue
             if name not in DEBUG_FIELDS:
                 raise KeyError(name)
             setattr(dbg, name, _ptr(t))

@@ -194,10 +194,12 @@ extern "C" moe_status moe_layer_forward(const void* x, int32_t T, const float* r
   if (!mark(3)) return MOE_ERR_CUDA;
   int32_t* status = d.status ? d.status : wsp.status;
   auto gemm = [&](bool gateup) -> cudaError_t {
-    return plan.tc ? launch_expert_gemm_tc(packed, w->fmt, E, H, F, T, k, fp4, gateup, wsp, status, d.trace, stream)
+    const GemmHooks hooks{d.test_withhold, d.wait_cycles};
+    return plan.tc ? launch_expert_gemm_tc(packed, w->fmt, E, H, F, T, k, fp4, gateup, wsp, status, d.trace, hooks,
+                                           stream)
                    : launch_expert_gemv(packed, w->packed_bytes, w->fmt, E, H, F, T * k, k, fp4, gateup,
                                         plan.max_chunks, plan.chunk_rows, wsp, status, gateup ? d.trace : nullptr,
-                                        stream);
+                                        hooks, stream);
   };
   if (gemm(true) != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(4)) return MOE_ERR_CUDA;

@@ -107,6 +107,8 @@ struct TcArgs {
   int32_t* status;
   unsigned long long* trace;  // diagnostics: per-stage clock64 stamps of CTA 0 (or null)
   Ring ring;
+  long long wait;             // budget of the pipeline waits, clock cycles
+  int withhold;               // test hook: the TMA warp issues no loads (the waits run out)
 };
 
 // Stamp event `ev` of global stage counter `i` (CTA 0 only, first MOE_TRACE_STAGES stages).
@@ -212,16 +214,16 @@ __device__ __forceinline__ uint64_t scale_stage_offset(int mt, int g, int K, int
 // them to the tensor core and release the stage to the MMA warp.  Returns
 // false if a bounded wait gave up.
 template <int NMAT, bool CG2, int F0, int F1>
-__device__ __noinline__ bool dequant_item(const Ring R, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
-                                          volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
-                                          uint32_t& phase, int& gstage, unsigned long long* trace) {
+__device__ __noinline__ bool dequant_item(const Ring R, long long wait, uint8_t* smem, uint64_t* load_full,
+                                          uint64_t* a_full, volatile int* abort_flag, int ksteps, int n, int u0,
+                                          int& stage, uint32_t& phase, int& gstage, unsigned long long* trace) {
   using C = TcCfg<NMAT, CG2>;
   constexpr int kUnits = NMAT * kGroups * 4 / kThreadsPerRow;
   static_assert(NMAT == 1 || kUnits % 2 == 0, "units must alternate matrices evenly");
   const int lane = threadIdx.x & 31;
   const int cg0 = u0 / NMAT;
   for (int ks = 0; ks < ksteps; ++ks) {
-    if (!__all_sync(0xffffffffu, ptx::mbar_wait(&load_full[stage], phase, abort_flag, kWaitLimit))) return false;
+    if (!__all_sync(0xffffffffu, ptx::mbar_wait(&load_full[stage], phase, abort_flag, wait))) return false;
     if (threadIdx.x == 0) trace_stamp(trace, 2, gstage);
     uint8_t* sb = smem + stage * R.stage_bytes;
     uint4 v[kUnits];
@@ -263,26 +265,26 @@ __device__ __noinline__ bool dequant_item(const Ring R, uint8_t* smem, uint64_t*
 
 // Runtime format pair -> the matching dequant_item instantiation.
 template <int NMAT, bool CG2, int F0>
-__device__ __forceinline__ bool dequant_item_f1(int f1, const Ring R, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
+__device__ __forceinline__ bool dequant_item_f1(int f1, const Ring R, long long wait, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
                                                 volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
                                                 uint32_t& phase, int& gstage, unsigned long long* trace) {
-  if (NMAT == 1) return dequant_item<NMAT, CG2, F0, F0>(R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+  if (NMAT == 1) return dequant_item<NMAT, CG2, F0, F0>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
   switch (f1) {
-    case MOE_FMT_INT2: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT2>(R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    case MOE_FMT_INT3: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT3>(R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    case MOE_FMT_INT4: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT4>(R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    default: return dequant_item<NMAT, CG2, F0, MOE_FMT_NVFP4>(R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT2: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT2>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT3: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT3>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT4: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT4>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    default: return dequant_item<NMAT, CG2, F0, MOE_FMT_NVFP4>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
   }
 }
 template <int NMAT, bool CG2>
-__device__ __forceinline__ bool dequant_item_any(int f0, int f1, const Ring R, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
+__device__ __forceinline__ bool dequant_item_any(int f0, int f1, const Ring R, long long wait, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
                                                  volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
                                                  uint32_t& phase, int& gstage, unsigned long long* trace) {
   switch (f0) {
-    case MOE_FMT_INT2: return dequant_item_f1<NMAT, CG2, MOE_FMT_INT2>(f1, R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    case MOE_FMT_INT3: return dequant_item_f1<NMAT, CG2, MOE_FMT_INT3>(f1, R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    case MOE_FMT_INT4: return dequant_item_f1<NMAT, CG2, MOE_FMT_INT4>(f1, R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    default: return dequant_item_f1<NMAT, CG2, MOE_FMT_NVFP4>(f1, R, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT2: return dequant_item_f1<NMAT, CG2, MOE_FMT_INT2>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT3: return dequant_item_f1<NMAT, CG2, MOE_FMT_INT3>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT4: return dequant_item_f1<NMAT, CG2, MOE_FMT_INT4>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    default: return dequant_item_f1<NMAT, CG2, MOE_FMT_NVFP4>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
   }
 }
 
@@ -350,7 +352,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // made warp-uniform, and only lane 0 issues TMA / MMA / commit, so no warp
   // reaches the final block barrier diverged.
   auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-    return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort_flag, kWaitLimit)) != 0;
+    return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort_flag, a.wait)) != 0;
   };
 
   if (warp == kTmaWarp) {
@@ -389,7 +391,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           ok = false;
           break;
         }
-        if (lane == 0) {
+        if (lane == 0 && !a.withhold) {
           trace_stamp(a.trace, 0, gstage);
           uint8_t* sb = smem + stage * R.stage_bytes;
           ptx::mbar_arrive_expect_tx(&load_full[stage], bytes);
@@ -405,8 +407,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         ++gstage;
         __syncwarp();
-        issued |= 1u << stage;
-        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+        if (!a.withhold) {
+          issued |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+        }
         if (++stage == R.stages) {
           stage = 0;
           phase ^= 1u;
@@ -415,7 +419,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     // never leave while a copy may still be landing in shared memory
     for (int s = 0; s < R.stages; ++s)
-      if (issued & (1u << s)) ptx::mbar_wait(&load_full[s], (issued_phase >> s) & 1u, abort_flag, kWaitLimit / 4);
+      if (issued & (1u << s)) ptx::mbar_drain(&load_full[s], (issued_phase >> s) & 1u, kWaitLimit / 4);
     __syncwarp();
   } else if (warp == kMmaWarp) {
     int stage = 0, gstage = 0;
@@ -479,7 +483,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (committed) {  // the last commit lands once every MMA issued by this CTA has completed
       const int last = (stage + R.stages - 1) % R.stages;
       const uint32_t par = (stage == 0) ? (phase ^ 1u) : phase;
-      ptx::mbar_wait(&stage_empty[last], par, abort_flag, kWaitLimit / 4);
+      ptx::mbar_drain(&stage_empty[last], par, kWaitLimit / 4);
     }
     __syncwarp();
   } else {
@@ -506,7 +510,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         fmt[m] = L.fmt[i];
         tsc[m] = fmt[m] == MOE_FMT_NVFP4 ? L.tscale[i] : 1.0f;
       }
-      if (!dequant_item_any<NMAT, CG2>(fmt[0], fmt[NMAT - 1], a.ring, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage,
+      if (!dequant_item_any<NMAT, CG2>(fmt[0], fmt[NMAT - 1], a.ring, a.wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage,
                                   phase, gstage, a.trace)) {
         ok = false;
         break;
@@ -663,13 +667,15 @@ cudaError_t launch_tc(TcArgs a, int max_words, const void* act, int rows_total, 
 
 cudaError_t launch_expert_gemm_tc(const uint8_t* packed, const uint8_t* fmt_host, int E, int H, int F, int T, int k,
                                   bool fp4, bool gateup, const Workspace& ws, int32_t* status, uint64_t* trace,
-                                  cudaStream_t stream) {
+                                  GemmHooks hooks, cudaStream_t stream) {
   // widest code format of the projections this launch reads (sizes the code slots)
   int max_words = 1;
   for (int e = 0; e < E; ++e)
     for (int p = gateup ? 0 : 2; p <= (gateup ? 1 : 2); ++p) max_words = std::max(max_words, fmt_words(fmt_host[e * 3 + p]));
   TcArgs a{};
   a.trace = gateup ? reinterpret_cast<unsigned long long*>(trace) : nullptr;
+  a.wait = hooks.wait_cycles ? (long long)hooks.wait_cycles : kWaitLimit;
+  a.withhold = hooks.withhold ? 1 : 0;
   a.packed = packed;
   a.E = E;
   a.H = H;

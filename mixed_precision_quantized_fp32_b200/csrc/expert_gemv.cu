@@ -87,6 +87,8 @@ struct GemvArgs {
   int32_t* status;
   unsigned long long* trace;  // diagnostics: clock64 stamps of CTA 0 (or null)
   StageLayout st;
+  long long wait;         // budget of the pipeline waits, clock cycles
+  int withhold;           // test hook: the TMA warp issues no loads (the waits run out)
 };
 
 // Stamp event `ev` of index `i` (CTA 0 only, first MOE_TRACE_STAGES indices).
@@ -274,10 +276,10 @@ template <int NMAT, int NT8, int F0, int F1>
 __device__ __forceinline__ void consume_tiles(const StageLayout& L, uint8_t* smem, uint64_t* full, uint64_t* empty,
                                               volatile int* abort_flag, int ntiles, int& stage, uint32_t& phase,
                                               bool& ok, float (&acc)[NMAT][2][NT8][4], unsigned long long* tr,
-                                              int& gtile) {
+                                              int& gtile, long long wait) {
   const int s = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
   for (int kt = 0; kt < ntiles; ++kt) {
-    if (kt > 0 && ok && !__all_sync(0xffffffffu, ptx::mbar_wait(&full[stage], phase, abort_flag, kGemvWait)))
+    if (kt > 0 && ok && !__all_sync(0xffffffffu, ptx::mbar_wait(&full[stage], phase, abort_flag, wait)))
       ok = false;
     if (threadIdx.x == 0) gtrace(tr, 2, gtile);
     if (ok) {
@@ -308,13 +310,13 @@ template <int NMAT, int NT8, int F0>
 __device__ __forceinline__ void consume_f1(int f1, const StageLayout& L, uint8_t* smem, uint64_t* full,
                                            uint64_t* empty, volatile int* abort_flag, int ntiles, int& stage,
                                            uint32_t& phase, bool& ok, float (&acc)[NMAT][2][NT8][4],
-                                           unsigned long long* tr, int& gtile) {
+                                           unsigned long long* tr, int& gtile, long long wait) {
   if (NMAT == 1 || F0 == MOE_FMT_NVFP4)
-    return consume_tiles<NMAT, NT8, F0, F0>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile);
+    return consume_tiles<NMAT, NT8, F0, F0>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile, wait);
   switch (f1) {
-    case MOE_FMT_INT2: return consume_tiles<NMAT, NT8, F0, MOE_FMT_INT2>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile);
-    case MOE_FMT_INT3: return consume_tiles<NMAT, NT8, F0, MOE_FMT_INT3>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile);
-    default: return consume_tiles<NMAT, NT8, F0, MOE_FMT_INT4>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile);
+    case MOE_FMT_INT2: return consume_tiles<NMAT, NT8, F0, MOE_FMT_INT2>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile, wait);
+    case MOE_FMT_INT3: return consume_tiles<NMAT, NT8, F0, MOE_FMT_INT3>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile, wait);
+    default: return consume_tiles<NMAT, NT8, F0, MOE_FMT_INT4>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile, wait);
   }
 }
 
@@ -469,7 +471,7 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
       }
       const int ntiles = done ? 1 : cur.d.ntiles;
       for (int kt = 0; kt < ntiles; ++kt) {
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kGemvWait))) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&empty[stage], phase ^ 1u, abort_flag, a.wait))) {
           ok = false;
           break;
         }
@@ -479,7 +481,7 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
           if (kt == 0) slot[stage] = cur.d;
           if (done) {
             ptx::mbar_arrive(&full[stage]);
-          } else {
+          } else if (!a.withhold) {
             ptx::mbar_arrive_expect_tx(&full[stage], cur.bytes);
             const int k = cur.kt0 + kt;
 #pragma unroll
@@ -497,10 +499,10 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
         }
         ++gtile;
         __syncwarp();
-        if (!done) {
+        if (!done && !a.withhold) {
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-        } else {
+        } else if (done) {
           armed &= ~(1u << stage);  // released by the consumers: its last copy has landed
         }
         if (++stage == SL.stages) {
@@ -527,7 +529,7 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
     uint32_t phase = 0;
     while (true) {
       // first stage of the next item (or the end marker); all consumer warps agree
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&full[stage], phase, abort_flag, kGemvWait))) *abort_flag = 1;
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&full[stage], phase, abort_flag, a.wait))) *abort_flag = 1;
       consumer_sync();
       if (*abort_flag) {
         ok = false;
@@ -552,10 +554,10 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc[m][t][nt][j] = 0.0f;
       switch (fm[0]) {
-        case MOE_FMT_INT2: consume_f1<NMAT, NT8, MOE_FMT_INT2>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile); break;
-        case MOE_FMT_INT3: consume_f1<NMAT, NT8, MOE_FMT_INT3>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile); break;
-        case MOE_FMT_INT4: consume_f1<NMAT, NT8, MOE_FMT_INT4>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile); break;
-        default: consume_f1<NMAT, NT8, MOE_FMT_NVFP4>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile); break;
+        case MOE_FMT_INT2: consume_f1<NMAT, NT8, MOE_FMT_INT2>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile, a.wait); break;
+        case MOE_FMT_INT3: consume_f1<NMAT, NT8, MOE_FMT_INT3>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile, a.wait); break;
+        case MOE_FMT_INT4: consume_f1<NMAT, NT8, MOE_FMT_INT4>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile, a.wait); break;
+        default: consume_f1<NMAT, NT8, MOE_FMT_NVFP4>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile, a.wait); break;
       }
       // lane outputs: weight row nl = 32s + 4g + 2t + (j >> 1), token row nt*8 + 2c + (j & 1)
       if (ok && a.P == 1) {
@@ -784,9 +786,12 @@ int gemv_split(long long R, int E, int N, int K, int nmat) {
 
 cudaError_t launch_expert_gemv(const uint8_t* packed, uint64_t packed_bytes, const uint8_t* fmt_host, int E, int H,
                                int F, int R, int k, bool fp4, bool gateup, int max_chunks, int chunk_rows,
-                               const Workspace& ws, int32_t* status, uint64_t* trace, cudaStream_t stream) {
+                               const Workspace& ws, int32_t* status, uint64_t* trace, GemmHooks hooks,
+                               cudaStream_t stream) {
   GemvArgs g{};
   g.trace = reinterpret_cast<unsigned long long*>(trace);
+  g.wait = hooks.wait_cycles ? (long long)hooks.wait_cycles : kGemvWait;
+  g.withhold = hooks.withhold ? 1 : 0;
   g.packed = packed;
   g.E = E;
   g.H = H;

@@ -24,9 +24,15 @@ cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4,
 cudaError_t launch_act_quant_h(int R, int F, const Workspace& ws, uint8_t* dbg_hq, float* dbg_sh,
                                cudaStream_t stream);
 
+// Test hooks of the expert GEMMs (moe_debug.test_withhold / wait_cycles).
+struct GemmHooks {
+  uint32_t withhold;     // nonzero: the copy warps issue no loads
+  uint32_t wait_cycles;  // pipeline wait budget, 0: default
+};
+
 cudaError_t launch_expert_gemm_tc(const uint8_t* packed, const uint8_t* fmt_host, int E, int H, int F, int T, int k,
                                   bool fp4, bool gateup, const Workspace& ws, int32_t* status, uint64_t* trace,
-                                  cudaStream_t stream);
+                                  GemmHooks hooks, cudaStream_t stream);
 
 // K parts of the decode GEMV for R expert rows on an N x K projection (nmat
 // matrices); the workspace holds P*R*N*nmat fp32 partials when P > 1.
@@ -34,7 +40,8 @@ int gemv_split(long long R, int E, int N, int K, int nmat);
 
 cudaError_t launch_expert_gemv(const uint8_t* packed, uint64_t packed_bytes, const uint8_t* fmt_host, int E, int H,
                                int F, int R, int k, bool fp4, bool gateup, int max_chunks, int chunk_rows,
-                               const Workspace& ws, int32_t* status, uint64_t* trace, cudaStream_t stream);
+                               const Workspace& ws, int32_t* status, uint64_t* trace, GemmHooks hooks,
+                               cudaStream_t stream);
 
 cudaError_t launch_combine(int T, int k, int H, const Workspace& ws, __nv_bfloat16* y, cudaStream_t stream);
 

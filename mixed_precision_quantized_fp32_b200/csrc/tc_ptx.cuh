@@ -38,6 +38,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Wait (bounded by `limit` cycles only) for async work that is still in flight at
+// exit: copies landing in shared memory, MMAs reading it.  Ignores the abort flag,
+// which is exactly when such work may be outstanding.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, long long limit) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > limit) return false;
+  return true;
+}
+
 // Bounded wait for the phase of parity `parity` to complete.  Gives up after
 // `limit` clock cycles, or at once when *abort is set; returns false then.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,

@@ -24,6 +24,7 @@ if not torch.cuda.is_available():
     pytest.skip("no CUDA device", allow_module_level=True)
 
 import mixed_precision_quantized_fp32_b200 as moe  # noqa: E402
+from mixed_precision_quantized_fp32_b200 import _lib  # noqa: E402
 
 
 def custom(name, T, H, F, E, k, fmt, bias=None):
@@ -194,6 +195,56 @@ def test_forward_cta_pairs_ragged_chunks():
     # (rounded up to 16) splits over the two CTAs at N/2 rows, well short of a full 128-row half.
     L = custom("pairs", 300, 512, 256, 12, 2, [[3, 2, 4], [4, 4, 4], [2, 2, 2], [4, 3, 2]] * 3)
     check_layer(L, 300)
+
+
+def _sweep_case(i):
+    """Seeded random shape: H, F in 128*{1..8}, E in {1..16}, k in {1..min(E, 8)}, T in {1..300};
+    every fourth case NVFP4, the rest a random integer width per expert and projection.  Cases
+    i % 5 == 2 push two experts' router bias to -1e4 (experts with no tokens), cases i % 5 == 4
+    push one expert's bias to +1e4 (every token picks it)."""
+    rng = np.random.default_rng(7000 + i)
+    H, F = 128 * int(rng.integers(1, 9)), 128 * int(rng.integers(1, 9))
+    E = int(rng.integers(1, 17))
+    k = int(rng.integers(1, min(E, 8) + 1))
+    T = int(rng.integers(1, 301))
+    fmt = [[16, 16, 16]] * E if i % 4 == 3 else rng.choice([2, 3, 4], size=(E, 3)).tolist()
+    bias = None
+    if i % 5 == 2 and E - 2 >= k:
+        bias = np.zeros(E, np.float32)
+        bias[rng.choice(E, 2, replace=False)] = -1e4
+    elif i % 5 == 4:
+        bias = np.zeros(E, np.float32)
+        bias[int(rng.integers(0, E))] = 1e4
+    tokens = np.sort(rng.choice(T, min(T, 48), replace=False))
+    return custom(f"sweep{i}", T, H, F, E, k, fmt), T, bias, tokens
+
+
+@pytest.mark.parametrize("i", range(16))
+def test_forward_random_shape_sweep(i):
+    L, T, bias, tokens = _sweep_case(i)
+    r = check_layer(L, T, tokens=tokens, bias=bias)
+    if bias is not None and bias.min() < 0:
+        assert np.all(r["counts"][bias < 0] == 0)      # the pushed-down experts got no rows
+    if bias is not None and bias.max() > 0:
+        assert r["counts"][int(np.argmax(bias))] == T  # every token chose the pushed-up expert
+
+
+@pytest.mark.parametrize("T", [8, 600])
+def test_bounded_wait_timeout_keeps_context_usable(T):
+    # Test hook: the expert GEMMs' copy warps withhold every load and the pipeline waits get a
+    # budget of 200k cycles (~0.1 ms).  The consumers give up, every role leaves its loop, the
+    # call reports MOE_ERR_TIMEOUT in the status word, and an ordinary call on the same context
+    # afterwards is still exact.  T=8 runs the decode GEMV, T=600 the tcgen05 GEMMs on CTA pairs.
+    L = custom("timeout", T, 512, 256, 4, 2, [[3, 2, 4], [4, 4, 4], [2, 2, 2], [4, 3, 2]])
+    layer = hp.gpu_pack(L)
+    x = W.device_x(T, L.H)
+    Wr, b = W.device_router(L)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    moe.moe_layer_forward(x, Wr, b, layer, L.k,
+                          debug={"status": st, "test_withhold": 1, "wait_cycles": 200_000})
+    torch.cuda.synchronize()
+    assert _lib.STATUS[int(st.item())] == "MOE_ERR_TIMEOUT"
+    check_layer(L, T)
 
 
 @pytest.mark.parametrize("T", [9, 300])
