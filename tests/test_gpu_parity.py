@@ -49,8 +49,14 @@ def run_gpu(L, layer, T, x=None, Wr=None, b=None, k=None):
                    sx=torch.empty(T, dtype=torch.float32, device="cuda"),
                    hq=torch.empty(R * L.F, dtype=torch.uint8, device="cuda"),
                    sh=torch.empty(R, dtype=torch.float32, device="cuda"))
-    y = moe.moe_layer_forward(x, Wr, b, layer, k, debug=dbg)
+    # y inside a guard band: 4 KiB of a sentinel (exact in bf16) on each side must survive the call
+    G, SENTINEL = 2048, -12288.0
+    buf = torch.full((T * L.H + 2 * G,), SENTINEL, dtype=torch.bfloat16, device="cuda")
+    y = buf[G:G + T * L.H].view(T, L.H)
+    moe.moe_layer_forward(x, Wr, b, layer, k, y=y, debug=dbg)
     torch.cuda.synchronize()
+    guard = torch.cat([buf[:G], buf[G + T * L.H:]])
+    assert bool((guard == SENTINEL).all()), "output guard band overwritten"
     out = {n: t.cpu().numpy() for n, t in dbg.items()}
     out["y"] = y
     assert out["status"][0] == 0
