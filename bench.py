@@ -16,6 +16,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -56,11 +57,19 @@ def peaks():
 TRAFFIC_SOURCES = ("expert_gemm_tc.cu", "tc_ptx.cuh", "moe_common.cuh")
 
 
+def _code_only(src: str) -> str:
+    """C/C++ source without comments and with whitespace runs collapsed."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return re.sub(r"\s+", " ", src).strip()
+
+
 def csrc_hash() -> str:
-    """Hash of the sources that define the dominant kernel (the tcgen05 expert GEMM)."""
+    """Hash of the code (comments and layout ignored) of the sources that define the
+    dominant kernel (the tcgen05 expert GEMM)."""
     h = hashlib.sha256()
     for fn in TRAFFIC_SOURCES:
-        h.update(open(os.path.join(CSRC, fn), "rb").read())
+        h.update(_code_only(open(os.path.join(CSRC, fn)).read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -6,21 +6,30 @@
 // sec. 2.3 / 3.5: experts stored as independently quantized 128-column blocks
 // that a custom kernel unpacks) with the activation fused into the epilogue
 // (its sec. 3.6, "fused linear + activation"), built for sm_100a:
-//   * one persistent CTA per SM walks (token chunk, 128-row weight tile) work
-//     items; chunk = up to 256 consecutive expert-sorted rows of one expert;
+//   * persistent clusters of two CTAs (one CTA per SM) walk (token chunk, weight
+//     tiles) work items; chunk = up to 256 consecutive expert-sorted rows of one
+//     expert; each CTA owns 128-row weight tiles (gate + up, or two down tiles);
 //   * warp 16 (one lane) streams each 64-input stage (two quantization groups):
-//     the activation tile with a 2D TMA load (128-byte swizzle) and the packed
-//     codes + scales of the weight tile with 1D bulk copies (never multicast);
+//     this CTA's half of the chunk's token rows with a 2D TMA load (128-byte
+//     swizzle) and the packed codes + scales of its weight tiles with 1D bulk
+//     copies (never multicast); the ring is as deep as the widest code format
+//     of the launch allows;
 //   * warps 0-15 turn codes into fp16 operands (exponent-bias unpack: a code u
 //     OR'ed into the mantissa of 1024.0 gives 1024+u exactly; one subtract
 //     and one multiply by the group scale) written straight into the swizzled
-//     K-major layout the tensor core reads;
-//   * warp 17 (one lane) issues tcgen05.mma M=128 (weight rows) x N<=256 (token
-//     rows) x K=16 and commits to mbarriers;
-//   * warps 0-15 then drain TMEM (tcgen05.ld) into the SwiGLU / scale epilogue.
-// Every mbarrier wait is bounded; a wait that gives up raises an abort flag so
-// every role leaves its loop, writes MOE_ERR_TIMEOUT to the status word and
-// the CTA frees its TMEM before returning.
+//     K-major layout the tensor core reads, then arrive on the even CTA's
+//     barrier;
+//   * warp 17 of the even CTA (one lane) issues tcgen05.mma.cta_group::2
+//     M=256 (128 weight rows from each CTA) x N<=256 (token rows, half from
+//     each CTA) x K=16 and commits to both CTAs' mbarriers;
+//   * warps 0-15 then drain their own TMEM (tcgen05.ld) into the SwiGLU / scale
+//     epilogue.
+// Shapes whose weight tiles do not pair run the same kernel on single CTAs
+// (cta_group::1, M=128, the whole token chunk per CTA).
+// Every mbarrier wait is bounded; a wait that gives up raises the abort flags
+// of both CTAs so every role leaves its loop and MOE_ERR_TIMEOUT goes to the
+// status word.  Copies and MMAs still in flight are waited for, and the pair
+// meets at a cluster barrier, before TMEM is freed and the CTAs return.
 #include <algorithm>
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
