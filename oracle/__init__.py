@@ -23,7 +23,7 @@ import numpy as np
 
 from . import build as _build
 
-FMT_INT2, FMT_INT3, FMT_INT4, FMT_NVFP4 = 2, 3, 4, 16
+FMT_INT1, FMT_INT2, FMT_INT3, FMT_INT4, FMT_NVFP4 = 1, 2, 3, 4, 16
 HDR_BYTES = 16384
 
 _lib = None

@@ -26,6 +26,10 @@
  * Readings taken where the pages are silent (each also stated at its function):
  *  - integer codes are symmetric: q in [-qmax, qmax], qmax = 2^(b-1)-1, the
  *    most negative code of [G] sec. 3.3 is left unused;
+ *  - the sub-2-bit cold tier ([X], closing section: cold experts below 2 bits,
+ *    precision falling with hotness) is a 1-bit sign code: q = +1 for w >= 0,
+ *    else -1, with the group scale s = fp16_rne(sum|w| / 32) (fp32 sum in
+ *    input order), the least-squares scale of a sign quantizer;
  *  - the scale of a group of 32 consecutive inputs of one output row is the
  *    fp16 round-to-nearest-even of the fp32 quotient amax/qmax (saturated to
  *    the largest finite fp16), and codes are taken against the rounded scale;
@@ -144,15 +148,20 @@ ORC_EXPORT double orc_e2m1_to_f64(uint8_t c) {
 /* ------------------------------------------------------------------------- */
 /* Weight formats.                                                           */
 /* ------------------------------------------------------------------------- */
-enum { ORC_INT2 = 2, ORC_INT3 = 3, ORC_INT4 = 4, ORC_NVFP4 = 16 };
+enum { ORC_INT1 = 1, ORC_INT2 = 2, ORC_INT3 = 3, ORC_INT4 = 4, ORC_NVFP4 = 16 };
 
-static int fmt_ok(int f) { return f == ORC_INT2 || f == ORC_INT3 || f == ORC_INT4 || f == ORC_NVFP4; }
+static int fmt_ok(int f) {
+  return f == ORC_INT1 || f == ORC_INT2 || f == ORC_INT3 || f == ORC_INT4 || f == ORC_NVFP4;
+}
 
 /* Integer group quantization of one row-major [N x K] fp32 matrix ([G] 3.3,
    [A] 4.2 with group 32).  Per (row n, group g of 32 consecutive k):
      amax = max |w|;  s = fp16_rne(amax / qmax) (fp32 division; saturated to
      65504);  q = clamp(rint(w / float(s)), -qmax, qmax) with fp32 division and
      round-half-even; s == 0 gives all-zero codes.
+   bits = 1 (sign code, [X] closing section): s = fp16_rne(sum|w| / 32) (fp32
+     sum in input order; saturated to 65504), q = +1 if w >= 0 else -1.  This s
+     minimizes sum (w - s*q)^2 over s for the signs q.
    q[N*K] are the signed codes, s16[N*(K/32)] the fp16 scale bit patterns. */
 ORC_EXPORT void orc_quant_int(const float* W, int N, int K, int bits, int8_t* q, uint16_t* s16) {
   const int qmax = (1 << (bits - 1)) - 1;
@@ -161,6 +170,15 @@ ORC_EXPORT void orc_quant_int(const float* W, int N, int K, int bits, int8_t* q,
   for (int n = 0; n < N; ++n) {
     for (int g = 0; g < G; ++g) {
       const float* w = W + (size_t)n * K + (size_t)g * 32;
+      if (bits == 1) {
+        float sum = 0.0f;
+        for (int i = 0; i < 32; ++i) sum += fabsf(w[i]);
+        uint16_t sb = orc_f64_to_f16((double)(sum / 32.0f));
+        if ((sb & 0x7FFFu) == 0x7C00u) sb = 0x7BFFu;
+        s16[(size_t)n * G + g] = sb;
+        for (int i = 0; i < 32; ++i) q[(size_t)n * K + (size_t)g * 32 + i] = (int8_t)(w[i] >= 0.0f ? 1 : -1);
+        continue;
+      }
       float amax = 0.0f;
       for (int i = 0; i < 32; ++i) {
         float a = fabsf(w[i]);
@@ -228,12 +246,15 @@ ORC_EXPORT void orc_quant_nvfp4(const float* W, int N, int K, uint8_t* v, uint8_
 /* concatenated).  Reading: tiles of 128 output rows x 128 inputs, tile order */
 /* n-block major, k-block minor.  Inside a tile, 32-bit little-endian words   */
 /* in the order [kg 0..3][word 0..b-1][n 0..127], where kg is the group of 32 */
-/* inputs inside the tile and b the word count of a group (2, 3, 4; NVFP4 4).*/
-/* Stored code u = q + 2^(b-1) (offset binary); NVFP4 stores the e2m1 code.   */
+/* inputs inside the tile and b the word count of a group (1, 2, 3, 4; NVFP4 */
+/* 4).  Stored code u = q + 2^(b-1) (offset binary); b = 1: u = (q + 1) / 2  */
+/* (the sign bit, 1 for q = +1); NVFP4 stores the e2m1 code.                  */
 /* Inside a word, the two codes of each consecutive pair (2j, 2j+1) sit 16    */
 /* bits apart (code 2j in the low half-word, code 2j+1 in the high one):      */
 /*   b = 4: codes 8w..8w+7 in word w; code 8w+2j at bits 4j..4j+3, code      */
 /*          8w+2j+1 at bits 16+4j..16+4j+3 (j = 0..3);                       */
+/*   b = 1: codes 0..31 in word 0; code 2j at bit j, code 2j+1 at bit 16+j    */
+/*          (j = 0..15);                                                      */
 /*   b = 2: codes 16w..16w+15 in word w; code 16w+2j at bits 2j..2j+1, code  */
 /*          16w+2j+1 at bits 16+2j..17+2j (j = 0..7);                        */
 /*   b = 3: words 0-1 hold the low two bits of u exactly as b = 2; word 2     */
@@ -271,6 +292,8 @@ static void put_code(uint32_t* words, int n, int k, int K, int fmt, uint32_t u) 
     words[word_index(n, k, K, 4, i / 8)] |= (u & 15u) << pair_shift(i, 4, 8);
   } else if (fmt == ORC_INT2) {
     words[word_index(n, k, K, 2, i / 16)] |= (u & 3u) << pair_shift(i, 2, 16);
+  } else if (fmt == ORC_INT1) {
+    words[word_index(n, k, K, 1, 0)] |= (u & 1u) << pair_shift(i, 1, 32);
   } else { /* INT3 */
     words[word_index(n, k, K, 3, i / 16)] |= (u & 3u) << pair_shift(i, 2, 16);
     words[word_index(n, k, K, 3, 2)] |= ((u >> 2) & 1u) << int3_high_shift(i);
@@ -282,6 +305,7 @@ static uint32_t get_code(const uint32_t* words, int n, int k, int K, int fmt) {
   if (fmt == ORC_NVFP4) return (words[word_index(n, k, K, 4, i / 8)] >> (4 * (i % 8))) & 15u;
   if (fmt == ORC_INT4) return (words[word_index(n, k, K, 4, i / 8)] >> pair_shift(i, 4, 8)) & 15u;
   if (fmt == ORC_INT2) return (words[word_index(n, k, K, 2, i / 16)] >> pair_shift(i, 2, 16)) & 3u;
+  if (fmt == ORC_INT1) return (words[word_index(n, k, K, 1, 0)] >> pair_shift(i, 1, 32)) & 1u;
   uint32_t lo = (words[word_index(n, k, K, 3, i / 16)] >> pair_shift(i, 2, 16)) & 3u;
   uint32_t hi = (words[word_index(n, k, K, 3, 2)] >> int3_high_shift(i)) & 1u;
   return lo | (hi << 2);
@@ -308,7 +332,8 @@ ORC_EXPORT void orc_pack_int(const int8_t* q, const uint16_t* s16, int N, int K,
 #pragma omp parallel for schedule(static)
   for (int n = 0; n < N; ++n)
     for (int k = 0; k < K; ++k)
-      put_code(words, n, k, K, bits, (uint32_t)(q[(size_t)n * K + k] + off));
+      put_code(words, n, k, K, bits,
+               bits == 1 ? (uint32_t)((q[(size_t)n * K + k] + 1) >> 1) : (uint32_t)(q[(size_t)n * K + k] + off));
   uint16_t* sc = (uint16_t*)scales;
   for (int n = 0; n < N; ++n)
     for (int g = 0; g < K / 32; ++g) sc[scale_index(n, g, K / 32)] = s16[(size_t)n * (K / 32) + g];
@@ -319,7 +344,10 @@ ORC_EXPORT void orc_unpack_int(const uint8_t* codes, const uint8_t* scales, int 
   const uint32_t* words = (const uint32_t*)codes;
   const int off = 1 << (bits - 1);
   for (int n = 0; n < N; ++n)
-    for (int k = 0; k < K; ++k) q[(size_t)n * K + k] = (int8_t)((int)get_code(words, n, k, K, bits) - off);
+    for (int k = 0; k < K; ++k) {
+      const int u = (int)get_code(words, n, k, K, bits);
+      q[(size_t)n * K + k] = (int8_t)(bits == 1 ? 2 * u - 1 : u - off);
+    }
   const uint16_t* sc = (const uint16_t*)scales;
   for (int n = 0; n < N; ++n)
     for (int g = 0; g < K / 32; ++g) s16[(size_t)n * (K / 32) + g] = sc[scale_index(n, g, K / 32)];
@@ -361,7 +389,8 @@ ORC_EXPORT void orc_decode_row(const uint8_t* codes, const uint8_t* scales, int 
     const uint16_t* sc = (const uint16_t*)scales;
     const int off = 1 << (fmt - 1);
     for (int k = 0; k < K; ++k) {
-      int q = (int)get_code(words, n, k, K, fmt) - off;
+      const int u = (int)get_code(words, n, k, K, fmt);
+      const int q = fmt == ORC_INT1 ? 2 * u - 1 : u - off;
       w[k] = orc_f16_to_f64(sc[scale_index(n, k / 32, K / 32)]) * (double)q;
     }
   }

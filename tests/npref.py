@@ -17,6 +17,14 @@ def quant_int(W, bits):
     qmax = (1 << (bits - 1)) - 1
     N, K = W.shape
     G = W.reshape(N, K // 32, 32)
+    if bits == 1:  # sign code, scale = fp16(sum|w| / 32) with the fp32 sum taken in input order
+        acc = np.zeros((N, K // 32), np.float32)
+        for i in range(32):
+            acc = (acc + np.abs(G[:, :, i])).astype(np.float32)
+        with np.errstate(over="ignore"):
+            s16 = (acc / np.float32(32)).astype(np.float32).astype(np.float16)
+        s16[np.isinf(s16)] = np.float16(65504.0)
+        return np.where(G >= 0, 1, -1).reshape(N, K).astype(np.int8), s16.view(np.uint16)
     amax = np.abs(G).max(axis=2)
     ratio = (amax / np.float32(qmax)).astype(np.float32)
     with np.errstate(over="ignore"):

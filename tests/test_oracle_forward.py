@@ -82,9 +82,12 @@ def test_act_quant_against_torch(orc):
     assert np.all(big == 448.0)
 
 
-@pytest.mark.parametrize("fmt_kind", ["int4", "mixed", "nvfp4"])
+@pytest.mark.parametrize("fmt_kind", ["int4", "mixed", "graded", "nvfp4"])
 def test_forward_against_dense_restatement(orc, fmt_kind):
-    if fmt_kind == "nvfp4":
+    if fmt_kind == "graded":  # precision falling with hotness: 4-, 2- and 1-bit experts
+        T, H, F, E, k = 12, 256, 384, 6, 2
+        fmt = np.array([[4, 4, 4], [2, 2, 2], [1, 1, 1], [4, 2, 1], [1, 2, 4], [2, 1, 2]], np.uint8)
+    elif fmt_kind == "nvfp4":
         T, H, F, E, k = 8, 256, 256, 16, 6
         fmt = np.full((E, 3), 16, np.uint8)
     elif fmt_kind == "mixed":
@@ -152,6 +155,21 @@ def test_k1_is_single_expert(orc):
     y = orc.moe_forward(layer, x, np.zeros((E, H), np.float32), b, 1)
     o = orc.down(layer, 1, orc.gateup(layer, 1, npref.bf16_to_f64(x)))
     np.testing.assert_array_equal(y, np.array([[orc.bf16_bits(v) for v in row] for row in o], np.uint16))
+
+
+def test_constant_weights_closed_form_sign_code(orc):
+    # every weight = c (few significant bits, so the fp32 sum of 32 of them is exact):
+    # s = fp16(32c/32) = c and every code is +1, so g_n = u_n = c*sum_k x_k.
+    T, H, F, E = 4, 256, 128, 1
+    c = np.float32(0.025390625)  # 1.625 * 2^-6
+    W = np.full((E, 3, H * F), c, np.float32)
+    layer = orc.pack_layer(W, 0, E, H, F, np.full((E, 3), 1, np.uint8))
+    x, _ = _inputs(T, H, E, seed=3)
+    a = npref.bf16_to_f64(x)
+    g = float(c) * a.sum(1)
+    h = orc.gateup(layer, 0, a)
+    want = g / (1 + np.exp(-g)) * g
+    np.testing.assert_allclose(h, np.repeat(want[:, None], F, 1), rtol=1e-12)
 
 
 def test_constant_weights_closed_form(orc):

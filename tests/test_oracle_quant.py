@@ -1,6 +1,6 @@
 """Pins for the oracle's weight quantization, packing and layer layout.
 
-  * hand-worked groups (tests/golden/int_group_examples.json): scale bits,
+  * hand-worked groups (tests/golden/int_group_examples.json, 1- to 4-bit): scale bits,
     codes (round-half-even ties) and packed words;
   * a hand-worked NVFP4 block (tests/golden/nvfp4_group_example.json): tensor
     scale, e4m3 block scale, e2m1 codes with ties to even, packed word and
@@ -71,15 +71,17 @@ def test_layout_positions_hand_computed(orc):
     # inside the tile, position 8 inside the group (an even code: 4-bit nibble 0 of
     # word 1; 2-bit field 4 of word 0; 3-bit field 4 of word 0 and, pair m=4 being
     # c=1, j=0, bit 8*0 + 1 + 0 = 1 of word 2).
+    # 1-bit: code 8 of the group at bit 0*16 + 8/2 = 4 of word (((1*2+1)*4+2)*1)*128+2 = 1794.
     N = K = 256
     cases = {
-        # bits: (code, [(byte offset, expected word), ...], base word)
+        # bits: (code, [(byte offset, expected word), ...], base word); other codes 0 (1-bit: +1)
+        1: (-1, [(7176, 0xFFFFFFEF)], 0xFFFFFFFF),
         4: (5, [(29192, 0x8888888D)], 0x88888888),
         2: (-1, [(14344, 0xAAAAA9AA)], 0xAAAAAAAA),
         3: (-3, [(21512, 0x00000100), (22536, 0xFFFFFFFD)], None),
     }
     for bits, (code, checks, base) in cases.items():
-        q = np.zeros((N, K), np.int8)
+        q = np.full((N, K), 1 if bits == 1 else 0, np.int8)
         q[130, 200] = code
         s = np.zeros((N, K // 32), np.uint16)
         s[130, 6] = 0x1234
@@ -106,7 +108,7 @@ def test_layout_positions_hand_computed(orc):
 
 
 def test_quant_int_matches_numpy(orc):
-    for bits in (2, 3, 4):
+    for bits in (1, 2, 3, 4):
         W = gen.normal_f32(0, 99 + bits, 0, 256 * 512, 0.02).reshape(256, 512)
         W[3, 64:96] = 0.0  # an all-zero group
         W[5, :32] *= np.float32(1e-6)  # tiny scales (fp16 subnormal)
@@ -114,13 +116,33 @@ def test_quant_int_matches_numpy(orc):
         qn, sn = npref.quant_int(W, bits)
         np.testing.assert_array_equal(s, sn)
         np.testing.assert_array_equal(q, qn)
+        if bits == 1:
+            assert set(np.unique(q)) <= {-1, 1}
+            assert np.all(q[3, 64:96] == 1) and s[3, 2] == 0
+            continue
         qmax = (1 << (bits - 1)) - 1
         assert q.min() >= -qmax and q.max() <= qmax
         assert np.all(q[3, 64:96] == 0) and s[3, 2] == 0
 
 
+def test_sign_code_scale_is_least_squares(orc):
+    # for a sign code q, sum (w - s q)^2 = sum w^2 - 2 s sum|w| + 32 s^2 is minimized at
+    # s = mean|w|, so the fp16 value nearest to it beats both fp16 neighbours
+    W = gen.normal_f32(0, 321, 0, 64 * 256, 0.02).reshape(64, 256)
+    q, s = orc.quant_int(W, 1)
+    G = W.reshape(64, 8, 32).astype(np.float64)
+    Q = q.reshape(64, 8, 32).astype(np.float64)
+    assert np.all(Q == np.where(G >= 0, 1.0, -1.0))
+    s16 = s.view(np.float16)
+    def err(sv):
+        return ((G - sv.astype(np.float64)[:, :, None] * Q) ** 2).sum(axis=2)
+    e0 = err(s16)
+    assert np.all(e0 <= err(np.nextafter(s16, np.float16(np.inf))))
+    assert np.all(e0 <= err(np.nextafter(s16, np.float16(0))))
+
+
 def test_int_roundtrip_and_requant(orc):
-    for bits in (2, 3, 4):
+    for bits in (1, 2, 3, 4):
         W = gen.normal_f32(0, 200 + bits, 0, 384 * 256, 0.02).reshape(384, 256)
         q, s = orc.quant_int(W, bits)
         codes, scales = orc.pack_int(q, s, bits)
@@ -134,6 +156,8 @@ def test_int_roundtrip_and_requant(orc):
         np.testing.assert_array_equal(s, s3)
         # decode_row through the packed layout equals s*q
         np.testing.assert_array_equal(orc.decode_matrix(codes, scales, bits, 384, 256), Wd)
+        if bits == 1:  # the sign code has its own pin (least-squares scale)
+            continue
         # error bound for values that were not clamped
         qmax = (1 << (bits - 1)) - 1
         sf = np.repeat(s.view(np.float16).astype(np.float64), 32, axis=1)
