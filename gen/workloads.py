@@ -5,7 +5,10 @@ Input recipe (seed 0): x = bf16 of N(0,1) values (tensor id 1, element t*H+h);
 router weights fp32 N(0, 0.02) (id 2, element e*H+h); expert (e, p) weights
 fp32 N(0, 0.02) (id 16+3e+p, row-major N x K).  The hot/cold layer adds the
 calibrated router bias of tests/golden/hotcold_bias.json and puts its 64 hot
-experts at 4 bits, the other 192 at 2 bits.  No public dataset is involved.
+experts at 4 bits, the other 192 at 2 bits.  The graded layer is the same
+layer with precision falling with hotness: the 64 hot experts at 4 bits, the
+next 64 by router bias (ties to the lower index) at 2 bits, the last 128 at
+1 bit (sign code).  No public dataset is involved.
 
 This module only builds inputs; it holds none of the layer's arithmetic.
 """
@@ -53,6 +56,17 @@ def _hotcold() -> Layer:
                  {"hot_experts": d["hot_experts"], "top32_share": d["top32_share"], "gini": d["gini"]})
 
 
+def _graded() -> Layer:
+    L = _hotcold()
+    hot = set(L.notes["hot_experts"])
+    rest = sorted((e for e in range(L.E) if e not in hot), key=lambda e: (-float(L.bias[e]), e))
+    fmt = np.full((L.E, 3), 1, np.uint8)
+    fmt[sorted(hot)] = 4
+    fmt[rest[:64]] = 2
+    return Layer("graded", L.H, L.F, L.E, L.k, fmt, L.decode_T, L.prefill_T, L.bias,
+                 dict(L.notes, warm_experts=sorted(rest[:64])))
+
+
 def layer(name: str) -> Layer:
     if name == "tiny":
         return Layer("tiny", 256, 512, 8, 2, np.full((8, 3), 4, np.uint8), (16,), ())
@@ -61,6 +75,8 @@ def layer(name: str) -> Layer:
                      (1, 8, 64), (2048,))
     if name == "hotcold":
         return _hotcold()
+    if name == "graded":
+        return _graded()
     if name == "nvfp4":
         return Layer("nvfp4", 2048, 768, 256, 6, np.full((256, 3), 16, np.uint8), (16,), (8192,))
     if name == "large":
@@ -69,7 +85,7 @@ def layer(name: str) -> Layer:
     raise KeyError(name)
 
 
-NAMES = ("tiny", "mixtral", "hotcold", "nvfp4", "large")
+NAMES = ("tiny", "mixtral", "hotcold", "nvfp4", "large", "graded")
 
 
 # ------------------------------------------------------------------ host inputs

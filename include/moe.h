@@ -67,6 +67,8 @@ typedef enum {
 
 /* Weight formats, chosen per expert and per projection. */
 enum {
+  MOE_FMT_INT1 = 1,   /* sign codes {-1,+1},      fp16 scale per 32 inputs (mean |w|): the
+                         sub-2-bit cold tier of the expert-aware quantisation page */
   MOE_FMT_INT2 = 2,   /* symmetric codes {-1,0,1}, fp16 scale per 32 inputs */
   MOE_FMT_INT3 = 3,   /* symmetric codes [-3,3],   fp16 scale per 32 inputs */
   MOE_FMT_INT4 = 4,   /* symmetric codes [-7,7],   fp16 scale per 32 inputs */

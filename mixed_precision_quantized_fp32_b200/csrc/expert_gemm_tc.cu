@@ -165,7 +165,18 @@ __device__ __forceinline__ uint4 dequant_chunk(const uint32_t* __restrict__ code
     const uint32_t s = reinterpret_cast<const uint16_t*>(scales)[n];
     const uint32_t s2 = s | (s << 16);
     constexpr uint32_t kMagic = 0x64006400u;
-    if (FMT == MOE_FMT_INT4) {
+    if (FMT == MOE_FMT_INT1) {
+      // sign code, pair j of chunk c at bit 4c + j (and 16 above): 1024 + 2^j u after
+      // the OR; one FMA with 2^-j and -1024*2^-j gives u, a second with 2s and -s
+      // gives s*(2u - 1) = +-s in one rounding
+      constexpr uint32_t kMul1[4] = {0x3C003C00u, 0x38003800u, 0x34003400u, 0x30003000u};  // 2^-j
+      constexpr uint32_t kSub1[4] = {0xE400E400u, 0xE000E000u, 0xDC00DC00u, 0xD800D800u};  // -1024*2^-j
+      const uint32_t w = codes[n] >> (4 * c);
+      const uint32_t s2x2 = h2mul(s2, 0x40004000u), neg_s2 = s2 ^ 0x80008000u;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        v[j] = h2fma(h2fma((w & (0x00010001u << j)) | kMagic, kMul1[j], kSub1[j]), s2x2, neg_s2);
+    } else if (FMT == MOE_FMT_INT4) {
       const uint32_t w = codes[c * 128 + n], w8 = w >> 8;
       v[0] = h2mul(h2fma((w & 0x000F000Fu) | kMagic, 0x3C003C00u, 0xE408E408u), s2);   // u - 8
       v[1] = h2mul(h2fma((w & 0x00F000F0u) | kMagic, 0x2C002C00u, 0xD480D480u), s2);   // 16u / 16 + 64 - 72
@@ -272,12 +283,17 @@ __device__ __noinline__ bool dequant_item(const Ring R, long long wait, uint8_t*
   return true;
 }
 
-// Runtime format pair -> the matching dequant_item instantiation.
-template <int NMAT, bool CG2, int F0>
+// Runtime format pair -> the matching dequant_item instantiation.  I1: the launch
+// meets 1-bit matrices; their cases are compiled only into the I1 kernels, so the
+// kernels for layers without them keep their size and register allocation.
+template <int NMAT, bool CG2, bool I1, int F0>
 __device__ __forceinline__ bool dequant_item_f1(int f1, const Ring R, long long wait, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
                                                 volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
                                                 uint32_t& phase, int& gstage, unsigned long long* trace) {
   if (NMAT == 1) return dequant_item<NMAT, CG2, F0, F0>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+  if constexpr (I1) {
+    if (f1 == MOE_FMT_INT1) return dequant_item<NMAT, CG2, F0, MOE_FMT_INT1>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+  }
   switch (f1) {
     case MOE_FMT_INT2: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT2>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
     case MOE_FMT_INT3: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT3>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
@@ -285,19 +301,22 @@ __device__ __forceinline__ bool dequant_item_f1(int f1, const Ring R, long long 
     default: return dequant_item<NMAT, CG2, F0, MOE_FMT_NVFP4>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
   }
 }
-template <int NMAT, bool CG2>
+template <int NMAT, bool CG2, bool I1>
 __device__ __forceinline__ bool dequant_item_any(int f0, int f1, const Ring R, long long wait, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
                                                  volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
                                                  uint32_t& phase, int& gstage, unsigned long long* trace) {
+  if constexpr (I1) {
+    if (f0 == MOE_FMT_INT1) return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_INT1>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+  }
   switch (f0) {
-    case MOE_FMT_INT2: return dequant_item_f1<NMAT, CG2, MOE_FMT_INT2>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    case MOE_FMT_INT3: return dequant_item_f1<NMAT, CG2, MOE_FMT_INT3>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    case MOE_FMT_INT4: return dequant_item_f1<NMAT, CG2, MOE_FMT_INT4>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    default: return dequant_item_f1<NMAT, CG2, MOE_FMT_NVFP4>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT2: return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_INT2>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT3: return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_INT3>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT4: return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_INT4>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    default: return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_NVFP4>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
   }
 }
 
-template <int NMAT, bool CG2>
+template <int NMAT, bool CG2, bool I1>
 __global__ void __launch_bounds__(kTcThreads, 1)
     expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
   using C = TcCfg<NMAT, CG2>;
@@ -519,7 +538,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         fmt[m] = L.fmt[i];
         tsc[m] = fmt[m] == MOE_FMT_NVFP4 ? L.tscale[i] : 1.0f;
       }
-      if (!dequant_item_any<NMAT, CG2>(fmt[0], fmt[NMAT - 1], a.ring, a.wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage,
+      if (!dequant_item_any<NMAT, CG2, I1>(fmt[0], fmt[NMAT - 1], a.ring, a.wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage,
                                   phase, gstage, a.trace)) {
         ok = false;
         break;
@@ -625,7 +644,7 @@ int sm_count() {
   return n[dev];
 }
 
-template <int NMAT, bool CG2>
+template <int NMAT, bool CG2, bool I1>
 cudaError_t launch_tc(TcArgs a, int max_words, const void* act, int rows_total, cudaStream_t stream) {
   using C = TcCfg<NMAT, CG2>;
   a.ring = make_ring<NMAT, CG2>(max_words);
@@ -643,7 +662,7 @@ cudaError_t launch_tc(TcArgs a, int max_words, const void* act, int rows_total, 
           CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  auto kern = expert_gemm_tc_kernel<NMAT, CG2>;
+  auto kern = expert_gemm_tc_kernel<NMAT, CG2, I1>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   if (!CG2) {
@@ -677,10 +696,15 @@ cudaError_t launch_tc(TcArgs a, int max_words, const void* act, int rows_total, 
 cudaError_t launch_expert_gemm_tc(const uint8_t* packed, const uint8_t* fmt_host, int E, int H, int F, int T, int k,
                                   bool fp4, bool gateup, const Workspace& ws, int32_t* status, uint64_t* trace,
                                   GemmHooks hooks, cudaStream_t stream) {
-  // widest code format of the projections this launch reads (sizes the code slots)
+  // widest code format of the projections this launch reads (sizes the code slots),
+  // and whether any of them is the 1-bit code (selects the kernels that decode it)
   int max_words = 1;
+  bool any1 = false;
   for (int e = 0; e < E; ++e)
-    for (int p = gateup ? 0 : 2; p <= (gateup ? 1 : 2); ++p) max_words = std::max(max_words, fmt_words(fmt_host[e * 3 + p]));
+    for (int p = gateup ? 0 : 2; p <= (gateup ? 1 : 2); ++p) {
+      max_words = std::max(max_words, fmt_words(fmt_host[e * 3 + p]));
+      any1 |= fmt_host[e * 3 + p] == MOE_FMT_INT1;
+    }
   TcArgs a{};
   a.trace = gateup ? reinterpret_cast<unsigned long long*>(trace) : nullptr;
   a.wait = hooks.wait_cycles ? (long long)hooks.wait_cycles : kWaitLimit;
@@ -701,8 +725,11 @@ cudaError_t launch_expert_gemm_tc(const uint8_t* packed, const uint8_t* fmt_host
     a.proj = 0;
     a.row_scale = fp4 ? ws.sx : nullptr;
     a.out = ws.h;
-    if ((F / kTcBM) % 2 == 0) return launch_tc<2, true>(a, max_words, ws.xs, R, stream);  // weight tiles in pairs of CTAs
-    return launch_tc<2, false>(a, max_words, ws.xs, R, stream);
+    if ((F / kTcBM) % 2 == 0)  // weight tiles in pairs of CTAs
+      return any1 ? launch_tc<2, true, true>(a, max_words, ws.xs, R, stream)
+                  : launch_tc<2, true, false>(a, max_words, ws.xs, R, stream);
+    return any1 ? launch_tc<2, false, true>(a, max_words, ws.xs, R, stream)
+                : launch_tc<2, false, false>(a, max_words, ws.xs, R, stream);
   }
   a.N = H;
   a.K = F;
@@ -711,10 +738,14 @@ cudaError_t launch_expert_gemm_tc(const uint8_t* packed, const uint8_t* fmt_host
   a.out = ws.o;
   if ((H / kTcBM) % 2 == 0) {  // pairs of weight tiles share each activation tile
     a.pair = 1;
-    if ((H / kTcBM) % 4 == 0) return launch_tc<2, true>(a, max_words, fp4 ? ws.hb : ws.h, R, stream);
-    return launch_tc<2, false>(a, max_words, fp4 ? ws.hb : ws.h, R, stream);
+    if ((H / kTcBM) % 4 == 0)
+      return any1 ? launch_tc<2, true, true>(a, max_words, fp4 ? ws.hb : ws.h, R, stream)
+                  : launch_tc<2, true, false>(a, max_words, fp4 ? ws.hb : ws.h, R, stream);
+    return any1 ? launch_tc<2, false, true>(a, max_words, fp4 ? ws.hb : ws.h, R, stream)
+                : launch_tc<2, false, false>(a, max_words, fp4 ? ws.hb : ws.h, R, stream);
   }
-  return launch_tc<1, false>(a, max_words, fp4 ? ws.hb : ws.h, R, stream);
+  return any1 ? launch_tc<1, false, true>(a, max_words, fp4 ? ws.hb : ws.h, R, stream)
+              : launch_tc<1, false, false>(a, max_words, fp4 ? ws.hb : ws.h, R, stream);
 }
 
 }  // namespace moe

@@ -96,9 +96,9 @@ __device__ __forceinline__ void gtrace(unsigned long long* tr, int ev, int i) {
   if (tr && blockIdx.x == 0 && i < MOE_TRACE_STAGES) tr[ev * MOE_TRACE_STAGES + i] = (unsigned long long)clock64();
 }
 
-__device__ __forceinline__ const CUtensorMap* map_of(int wpg, const CUtensorMap* m2, const CUtensorMap* m3,
-                                                     const CUtensorMap* m4) {
-  return wpg == 2 ? m2 : wpg == 3 ? m3 : m4;
+__device__ __forceinline__ const CUtensorMap* map_of(int wpg, const CUtensorMap* m1, const CUtensorMap* m2,
+                                                     const CUtensorMap* m3, const CUtensorMap* m4) {
+  return wpg == 1 ? m1 : wpg == 2 ? m2 : wpg == 3 ? m3 : m4;
 }
 
 // ------------------------------------------------------------------ small PTX helpers
@@ -148,15 +148,21 @@ constexpr uint32_t h2c(uint32_t h) { return h | (h << 16); }
 
 // Activation multiplier 1/f_j (fp16x2) for pair j (j = 0..3) of a lane's eight
 // inputs, whose codes sit in a field of weight f_j: INT4 1, 16, 1, 16 (fields at
-// bits 0 and 4; pairs 2, 3 after >> 8); INT2 and INT3 4^j (fields at bits 2j).
+// bits 0 and 4; pairs 2, 3 after >> 8); INT2 and INT3 4^j (fields at bits 2j);
+// INT1 2^j (fields at bit j), times 2 for the sign code's q = 2u - 1.
 __host__ __device__ constexpr uint32_t act_mul(int fmt, int j) {
   return fmt == MOE_FMT_NVFP4 ? h2c(0x3C00u)
+         : fmt == MOE_FMT_INT1 ? (j == 0 ? h2c(0x4000u) : j == 1 ? h2c(0x3C00u) : j == 2 ? h2c(0x3800u) : h2c(0x3400u))
          : fmt == MOE_FMT_INT4 ? ((j & 1) ? h2c(0x2C00u) : h2c(0x3C00u))   // 1, 1/16
          : (j == 0 ? h2c(0x3C00u) : j == 1 ? h2c(0x3400u) : j == 2 ? h2c(0x2C00u) : h2c(0x2400u));  // 4^-j
 }
-// -offset * 2^-24: times the group sum of the activations, the MMA's C input.
+// -offset * 2^-24: times the group sum of the activations, the MMA's C input
+// (INT1: q = 2u - 1, so with the activations doubled the offset is 1).
 __host__ __device__ constexpr float offset_term(int fmt) {
-  return fmt == MOE_FMT_INT4 ? -8.0f / 16777216.0f : fmt == MOE_FMT_INT3 ? -4.0f / 16777216.0f : -2.0f / 16777216.0f;
+  return fmt == MOE_FMT_INT4 ? -8.0f / 16777216.0f
+         : fmt == MOE_FMT_INT3 ? -4.0f / 16777216.0f
+         : fmt == MOE_FMT_INT1 ? -1.0f / 16777216.0f
+                               : -2.0f / 16777216.0f;
 }
 
 // Address of the 16-byte chunk of rows 4g..4g+3 in word-row z of a code box
@@ -204,7 +210,17 @@ __device__ __forceinline__ void group_mma(const uint8_t* box, const uint8_t* sc,
     }
     return;
   }
-  if (FMT == MOE_FMT_INT4) {
+  if (FMT == MOE_FMT_INT1) {
+    // one word per row and group: the lane's pairs j at bits 4c + j (and 16 above)
+    const uint4 w = lds128(code_chunk(box, kg, y, g));
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t ws = wv[i] >> (4 * c);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) p[i][j] = ws & (0x00010001u << j);
+    }
+  } else if (FMT == MOE_FMT_INT4) {
     const uint4 w = lds128(code_chunk(box, 4 * kg + c, y, g));
     const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -248,7 +264,7 @@ __device__ __forceinline__ void group_mma(const uint8_t* box, const uint8_t* sc,
 #pragma unroll
   for (int nt = 0; nt < NT8; ++nt) {
     const uint4 xr = lds128(xs + nt * 2048);
-    const uint32_t b0 = xr.x, b1 = hmul2(xr.y, act_mul(FMT, 1));
+    const uint32_t b0 = FMT == MOE_FMT_INT1 ? hmul2(xr.x, act_mul(FMT, 0)) : xr.x, b1 = hmul2(xr.y, act_mul(FMT, 1));
     const uint32_t b2 = FMT == MOE_FMT_INT4 ? xr.z : hmul2(xr.z, act_mul(FMT, 2));
     const uint32_t b3 = hmul2(xr.w, act_mul(FMT, 3));
     const float d0 = offset_term(FMT) * ldsf(gs + nt * 128), d1 = offset_term(FMT) * ldsf(gs + nt * 128 + 16);
@@ -306,13 +322,20 @@ __device__ __forceinline__ void consume_tiles(const StageLayout& L, uint8_t* sme
   }
 }
 
-template <int NMAT, int NT8, int F0>
+// I1: the launch meets 1-bit matrices.  Their cases are compiled only into the
+// I1 instantiations, so kernels for layers without them keep their size and
+// register allocation.
+template <int NMAT, int NT8, int F0, bool I1>
 __device__ __forceinline__ void consume_f1(int f1, const StageLayout& L, uint8_t* smem, uint64_t* full,
                                            uint64_t* empty, volatile int* abort_flag, int ntiles, int& stage,
                                            uint32_t& phase, bool& ok, float (&acc)[NMAT][2][NT8][4],
                                            unsigned long long* tr, int& gtile, long long wait) {
   if (NMAT == 1 || F0 == MOE_FMT_NVFP4)
     return consume_tiles<NMAT, NT8, F0, F0>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile, wait);
+  if constexpr (I1) {
+    if (f1 == MOE_FMT_INT1)
+      return consume_tiles<NMAT, NT8, F0, MOE_FMT_INT1>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile, wait);
+  }
   switch (f1) {
     case MOE_FMT_INT2: return consume_tiles<NMAT, NT8, F0, MOE_FMT_INT2>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile, wait);
     case MOE_FMT_INT3: return consume_tiles<NMAT, NT8, F0, MOE_FMT_INT3>(L, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, tr, gtile, wait);
@@ -413,8 +436,9 @@ __device__ __forceinline__ float store_output(const GemvArgs& a, int r, int n, c
   return o;
 }
 
-template <int NMAT, int NT8>
-__global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) : 2) expert_gemv_kernel(const __grid_constant__ CUtensorMap tm_w2,
+template <int NMAT, int NT8, bool I1>
+__global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) : 2) expert_gemv_kernel(const __grid_constant__ CUtensorMap tm_w1,
+                                                                   const __grid_constant__ CUtensorMap tm_w2,
                                                                    const __grid_constant__ CUtensorMap tm_w3,
                                                                    const __grid_constant__ CUtensorMap tm_w4,
                                                                    const __grid_constant__ CUtensorMap tm_x,
@@ -438,6 +462,7 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
     ptx::fence_mbar_init();
   }
   if (warp == kProducer && lane == 0) {
+    ptx::prefetch_tmap(&tm_w1);
     ptx::prefetch_tmap(&tm_w2);
     ptx::prefetch_tmap(&tm_w3);
     ptx::prefetch_tmap(&tm_w4);
@@ -487,7 +512,7 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
               const int z = cur.z0[m] + k * 4 * cur.wpg[m];
-              const CUtensorMap* map = map_of(cur.wpg[m], &tm_w2, &tm_w3, &tm_w4);
+              const CUtensorMap* map = map_of(cur.wpg[m], &tm_w1, &tm_w2, &tm_w3, &tm_w4);
               tma_load_3d(sb + SL.code_off[m], map, 0, 0, z, &full[stage]);
               tma_load_3d(sb + SL.code_off[m] + SL.box[m], map, 0, 2, z, &full[stage]);
               ptx::bulk_load(sb + SL.scale_off[m], cur.sptr[m] + (size_t)k * 1024u, 1024u, &full[stage]);
@@ -553,11 +578,18 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
           for (int nt = 0; nt < NT8; ++nt)
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc[m][t][nt][j] = 0.0f;
-      switch (fm[0]) {
-        case MOE_FMT_INT2: consume_f1<NMAT, NT8, MOE_FMT_INT2>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile, a.wait); break;
-        case MOE_FMT_INT3: consume_f1<NMAT, NT8, MOE_FMT_INT3>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile, a.wait); break;
-        case MOE_FMT_INT4: consume_f1<NMAT, NT8, MOE_FMT_INT4>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile, a.wait); break;
-        default: consume_f1<NMAT, NT8, MOE_FMT_NVFP4>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile, a.wait); break;
+      bool first_1bit = false;
+      if constexpr (I1) {
+        if (fm[0] == MOE_FMT_INT1) {
+          consume_f1<NMAT, NT8, MOE_FMT_INT1, I1>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile, a.wait);
+          first_1bit = true;
+        }
+      }
+      if (!first_1bit) switch (fm[0]) {
+        case MOE_FMT_INT2: consume_f1<NMAT, NT8, MOE_FMT_INT2, I1>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile, a.wait); break;
+        case MOE_FMT_INT3: consume_f1<NMAT, NT8, MOE_FMT_INT3, I1>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile, a.wait); break;
+        case MOE_FMT_INT4: consume_f1<NMAT, NT8, MOE_FMT_INT4, I1>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile, a.wait); break;
+        default: consume_f1<NMAT, NT8, MOE_FMT_NVFP4, I1>(fm[1], SL, smem, full, empty, abort_flag, ntiles, stage, phase, ok, acc, a.trace, gtile, a.wait); break;
       }
       // lane outputs: weight row nl = 32s + 4g + 2t + (j >> 1), token row nt*8 + 2c + (j & 1)
       if (ok && a.P == 1) {
@@ -735,11 +767,12 @@ StageLayout stage_layout(int nmat, int nt8, const int* wmax) {
   return L;
 }
 
-template <int NMAT, int NT8>
+template <int NMAT, int NT8, bool I1>
 cudaError_t launch_n(GemvArgs g, const uint8_t* packed, uint64_t packed_bytes, const void* act, const float* sums,
                      const int* wmax, int max_chunks, cudaStream_t stream) {
-  CUtensorMap m2, m3, m4, mx, ms;
-  if (!encode_code_map(&m2, packed, packed_bytes, 2) || !encode_code_map(&m3, packed, packed_bytes, 3) ||
+  CUtensorMap m1, m2, m3, m4, mx, ms;
+  if (!encode_code_map(&m1, packed, packed_bytes, 1) || !encode_code_map(&m2, packed, packed_bytes, 2) ||
+      !encode_code_map(&m3, packed, packed_bytes, 3) ||
       !encode_code_map(&m4, packed, packed_bytes, 4) ||
       !encode_rows_map(&mx, act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, g.R, g.K, 128, 8 * NT8))
     return cudaErrorInvalidValue;
@@ -752,7 +785,7 @@ cudaError_t launch_n(GemvArgs g, const uint8_t* packed, uint64_t packed_bytes, c
   }
   g.st = stage_layout(NMAT, NT8, wmax);
   const int smem = g.st.stages * g.st.bytes + 1024 + kCtrlBytes;
-  auto kern = expert_gemv_kernel<NMAT, NT8>;
+  auto kern = expert_gemv_kernel<NMAT, NT8, I1>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   int per_sm = 0;
@@ -762,7 +795,7 @@ cudaError_t launch_n(GemvArgs g, const uint8_t* packed, uint64_t packed_bytes, c
   long long grid = (long long)gemv_sm_count() * (per_sm > 0 ? per_sm : 1);
   if (grid > items) grid = items;
   if (grid < 1) grid = 1;
-  kern<<<(unsigned)grid, kGemvThreads, smem, stream>>>(m2, m3, m4, mx, ms, g);
+  kern<<<(unsigned)grid, kGemvThreads, smem, stream>>>(m1, m2, m3, m4, mx, ms, g);
   return cudaGetLastError();
 }
 
@@ -834,8 +867,16 @@ cudaError_t launch_expert_gemv(const uint8_t* packed, uint64_t packed_bytes, con
   const int nmat = gateup ? 2 : 1;
   g.P = gemv_split(R, E, g.N, g.K, nmat);
   if (chunk_rows != 8) return cudaErrorInvalidValue;  // the host plans 8-row chunks (one token tile)
-  cudaError_t err = gateup ? launch_n<2, 1>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream)
-                           : launch_n<1, 1>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream);
+  bool any1 = false;  // a 1-bit matrix among this projection's
+  for (int e = 0; e < E; ++e)
+    for (int m = 0; m < (gateup ? 2 : 1); ++m) any1 |= fmt_host[e * 3 + (gateup ? m : 2)] == MOE_FMT_INT1;
+  cudaError_t err;
+  if (gateup)
+    err = any1 ? launch_n<2, 1, true>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream)
+               : launch_n<2, 1, false>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream);
+  else
+    err = any1 ? launch_n<1, 1, true>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream)
+               : launch_n<1, 1, false>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream);
   if (err != cudaSuccess || g.P == 1) return err;
   if (gateup)
     gemv_fixup_kernel<2><<<dim3(R, (g.N + 255) / 256), 256, 0, stream>>>(g, ws.idx);

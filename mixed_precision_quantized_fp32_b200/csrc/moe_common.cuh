@@ -21,7 +21,7 @@ constexpr int kMaxE = 256;
 constexpr int kMaxK = 8;
 
 __host__ __device__ inline bool fmt_known(int f) {
-  return f == MOE_FMT_INT2 || f == MOE_FMT_INT3 || f == MOE_FMT_INT4 || f == MOE_FMT_NVFP4;
+  return f == MOE_FMT_INT1 || f == MOE_FMT_INT2 || f == MOE_FMT_INT3 || f == MOE_FMT_INT4 || f == MOE_FMT_NVFP4;
 }
 // u32 words per group of 32 inputs
 __host__ __device__ inline int fmt_words(int f) { return f == MOE_FMT_NVFP4 ? 4 : f; }

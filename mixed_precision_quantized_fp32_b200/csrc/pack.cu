@@ -86,15 +86,24 @@ __global__ void pack_int_kernel(const float* __restrict__ W, int N, int K, uint3
     w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
   }
   float amax = 0.0f;
+  if (BITS == 1) {  // sign code: the scale is the mean |w| (fp32 sum in input order)
 #pragma unroll
-  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(w[i]));
-  __half sh = __float2half_rn(__fdiv_rn(amax, (float)QMAX));
+    for (int i = 0; i < 32; ++i) amax = __fadd_rn(amax, fabsf(w[i]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(w[i]));
+  }
+  __half sh = __float2half_rn(__fdiv_rn(amax, BITS == 1 ? 32.0f : (float)QMAX));
   uint16_t sbits = __half_as_ushort(sh);
   if ((sbits & 0x7FFFu) == 0x7C00u) sbits = 0x7BFFu;  // saturate the scale
   const float s = __half2float(__ushort_as_half(sbits));
   uint32_t u[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
+    if (BITS == 1) {  // sign bit: u = (q + 1) / 2 with q = +1 for w >= 0
+      u[i] = w[i] >= 0.0f ? 1u : 0u;
+      continue;
+    }
     int q = 0;
     if (s != 0.0f) {
       float r = rintf(__fdiv_rn(w[i], s));
@@ -106,7 +115,12 @@ __global__ void pack_int_kernel(const float* __restrict__ W, int N, int K, uint3
   // Inside a word, the two codes of a pair (2j, 2j+1) sit 16 bits apart, so a
   // mask of the shifted word yields both as the low bits of two half-words.
   const int k0 = g * 32;
-  if (BITS == 4) {
+  if (BITS == 1) {  // code 2j at bit j, code 2j+1 at bit 16+j
+    uint32_t v = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v |= (u[2 * j] << j) | (u[2 * j + 1] << (16 + j));
+    codes[word_index(n, k0, K, 1, 0)] = v;
+  } else if (BITS == 4) {
 #pragma unroll
     for (int wd = 0; wd < 4; ++wd) {
       uint32_t v = 0;
@@ -231,6 +245,7 @@ cudaError_t launch_pack(const float* W, int e0, int ne, int E, int H, int F, con
         uint16_t* sc = (uint16_t*)(out + scale_off[e * 3 + p]);
         if (f == MOE_FMT_INT4) pack_int_kernel<4><<<blocks, 256, 0, stream>>>(w, N, K, codes, sc);
         else if (f == MOE_FMT_INT3) pack_int_kernel<3><<<blocks, 256, 0, stream>>>(w, N, K, codes, sc);
+        else if (f == MOE_FMT_INT1) pack_int_kernel<1><<<blocks, 256, 0, stream>>>(w, N, K, codes, sc);
         else pack_int_kernel<2><<<blocks, 256, 0, stream>>>(w, N, K, codes, sc);
       }
       err = cudaGetLastError();

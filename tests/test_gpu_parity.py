@@ -28,6 +28,8 @@ from mixed_precision_quantized_fp32_b200 import _lib  # noqa: E402
 
 
 def custom(name, T, H, F, E, k, fmt, bias=None):
+    # a named configuration's packed buffer is cached by name, so custom layers use other names
+    assert name not in W.NAMES, name
     L = W.Layer(name, H, F, E, k, np.asarray(fmt, np.uint8).reshape(E, 3), (T,), (), bias)
     return L
 
@@ -117,7 +119,8 @@ def test_device_generator_matches_host():
 PACK_CASES = [
     ("int4", 384, 256, 3, [[4, 4, 4]] * 3),
     ("mixed", 256, 640, 6, [[3, 2, 4], [4, 4, 4], [2, 2, 2], [4, 4, 2], [3, 3, 3], [2, 4, 3]]),
-    ("nvfp4", 256, 384, 4, [[16, 16, 16]] * 4),
+    ("nvfp4_small", 256, 384, 4, [[16, 16, 16]] * 4),
+    ("graded_mix", 256, 384, 6, [[4, 4, 4], [2, 2, 2], [1, 1, 1], [4, 2, 1], [1, 2, 4], [2, 1, 2]]),
 ]
 
 
@@ -145,7 +148,33 @@ def test_pack_edge_values_bit_exact():
     np.testing.assert_array_equal(packed.cpu().numpy(), orc.pack_layer(Wh, 0, 3, 256, 256, fmt))
 
 
-@pytest.mark.parametrize("name", ["tiny", "mixtral", "hotcold", "nvfp4", "large"])
+def test_pack_edge_values_sign_code():
+    # 1-bit sign code: an all-zero matrix (scale 0, every code +1), signed zeros, tiny
+    # values (fp16-subnormal scale), and a group whose mean |w| overflows fp16 (scale
+    # saturated to 65504)
+    L = custom("edge1", 1, 256, 256, 2, 1, [[1, 1, 1], [1, 1, 1]])
+    fmt = L.fmt.reshape(-1)
+    Wh = np.stack([W.expert_w(e, 256, 256) for e in range(2)])
+    Wh[0, 0] = 0.0
+    Wh[0, 1, :4096] *= np.float32(1e-7)
+    Wh[0, 2, :32] = np.float32(70000.0)
+    Wh[1, 0, ::7] = np.float32(-0.0)
+    total = moe.pack_layout(2, 256, 256, fmt)[0]
+    packed = moe.alloc_packed(total)
+    moe.moe_pack(torch.from_numpy(Wh).cuda(), 0, 2, 256, 256, fmt, packed)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(packed.cpu().numpy(), orc.pack_layer(Wh, 0, 2, 256, 256, fmt))
+
+
+@pytest.mark.parametrize("T", [37, 600])
+def test_forward_graded_tiers(T):
+    # precision falling with hotness, down to the 1-bit sign code; T=37 runs the GEMV,
+    # T=600 the tcgen05 GEMMs on CTA pairs (F/128 = 2, H/128 = 4)
+    L = custom("graded_small", T, 512, 256, 6, 2, [[4, 4, 4], [2, 2, 2], [1, 1, 1], [4, 2, 1], [1, 2, 4], [2, 1, 2]])
+    check_layer(L, T)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mixtral", "hotcold", "nvfp4", "large", "graded"])
 def test_pack_bit_exact_configs(name):
     L = W.layer(name)
     layer = hp.gpu_pack_cached(L)
@@ -154,6 +183,9 @@ def test_pack_bit_exact_configs(name):
     elif name == "hotcold":
         hot = L.notes["hot_experts"]
         sample = [hot[0], next(e for e in range(L.E) if e not in hot), L.E - 1]
+    elif name == "graded":  # one expert of each tier: 4-, 2- and 1-bit
+        tiers = [int(np.flatnonzero(L.fmt[:, 0] == b)[0]) for b in (4, 2, 1)]
+        sample = sorted(tiers)
     else:
         sample = [0, L.E - 1]
     want = hp.oracle_pack(L, sample)
@@ -205,7 +237,7 @@ def test_forward_cta_pairs_ragged_chunks():
 
 def _sweep_case(i):
     """Seeded random shape: H, F in 128*{1..8}, E in {1..16}, k in {1..min(E, 8)}, T in {1..300};
-    every fourth case NVFP4, the rest a random integer width per expert and projection.  Cases
+    every fourth case NVFP4, the rest a random integer width (1 to 4 bits) per expert and projection.  Cases
     i % 5 == 2 push two experts' router bias to -1e4 (experts with no tokens), cases i % 5 == 4
     push one expert's bias to +1e4 (every token picks it)."""
     rng = np.random.default_rng(7000 + i)
@@ -213,7 +245,7 @@ def _sweep_case(i):
     E = int(rng.integers(1, 17))
     k = int(rng.integers(1, min(E, 8) + 1))
     T = int(rng.integers(1, 301))
-    fmt = [[16, 16, 16]] * E if i % 4 == 3 else rng.choice([2, 3, 4], size=(E, 3)).tolist()
+    fmt = [[16, 16, 16]] * E if i % 4 == 3 else rng.choice([1, 2, 3, 4], size=(E, 3)).tolist()
     bias = None
     if i % 5 == 2 and E - 2 >= k:
         bias = np.zeros(E, np.float32)
@@ -426,6 +458,7 @@ CONFIG_RUNS = [
     ("hotcold", 32, None), ("nvfp4", 16, None), ("large", 64, [0, 1, 2, 63]),
     ("mixtral", 2048, [0, 1, 1000, 2047]), ("hotcold", 4096, [0, 4095]),
     ("nvfp4", 8192, [0, 8191]), ("large", 8192, [0, 8191]),
+    ("graded", 32, None), ("graded", 4096, [0, 1, 2047, 4095]),
 ]
 
 
