@@ -99,6 +99,10 @@ enum {
  *     s = fp16 round-to-nearest-even of the fp32 quotient amax/qmax, saturated
  *     to 65504; q = clamp(rint(w/s), -qmax, qmax) with an IEEE fp32 division
  *     and round-half-even (s == 0 gives q = 0).  Dequantized weight = s*q.
+ *   1-bit sign code (the sub-2-bit cold tier): per row and group of 32,
+ *     s = fp16 round-to-nearest-even of (fp32 sum of |w| in input order)/32,
+ *     saturated to 65504 (the least-squares scale of a sign code); q = +1 for
+ *     w >= 0, else -1.  Dequantized weight = s*q.
  *   NVFP4: sT = amax(matrix)/2688 in fp32 (1 if the matrix is all zero);
  *     per row and block of 16 inputs: sb = e4m3(blockmax/(6*sT)) (round to
  *     nearest even, saturate to 448); v = e2m1(w/(sb*sT)) (nearest even,
@@ -106,12 +110,15 @@ enum {
  * Code layout: tiles of 128 outputs x 128 inputs, tile order output-block
  * major, input-block minor.  Inside a tile, u32 words ordered
  * [kg 0..3][word 0..b-1][n 0..127] (kg = group of 32 inputs inside the tile,
- * b = 2, 3, 4 words per group; NVFP4 uses 4).  Stored integer code u = q+2^(b-1).
+ * b = 1, 2, 3, 4 words per group; NVFP4 uses 4).  Stored integer code
+ * u = q+2^(b-1); 1-bit: u = (q+1)/2.
  * Inside an integer word the two codes of each pair (2j, 2j+1) sit 16 bits
  * apart (even code in the low half-word), so one mask of a shifted word
  * yields both:
  *   4-bit: codes 8w..8w+7 in word w; code 8w+2j at bits 4j..4j+3, code
  *          8w+2j+1 at bits 16+4j..16+4j+3 (j = 0..3)
+ *   1-bit: codes 0..31 in word 0; code 2j at bit j, code 2j+1 at bit 16+j
+ *          (j = 0..15)
  *   2-bit: codes 16w..16w+15 in word w; code 16w+2j at bits 2j..2j+1, code
  *          16w+2j+1 at bits 16+2j..17+2j (j = 0..7)
  *   3-bit: words 0-1 hold the low two bits of u as for 2-bit; word 2 holds

@@ -16,7 +16,9 @@
 //
 // Per group of 32 inputs, lane (g, c) holds word(s) of rows 4g..4g+3 covering
 // inputs 8c..8c+7.  It turns each pair of codes into one fp16x2 A-fragment
-// register with one AND (INT3: one more op per pair merges the high-bit plane):
+// register with one AND (INT3: one more op per pair merges the high-bit plane;
+// the 1-bit sign code's fields sit at bit j, with activations doubled so the
+// MMA sums (2u - 1)*x):
 //   * the masked field is read as an fp16 subnormal: a code u in a field of
 //     power-of-two weight f (bit position 2j or 4j of a half-word) is exactly
 //     u * f * 2^-24;
