@@ -102,7 +102,9 @@ enum {
  *   1-bit sign code (the sub-2-bit cold tier): per row and group of 32,
  *     s = fp16 round-to-nearest-even of (fp32 sum of |w| in input order)/32,
  *     saturated to 65504 (the least-squares scale of a sign code); q = +1 for
- *     w >= 0, else -1.  Dequantized weight = s*q.
+ *     w >= 0, else -1.  Dequantized weight = s*q.  Decode batches read the
+ *     inputs of a 1-bit matrix doubled in fp16, so they must stay below 32752
+ *     in magnitude.
  *   NVFP4: sT = amax(matrix)/2688 in fp32 (1 if the matrix is all zero);
  *     per row and block of 16 inputs: sb = e4m3(blockmax/(6*sT)) (round to
  *     nearest even, saturate to 448); v = e2m1(w/(sb*sT)) (nearest even,
