@@ -65,6 +65,12 @@ def test_pack_argument_errors():
     bad = fmt.copy()
     bad[2, 1] = 5
     assert _pack(None, 0, 0, 4, 256, 256, bad, None, 0)[0] == "MOE_ERR_FORMAT"
+    bad[2, 1] = 0
+    assert _pack(None, 0, 0, 4, 256, 256, bad, None, 0)[0] == "MOE_ERR_FORMAT"
+    one = fmt.copy()
+    one[1] = 1                                            # 1-bit codes: N*K/8 bytes, fp16 scales
+    st, t1 = _pack(None, 0, 0, 4, 256, 256, one, None, 0)[:2]
+    assert st == "MOE_OK" and t1 == moe.pack_layout(4, 256, 256, one)[0] < total
     assert _pack(None, 0, 0, 4, 256, 256, fmt, None, 0, want_total=False)[0] == "MOE_ERR_ARG"
     assert _pack(None, 0, 1, 4, 256, 256, fmt, FAKE, total)[0] == "MOE_ERR_ARG"   # W null
     assert _pack(FAKE, 3, 2, 4, 256, 256, fmt, FAKE, total)[0] == "MOE_ERR_ARG"   # e0+ne > E
@@ -80,7 +86,7 @@ def _fwd(T, k, E=8, H=256, F=512, fmt=None, x=FAKE, rw=FAKE, y=FAKE, packed=FAKE
     f = np.ascontiguousarray(fmt).ravel()
     if packed_bytes is None:
         packed_bytes = moe.pack_layout(E, H, F, f)[0] if (E <= 256 and H % 128 == 0 and F % 128 == 0
-                                                          and set(f) <= {2, 3, 4, 16}) else 1 << 40
+                                                          and set(f) <= {1, 2, 3, 4, 16}) else 1 << 40
     w = _lib.MoeWeights(E, H, F, f.ctypes.data, packed, packed_bytes)
     need = C.c_uint64(0)
     rc = _lib.load().moe_layer_forward(x, T, rw, None, C.byref(w), k, y, None if query else ws, ws_bytes,
@@ -102,6 +108,12 @@ def test_forward_argument_errors():
     mixed[3, 2] = 4
     assert _fwd(16, 2, fmt=mixed)[0] == "MOE_ERR_FORMAT"
     assert _fwd(16, 2, fmt=np.full((8, 3), 7))[0] == "MOE_ERR_FORMAT"
+    mixed1 = np.full((8, 3), 16, np.uint8)
+    mixed1[5, 0] = 1                                      # the 1-bit code is an integer format too
+    assert _fwd(16, 2, fmt=mixed1)[0] == "MOE_ERR_FORMAT"
+    graded = np.tile(np.array([[4, 2, 1], [1, 1, 1]], np.uint8), (4, 1))
+    st, need_g = _fwd(16, 2, fmt=graded, query=True)       # 1-bit matrices are accepted
+    assert st == "MOE_OK" and need_g > 0
     assert _fwd(0, 2)[0] == "MOE_OK"                      # empty batch: nothing to do
     assert _fwd(16, 2, x=None)[0] == "MOE_ERR_ARG"
     assert _fwd(16, 2, y=None)[0] == "MOE_ERR_ARG"
