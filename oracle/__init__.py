@@ -12,7 +12,9 @@ the definition it follows in its C counterpart.
 
 Parity status of each function (its pins are the ``-m "not gpu"`` tests in
 ``tests/test_oracle_*.py``): every function here is pinned; see the test
-module docstrings for which property pins which function.
+module docstrings for which property pins which function.  ``outliers.py``
+(outlier isolation, numpy on top of these functions) is pinned by
+``tests/test_oracle_outliers.py``.
 """
 from __future__ import annotations
 
