@@ -13,8 +13,9 @@ the definition it follows in its C counterpart.
 Parity status of each function (its pins are the ``-m "not gpu"`` tests in
 ``tests/test_oracle_*.py``): every function here is pinned; see the test
 module docstrings for which property pins which function.  ``outliers.py``
-(outlier isolation, numpy on top of these functions) is pinned by
-``tests/test_oracle_outliers.py``.
+(outlier isolation) and ``nvfp4_act.py`` (NVFP4 activations), numpy on top
+of these functions, are pinned by ``tests/test_oracle_outliers.py`` and
+``tests/test_oracle_nvfp4_act.py``.
 """
 from __future__ import annotations
 
