@@ -1,10 +1,12 @@
 """Benchmark of the quantized MoE FFN layer forward on B200.
 
-Default workload: the Mixtral-like layer (H=4096, F=14336, E=8, top-2; gate
-3-bit, up 2-bit, down 4-bit, group 32 with fp16 scales) run as prefill of
-T=2048 tokens.  One step = one full layer forward (router, top-k, permute,
-gather, gate/up GEMM + SwiGLU, down GEMM, combine) over one batch.  Decode
-batches T=1/8/64 of the same layer are reported under "runs".
+Contract workload: the large-expert layer (H=12288, F=14336, E=128, top-2;
+gate/up 4-bit, down 2-bit, group 32 with fp16 scales; 32.4 GB packed) run as
+prefill of T=8192 tokens, the largest configuration of the workload set.  One
+step = one full layer forward (router, top-k, permute, gather, gate/up GEMM +
+SwiGLU, down GEMM, combine) over one batch.  Every other layer and batch of the
+set (tiny T=16; Mixtral-like T=1/8/64/2048; hot/cold T=32/4096; NVFP4
+T=16/8192; large T=64; graded T=32/4096) is reported under "runs".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -36,8 +38,6 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 CSRC = os.path.join(ROOT, "mixed_precision_quantized_fp32_b200", "csrc")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-KERNELS_PER_FORWARD_INT = 9     # router, top-k, 3 permute, gather, gate/up, down, combine
-KERNELS_PER_FORWARD_FP4 = 11    # + x quant, h quant
 
 
 def workload_desc(L: W.Layer, T: int, mode: str) -> str:
@@ -183,15 +183,28 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
-def expert_gateup_bytes(L: W.Layer, moe) -> np.ndarray:
-    """Packed bytes (codes + scales) of the gate and up matrices of each expert."""
-    out = np.zeros(L.E)
-    for e in range(L.E):
-        for p in (0, 1):
-            f = int(L.fmt[e, p])
-            n = L.F * L.H
-            out[e] += n * (4 if f == 16 else f) / 8 + (n / 16)
-    return out
+HEADLINE = ("large", 8192)
+RUNS = [("tiny", 16), ("mixtral", 1), ("mixtral", 8), ("mixtral", 64), ("mixtral", 2048),
+        ("hotcold", 32), ("hotcold", 4096), ("nvfp4", 16), ("nvfp4", 8192), ("large", 64),
+        ("graded", 32), ("graded", 4096)]
+STAGES = ["router_topk", "permute", "gather", "gateup", "h_quant", "down", "combine"]
+
+
+def matrix_bytes(L: W.Layer, e: int, p: int) -> float:
+    """Packed bytes (codes + scales) of matrix p of expert e."""
+    f = int(L.fmt[e, p])
+    n = L.F * L.H
+    return n * (4 if f == 16 else f) / 8 + n / 16
+
+
+def launches_per_forward(L: W.Layer, T: int) -> int:
+    """Kernels one forward launches on the prefill (tcgen05) path: router (split of the fp32
+    weights + GEMM when T > 64 and E > 32, else one kernel) + top-k, permutation (one kernel
+    when T*k <= 1024, else three), activation gather (NVFP4: quantize + gather), gate/up,
+    h quantization (NVFP4), down, combine."""
+    router = 2 if (T > 64 and L.E > 32) else 1
+    perm = 1 if T * L.k <= 1024 else 3
+    return router + 1 + perm + (2 if L.fp4 else 1) + 1 + (1 if L.fp4 else 0) + 1 + 1
 
 
 def gpu_pack(L: W.Layer, moe, dev):
@@ -205,7 +218,62 @@ def gpu_pack(L: W.Layer, moe, dev):
         ne = min(per, L.E - e0)
         moe.moe_pack(W.device_expert_weights(L, e0, ne, out=stage[:ne]), e0, L.E, L.H, L.F, fmt, packed)
     torch.cuda.synchronize()
+    del stage
     return moe.PackedLayer(L.E, L.H, L.F, fmt, packed)
+
+
+def measure_batch(L: W.Layer, layer, T: int, moe, dev, pk, flush, n: int, seed: int = 0):
+    """One layer / batch: event-timed forwards (L2 flushed before each decode step) and the
+    roofline of its gate/up and down kernels.  Decode batches add CUDA-graph replay."""
+    import torch
+    decode = T in L.decode_T
+    nev = moe.MOE_STAGE_EVENTS
+    Wr, b = W.device_router(L)
+    x = torch.empty((T, L.H), dtype=torch.bfloat16, device=dev)
+    W.fill_device_bf16(x, seed, W.TID_X, 1.0)
+    ws = moe.alloc_packed(moe.workspace_bytes(layer, T, L.k), dev)
+    y = torch.empty_like(x)
+    cnt = torch.zeros(L.E, dtype=torch.int32, device=dev)
+    moe.moe_layer_forward(x, Wr, b, layer, L.k, y=y, ws=ws, debug={"counts": cnt})
+    torch.cuda.synchronize()
+    active = np.nonzero(cnt.cpu().numpy())[0]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(n)]
+    for row in ev:
+        for e_ in row:
+            e_.record()
+    for _ in range(3):
+        moe.moe_layer_forward(x, Wr, b, layer, L.k, y=y, ws=ws)
+    for i in range(n):
+        if decode:
+            flush.zero_()
+        moe.moe_layer_forward(x, Wr, b, layer, L.k, y=y, ws=ws, stage_events=ev[i])
+    torch.cuda.synchronize()
+    st = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(nev - 1)] for i in range(n)]).mean(0)
+    step = float(np.mean([ev[i][0].elapsed_time(ev[i][-1]) for i in range(n)]))
+    gu, dn = float(st[3]), float(st[5])
+    mode = "decode" if decode else "prefill"
+    out = {"workload": workload_desc(L, T, mode), "layer": L.name, "T": T, "mode": mode,
+           "tokens_per_s": round(T / step * 1e3, 1), "ms_per_step": round(step, 4),
+           "active_experts": int(len(active)),
+           "stages_ms": dict(zip(STAGES, [round(float(v), 4) for v in st]))}
+    if decode:
+        gms = graph_step_ms(lambda: moe.moe_layer_forward(x, Wr, b, layer, L.k, y=y, ws=ws), flush, n)
+        out["graph_tokens_per_s"] = round(T / gms * 1e3, 1)
+        out["graph_ms_per_step"] = round(gms, 4)
+        bg = sum(matrix_bytes(L, int(e), 0) + matrix_bytes(L, int(e), 1) for e in active)
+        bd = sum(matrix_bytes(L, int(e), 2) for e in active)
+        for key, by, t in (("gateup", bg, gu), ("down", bd, dn)):
+            out[key] = {"bound": "hbm", "achieved": round(by / t / 1e6, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(by / t / 1e6 / pk["hbm_gbs"], 4), "algorithmic_bytes_per_launch": by,
+                        "avg_launch_ms": round(t, 4)}
+    else:
+        fl = 2.0 * T * L.k * L.H * L.F
+        for key, f, t in (("gateup", 2 * fl, gu), ("down", fl, dn)):
+            out[key] = {"bound": "tensor", "achieved": round(f / t / 1e9, 1), "peak": pk["bf16_tflops"],
+                        "unit": "TFLOP/s", "frac": round(f / t / 1e9 / pk["bf16_tflops"], 4),
+                        "algorithmic_flops_per_launch": f, "avg_launch_ms": round(t, 4)}
+    del ws, x, y
+    return out
 
 
 def run_ours(args, rank, world, local_rank):
@@ -215,8 +283,8 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    L = W.layer("mixtral")
-    T = 2048
+    name, T = HEADLINE
+    L = W.layer(name)
     layer = gpu_pack(L, moe, dev)
     x = torch.empty((T, L.H), dtype=torch.bfloat16, device=dev)
     W.fill_device_bf16(x, replica_seed(rank), W.TID_X, 1.0)   # each replica its own tokens
@@ -309,57 +377,37 @@ def run_ours(args, rank, world, local_rank):
     gateup_ms = float(stage_ms[:, 3].mean())
     down_ms = float(stage_ms[:, 5].mean())
     flops_gateup = 2.0 * T * L.k * 2 * L.H * L.F
+    flops_down = 2.0 * T * L.k * L.H * L.F
     achieved = flops_gateup / (gateup_ms / 1e3) / 1e12
-    traffic = ncu_traffic("gateup_prefill_mixtral")
-    roofline = {"bound": "tensor", "kernel": "expert GEMM gate/up + SwiGLU (fp16 operands)",
+    roofline = {"bound": "tensor", "kernel": "expert GEMM gate/up + SwiGLU (tcgen05, fp16 operands)",
                 "achieved": round(achieved, 2), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": traffic,
+                "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": ncu_traffic(f"gateup_prefill_{name}"),
                 "peak_source": f"{pk_kind} dense bf16 (= fp16) burst, MEASURED_PEAKS.json"
                 if pk_kind == "measured" else "fallback 1.59 PFLOP/s",
-                "algorithmic_flops_per_launch": flops_gateup, "avg_launch_ms": round(gateup_ms, 4)}
-    stages = dict(zip(["router_topk", "permute", "gather", "gateup", "h_quant", "down", "combine"],
-                      [round(float(v), 4) for v in stage_ms.mean(0)]))
+                "algorithmic_flops_per_launch": flops_gateup, "avg_launch_ms": round(gateup_ms, 4),
+                "down": {"achieved": round(flops_down / (down_ms / 1e3) / 1e12, 2),
+                         "frac": round(flops_down / (down_ms / 1e3) / 1e12 / pk["bf16_tflops"], 4),
+                         "avg_launch_ms": round(down_ms, 4),
+                         "traffic": ncu_traffic(f"down_prefill_{name}")}}
+    stages = dict(zip(STAGES, [round(float(v), 4) for v in stage_ms.mean(0)]))
+    del ws, x_dev, y_dev, layer
+    torch.cuda.empty_cache()
 
-    # ---- decode batches of the same layer (HBM-bound; L2 flushed between steps)
+    # ---- every other layer and batch of the workload set
     runs = []
-    if not args.no_decode:
+    if not args.no_runs:
         flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-        eb = expert_gateup_bytes(L, moe)
-        for Td in (1, 8, 64):
-            xd = torch.empty((Td, L.H), dtype=torch.bfloat16, device=dev)
-            W.fill_device_bf16(xd, replica_seed(rank), W.TID_X, 1.0)
-            wsd = moe.alloc_packed(moe.workspace_bytes(layer, Td, L.k), dev)
-            cnt = torch.zeros(L.E, dtype=torch.int32, device=dev)
-            moe.moe_layer_forward(xd, Wr, b, layer, L.k, ws=wsd, debug={"counts": cnt})
-            torch.cuda.synchronize()
-            active = cnt.cpu().numpy() > 0
-            nd = max(args.steps, 10)
-            evd = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(nd)]
-            for row in evd:
-                for e in row:
-                    e.record()
-            for _ in range(3):
-                moe.moe_layer_forward(xd, Wr, b, layer, L.k, ws=wsd)
-            for s in range(nd):
-                flush.zero_()
-                moe.moe_layer_forward(xd, Wr, b, layer, L.k, ws=wsd, stage_events=evd[s])
-            torch.cuda.synchronize()
-            st = np.array([[evd[s][i].elapsed_time(evd[s][i + 1]) for i in range(nev - 1)] for s in range(nd)])
-            stp = np.array([evd[s][0].elapsed_time(evd[s][-1]) for s in range(nd)])
-            gu = float(st[:, 3].mean())
-            by = float(eb[active].sum())
-            yd = torch.empty_like(xd)
-            gms = graph_step_ms(lambda: moe.moe_layer_forward(xd, Wr, b, layer, L.k, y=yd, ws=wsd), flush, nd)
-            runs.append({"workload": workload_desc(L, Td, "decode"), "tokens_per_s": round(Td / (stp.mean() / 1e3), 1),
-                         "ms_per_step": round(float(stp.mean()), 4),
-                         "graph_tokens_per_s": round(Td / (gms / 1e3), 1), "graph_ms_per_step": round(gms, 4),
-                         "active_experts": int(active.sum()),
-                         "gateup": {"bound": "hbm", "achieved": round(by / (gu / 1e3) / 1e9, 1),
-                                    "peak": pk["hbm_gbs"], "unit": "GB/s",
-                                    "frac": round(by / (gu / 1e3) / 1e9 / pk["hbm_gbs"], 4),
-                                    "algorithmic_bytes_per_launch": by, "avg_launch_ms": round(gu, 4)},
-                         "stages_ms": dict(zip(stages.keys(), [round(float(v), 4) for v in st.mean(0)]))})
+        done = {}
+        for rn, rT in RUNS:
+            if rn not in done:
+                done.clear()
+                torch.cuda.empty_cache()
+                done[rn] = gpu_pack(W.layer(rn), moe, dev)
+            runs.append(measure_batch(W.layer(rn), done[rn], rT, moe, dev, pk, flush, max(args.steps // 2, 10),
+                                      seed=replica_seed(rank)))
+        done.clear()
         del flush
+        torch.cuda.empty_cache()
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -368,86 +416,35 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded counter-based generator; random-init weights)",
         "config": {"workload": workload_desc(L, T, "prefill"), "global_batch": T * world,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (617 MB packed weights streamed per step)"},
+                   "l2": "inputs larger than L2 (32.4 GB packed weights streamed per step)"},
         "roofline": roofline,
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2),
                 "overlap": "double-buffered: copy streams move step i+1's input and step i-1's output while "
                            "step i computes"},
-        "gpu_launches": KERNELS_PER_FORWARD_INT * args.steps,
+        "gpu_launches": launches_per_forward(L, T) * args.steps,
         "clocks": clk, "stages_ms": stages, "runs": runs,
     }
-    return out, layer
+    return out
 
 
 # ------------------------------------------------------------------ all layers (report)
-def matrix_bytes(L: W.Layer, e: int, p: int) -> float:
-    f = int(L.fmt[e, p])
-    n = L.F * L.H
-    return n * (4 if f == 16 else f) / 8 + n / 16
-
-
 def run_suite(args):
-    """Every layer of the workload set, decode and prefill batches: tokens/s and the
-    roofline of the gate/up and down kernels.  One JSON line per batch."""
+    """Every batch of the named layers: tokens/s and the roofline of the gate/up and down
+    kernels, one JSON line per batch."""
     import torch
 
     import mixed_precision_quantized_fp32_b200 as moe
     dev = torch.device("cuda", 0)
     pk, _ = peaks()
-    nev = moe.MOE_STAGE_EVENTS
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     for name in args.suite.split(","):
         L = W.layer(name)
         layer = gpu_pack(L, moe, dev)
-        Wr, b = W.device_router(L)
         for T in list(L.decode_T) + list(L.prefill_T):
             if args.batch and T != args.batch:
                 continue
-            decode = T in L.decode_T
-            x = torch.empty((T, L.H), dtype=torch.bfloat16, device=dev)
-            W.fill_device_bf16(x, 0, W.TID_X, 1.0)
-            ws = moe.alloc_packed(moe.workspace_bytes(layer, T, L.k), dev)
-            cnt = torch.zeros(L.E, dtype=torch.int32, device=dev)
-            moe.moe_layer_forward(x, Wr, b, layer, L.k, ws=ws, debug={"counts": cnt})
-            torch.cuda.synchronize()
-            counts = cnt.cpu().numpy()
-            active = np.nonzero(counts)[0]
-            n = 10
-            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(n)]
-            for row in ev:
-                for e_ in row:
-                    e_.record()
-            for _ in range(3):
-                moe.moe_layer_forward(x, Wr, b, layer, L.k, ws=ws)
-            for i in range(n):
-                if decode:
-                    flush.zero_()
-                moe.moe_layer_forward(x, Wr, b, layer, L.k, ws=ws, stage_events=ev[i])
-            torch.cuda.synchronize()
-            st = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(nev - 1)] for i in range(n)]).mean(0)
-            step = float(np.mean([ev[i][0].elapsed_time(ev[i][-1]) for i in range(n)]))
-            gu, dn = float(st[3]), float(st[5])
-            out = {"layer": name, "T": T, "mode": "decode" if decode else "prefill", "tokens_per_s": round(T / step * 1e3, 1),
-                   "ms_per_step": round(step, 4), "active_experts": int(len(active)),
-                   "stages_ms": dict(zip(["router_topk", "permute", "gather", "gateup", "h_quant", "down", "combine"],
-                                         [round(float(v), 4) for v in st]))}
-            if decode:
-                yg = torch.empty_like(x)
-                gms = graph_step_ms(lambda: moe.moe_layer_forward(x, Wr, b, layer, L.k, y=yg, ws=ws), flush, n)
-                out["graph_tokens_per_s"] = round(T / gms * 1e3, 1)
-                out["graph_ms_per_step"] = round(gms, 4)
-                bg = sum(matrix_bytes(L, int(e), 0) + matrix_bytes(L, int(e), 1) for e in active)
-                bd = sum(matrix_bytes(L, int(e), 2) for e in active)
-                out["gateup"] = {"GB/s": round(bg / gu / 1e6, 1), "frac_hbm": round(bg / gu / 1e6 / pk["hbm_gbs"], 4)}
-                out["down"] = {"GB/s": round(bd / dn / 1e6, 1), "frac_hbm": round(bd / dn / 1e6 / pk["hbm_gbs"], 4)}
-                out["layer_GB/s_weights"] = round((bg + bd) / step / 1e6, 1)
-            else:
-                fl = 2.0 * T * L.k * L.H * L.F
-                out["gateup"] = {"TFLOP/s": round(2 * fl / gu / 1e9, 1), "frac_tensor": round(2 * fl / gu / 1e9 / pk["bf16_tflops"], 4)}
-                out["down"] = {"TFLOP/s": round(fl / dn / 1e9, 1), "frac_tensor": round(fl / dn / 1e9 / pk["bf16_tflops"], 4)}
-            print(json.dumps(out), flush=True)
-            del ws, x
+            print(json.dumps(measure_batch(L, layer, T, moe, dev, pk, flush, 10)), flush=True)
         del layer
         torch.cuda.empty_cache()
 
@@ -491,7 +488,10 @@ class OracleSample:
             n = min(self.T_full, max(n + 1, int(n * min(4.0, 0.9 * budget_s / dt))))
 
     def describe(self, n: int) -> str:
-        return f"first {n} of {self.T_full} tokens of the same batch (oracle packing untimed)"
+        return (f"first {n} of {self.T_full} tokens of the same batch, {len(self.packed)} of {self.L.E} experts "
+                f"active (oracle packing untimed; the oracle decodes each active expert's rows once per call, "
+                f"so with fewer rows per expert than the full batch this rate is a lower bound of its "
+                f"full-batch rate)")
 
 
 def oracle_time(L: W.Layer, T_full: int, budget_s: float, x_seed: int = 0):
@@ -505,8 +505,8 @@ def oracle_time(L: W.Layer, T_full: int, budget_s: float, x_seed: int = 0):
 def run_reference(args, rank, world):
     if rank != 0:
         return None
-    L = W.layer("mixtral")
-    T = 2048
+    name, T = HEADLINE
+    L = W.layer(name)
     s = OracleSample(L, T)
     n = s.calibrate(max(2.0, 60.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
@@ -531,11 +531,11 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--no-decode", action="store_true", help="skip the decode runs")
+    ap.add_argument("--no-runs", action="store_true", help="skip the other layers and batches (\"runs\")")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--suite", default="", help="comma-separated layers to report instead of the contract line "
-                                                "(tiny,mixtral,hotcold,nvfp4,large)")
+                                                "(tiny,mixtral,hotcold,nvfp4,large,graded)")
     ap.add_argument("--batch", type=int, default=0, help="with --suite: only this batch size")
     args = ap.parse_args()
     if args.suite:
@@ -560,12 +560,12 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
-    out, _ = run_ours(args, rank, world, local_rank)
+    out = run_ours(args, rank, world, local_rank)
     if world > 1:
         torch.distributed.barrier()
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            v, sample, cores = oracle_time(W.layer("mixtral"), 2048, args.cpu_budget)
+            v, sample, cores = oracle_time(W.layer(HEADLINE[0]), HEADLINE[1], args.cpu_budget)
             out["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                    "sample": sample}
         print(json.dumps(out), flush=True)

@@ -28,13 +28,19 @@
  *  - Pointers are DEVICE pointers unless marked HOST.  The caller owns all
  *    memory; the library allocates no device or pinned memory and keeps no
  *    state between calls except a per-process cache of device properties.
+ *    Two exceptions belong to moe_layer_forward_noalloc alone: its fixed
+ *    scratch array (a __device__ array that every GPU loading the library
+ *    holds) and a per-device cache of that array's address (see there).
  *  - Calls are asynchronous on `stream`; nothing is synchronized inside.
  *  - Errors are reported by the return code only.  Arguments are validated
  *    before anything is launched, so a call that returns an error other than
  *    MOE_ERR_CUDA has launched nothing.
- *  - Device-side failures (a bounded wait that gave up, a range check) are
- *    written as a moe_status value to moe_debug.status when that pointer is
- *    given (the caller zeroes it and reads it after synchronizing).
+ *  - Device-side failures (a bounded wait that gave up, an fp16 range
+ *    overflow) are written as a moe_status value to moe_debug.status when that
+ *    pointer is given (the caller zeroes it and reads it after synchronizing).
+ *    They happen after the call has returned, so its return code cannot carry
+ *    them: without moe_debug.status a call that met one still returns MOE_OK
+ *    and its y is undefined.
  */
 #ifndef MOE_H_
 #define MOE_H_
@@ -62,7 +68,9 @@ typedef enum {
                              or a packed buffer whose header disagrees */
   MOE_ERR_CUDA = 6,       /* a CUDA runtime call or launch failed */
   MOE_ERR_TIMEOUT = 7,    /* device-side bounded wait gave up (status word only) */
-  MOE_ERR_UNSUPPORTED_DEVICE = 8 /* current device is not compute capability 10.x */
+  MOE_ERR_UNSUPPORTED_DEVICE = 8, /* current device is not compute capability 10.0 */
+  MOE_ERR_RANGE = 9       /* integer-format layer: a SwiGLU output h reached the fp16 limit
+                             (|h| >= 65520 rounds to inf); status word only */
 } moe_status;
 
 /* Weight formats, chosen per expert and per projection. */
@@ -102,9 +110,7 @@ enum {
  *   1-bit sign code (the sub-2-bit cold tier): per row and group of 32,
  *     s = fp16 round-to-nearest-even of (fp32 sum of |w| in input order)/32,
  *     saturated to 65504 (the least-squares scale of a sign code); q = +1 for
- *     w >= 0, else -1.  Dequantized weight = s*q.  Decode batches read the
- *     inputs of a 1-bit matrix doubled in fp16, so they must stay below 32752
- *     in magnitude.
+ *     w >= 0, else -1.  Dequantized weight = s*q.
  *   NVFP4: sT = amax(matrix)/2688 in fp32 (1 if the matrix is all zero);
  *     per row and block of 16 inputs: sb = e4m3(blockmax/(6*sT)) (round to
  *     nearest even, saturate to 448); v = e2m1(w/(sb*sT)) (nearest even,
@@ -230,8 +236,13 @@ typedef struct {
  *      the sum); NVFP4 layers then quantize each h row to e4m3 (amax/448);
  *   6. o = Wd h per row; y[t] = bf16( sum_j w[t][j] * o[row(t,j)] ) summed in
  *      fp32 in ascending j.
- * Integer-format layers convert x and h to fp16, so |x| and |h| must stay
- * below 65504.  Layers must be all-NVFP4 or all-integer (MOE_ERR_FORMAT).
+ * Integer-format layers run their expert GEMMs on fp16 operands.  A token
+ * whose max |x| reaches 2^15 is scaled by a power of two 2^-e (exact) before
+ * its fp16 conversion and its gate/up sums by 2^e after, so every finite bf16
+ * x is accepted.  The SwiGLU output h is stored in fp16: an |h| that rounds
+ * beyond 65504 writes MOE_ERR_RANGE to moe_debug.status (y is then not
+ * finite).  NVFP4 layers scale x and h per row and have no such limit.
+ * Layers must be all-NVFP4 or all-integer (MOE_ERR_FORMAT).
  * Errors: MOE_ERR_ARG, MOE_ERR_ALIGN, MOE_ERR_SHAPE, MOE_ERR_FORMAT,
  *   MOE_ERR_WORKSPACE, MOE_ERR_UNSUPPORTED_DEVICE, MOE_ERR_CUDA.
  */
@@ -258,11 +269,17 @@ MOE_API moe_status moe_layer_forward(const void* x, int32_t T, const float* rout
  *
  * The first call on a device looks up the array's device address with
  * cudaGetSymbolAddress (with that device current) and caches it; make that
- * first call before any stream capture.  Every call shares the one array and
- * leaves its contents behind, so calls that overlap on the GPU (other streams,
- * other host threads) race on it: serialize them.  Nothing in the array needs
- * to start at zero: every byte the forward reads is written earlier in the
- * same call.  Errors: as moe_layer_forward.
+ * first call before any stream capture.  The cached address belongs to the
+ * device's current context: a cudaDeviceReset (or any other teardown of the
+ * primary context) while the library is in use leaves it stale, so do not
+ * reset a device between calls of this entry point.  Every call shares the
+ * one array and leaves its contents behind, so calls that overlap on the GPU
+ * (other streams, other host threads) race on it: serialize them.  Nothing in
+ * the array needs to start at zero: every byte the forward reads is written
+ * earlier in the same call.  The array also holds the status word used when
+ * dbg or dbg->status is NULL, which the caller cannot read: pass
+ * moe_debug.status to see device-side errors (MOE_ERR_TIMEOUT, MOE_ERR_RANGE).
+ * Errors: as moe_layer_forward.
  */
 #define MOE_NOALLOC_SCRATCH_BYTES (32ull << 20)
 MOE_API moe_status moe_layer_forward_noalloc(const void* x, int32_t T, const float* router_w,

@@ -19,6 +19,7 @@ MOE_TRACE_STAGES = 1024
 STATUS = {
     0: "MOE_OK", 1: "MOE_ERR_ARG", 2: "MOE_ERR_ALIGN", 3: "MOE_ERR_SHAPE", 4: "MOE_ERR_WORKSPACE",
     5: "MOE_ERR_FORMAT", 6: "MOE_ERR_CUDA", 7: "MOE_ERR_TIMEOUT", 8: "MOE_ERR_UNSUPPORTED_DEVICE",
+    9: "MOE_ERR_RANGE",
 }
 
 EXPORTS = ("moe_pack", "moe_layer_forward", "moe_layer_forward_noalloc")

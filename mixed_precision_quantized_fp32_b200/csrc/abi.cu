@@ -9,17 +9,19 @@ namespace moe {
 namespace {
 
 constexpr int kMaxDev = 64;
-int g_dev_ok[kMaxDev];  // 0 unknown, 1 sm_10x, -1 other (per-process property cache)
+int g_dev_ok[kMaxDev];  // 0 unknown, 1 sm_100, -1 other (per-process property cache)
 
 moe_status check_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDev) return MOE_ERR_UNSUPPORTED_DEVICE;
   if (g_dev_ok[dev] == 0) {
-    int major = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    // the library ships sm_100a code only, which runs on compute capability 10.0 alone
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
       return MOE_ERR_CUDA;
-    g_dev_ok[dev] = (major == 10) ? 1 : -1;
+    g_dev_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
   }
   return g_dev_ok[dev] == 1 ? MOE_OK : MOE_ERR_UNSUPPORTED_DEVICE;
 }
@@ -92,6 +94,7 @@ uint64_t carve(uint8_t* base, int T, int k, int E, int H, int F, bool fp4, const
     ws.xq = (uint8_t*)take((uint64_t)T * H);
     ws.sx = (float*)take((uint64_t)T * 4);
   }
+  if (!fp4) ws.xinv = (float*)take(R * 4);
   ws.xs = take(R * H * 2);
   ws.h = take(R * F * (fp4 ? 4 : 2));
   if (fp4) {

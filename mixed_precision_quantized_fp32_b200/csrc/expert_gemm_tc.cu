@@ -110,6 +110,7 @@ struct TcArgs {
   const int32_t* chunks;   // (expert, first row, rows) triples
   const int32_t* chunk_count;
   const float* row_scale;  // NVFP4: gate/up -> per-token sx, down -> per-row sh; null for integer layers
+  const float* xinv;       // integer gate/up: per-row 2^e undoing the activations' prescale (null otherwise)
   const int32_t* perm;
   int topk;
   void* out;               // gate/up: h [rows][F] (fp16, or fp32 for NVFP4); down: o fp32 [rows][H]
@@ -553,6 +554,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ptx::tc_fence_after();
       const int nrow = (a.pair ? 2 * mt : mt) * kTcBM + q * 32 + lane;
       const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+      bool range = false;  // an fp16 SwiGLU output overflowed
       for (int cb = cq * kColsPerWarp; cb < cq * kColsPerWarp + kColsPerWarp && cb < rows; cb += 16) {
         uint32_t r0[16], r1[16];
         ptx::tmem_ld16(lane_base + (uint32_t)cb, r0);
@@ -580,7 +582,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               u *= sx * tsc[1];
               reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = __fdividef(g, 1.0f + __expf(-g)) * u;
             } else {
-              reinterpret_cast<__half*>(a.out)[(size_t)r * a.N + nrow] = __float2half_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
+              if (a.xinv) {
+                const float xi = a.xinv[r];
+                g *= xi;
+                u *= xi;
+              }
+              const __half h = __float2half_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
+              range |= __hisinf(h) != 0;
+              reinterpret_cast<__half*>(a.out)[(size_t)r * a.N + nrow] = h;
             }
           } else {
             float o = __uint_as_float(r0[j]);
@@ -589,6 +598,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
+      if (range && a.status) atomicCAS(a.status, 0, (int32_t)MOE_ERR_RANGE);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -724,6 +734,7 @@ cudaError_t launch_expert_gemm_tc(const uint8_t* packed, const uint8_t* fmt_host
     a.K = H;
     a.proj = 0;
     a.row_scale = fp4 ? ws.sx : nullptr;
+    a.xinv = fp4 ? nullptr : ws.xinv;
     a.out = ws.h;
     if ((F / kTcBM) % 2 == 0)  // weight tiles in pairs of CTAs
       return any1 ? launch_tc<2, true, true>(a, max_words, ws.xs, R, stream)

@@ -17,8 +17,8 @@
 // Per group of 32 inputs, lane (g, c) holds word(s) of rows 4g..4g+3 covering
 // inputs 8c..8c+7.  It turns each pair of codes into one fp16x2 A-fragment
 // register with one AND (INT3: one more op per pair merges the high-bit plane;
-// the 1-bit sign code's fields sit at bit j, with activations doubled so the
-// MMA sums (2u - 1)*x):
+// the 1-bit sign code's fields sit at bit j, the MMA sums (u - 1/2)*x and the
+// group scale is doubled):
 //   * the masked field is read as an fp16 subnormal: a code u in a field of
 //     power-of-two weight f (bit position 2j or 4j of a half-word) is exactly
 //     u * f * 2^-24;
@@ -80,6 +80,7 @@ struct GemvArgs {
   const int32_t* chunks;  // (expert, first row, rows)
   const int32_t* chunk_count;
   const float* row_scale; // NVFP4: gate/up -> per-token sx, down -> per-row sh; null for integer layers
+  const float* xinv;      // integer gate/up: per-row 2^e undoing the activations' prescale (null otherwise)
   const int32_t* perm;
   bool sums;              // integer layer: activation group sums are loaded with the tiles
   void* out;              // gate/up: h [R][F] (fp16, or fp32 for NVFP4); down: o fp32 [R][H]
@@ -151,21 +152,24 @@ constexpr uint32_t h2c(uint32_t h) { return h | (h << 16); }
 // Activation multiplier 1/f_j (fp16x2) for pair j (j = 0..3) of a lane's eight
 // inputs, whose codes sit in a field of weight f_j: INT4 1, 16, 1, 16 (fields at
 // bits 0 and 4; pairs 2, 3 after >> 8); INT2 and INT3 4^j (fields at bits 2j);
-// INT1 2^j (fields at bit j), times 2 for the sign code's q = 2u - 1.
+// INT1 2^j (fields at bit j).  Every multiplier is at most 1, so the products
+// stay in range for any fp16 activation.
 __host__ __device__ constexpr uint32_t act_mul(int fmt, int j) {
   return fmt == MOE_FMT_NVFP4 ? h2c(0x3C00u)
-         : fmt == MOE_FMT_INT1 ? (j == 0 ? h2c(0x4000u) : j == 1 ? h2c(0x3C00u) : j == 2 ? h2c(0x3800u) : h2c(0x3400u))
+         : fmt == MOE_FMT_INT1 ? (j == 0 ? h2c(0x3C00u) : j == 1 ? h2c(0x3800u) : j == 2 ? h2c(0x3400u) : h2c(0x3000u))
          : fmt == MOE_FMT_INT4 ? ((j & 1) ? h2c(0x2C00u) : h2c(0x3C00u))   // 1, 1/16
          : (j == 0 ? h2c(0x3C00u) : j == 1 ? h2c(0x3400u) : j == 2 ? h2c(0x2C00u) : h2c(0x2400u));  // 4^-j
 }
-// -offset * 2^-24: times the group sum of the activations, the MMA's C input
-// (INT1: q = 2u - 1, so with the activations doubled the offset is 1).
+// -offset * 2^-24: times the group sum of the activations, the MMA's C input.
+// INT1: the sign code q = 2u - 1 = 2(u - 1/2), so the MMA sums (u - 1/2) x and
+// the group scale is doubled (group_scale_mul).
 __host__ __device__ constexpr float offset_term(int fmt) {
   return fmt == MOE_FMT_INT4 ? -8.0f / 16777216.0f
          : fmt == MOE_FMT_INT3 ? -4.0f / 16777216.0f
-         : fmt == MOE_FMT_INT1 ? -1.0f / 16777216.0f
+         : fmt == MOE_FMT_INT1 ? -0.5f / 16777216.0f
                                : -2.0f / 16777216.0f;
 }
+__host__ __device__ constexpr float group_scale_mul(int fmt) { return fmt == MOE_FMT_INT1 ? 2.0f : 1.0f; }
 
 // Address of the 16-byte chunk of rows 4g..4g+3 in word-row z of a code box
 // (lines of 128 bytes: line = 2z + slice; 128-byte swizzle: chunk ^= line % 8).
@@ -262,11 +266,12 @@ __device__ __forceinline__ void group_mma(const uint8_t* box, const uint8_t* sc,
     }
   }
   const uint2 s4 = lds64(sc + kg * 256 + (32 * s + 4 * g) * 2);  // fp16 scales of rows 4g..4g+3
-  const float sr[4] = {half_lo(s4.x), half_hi(s4.x), half_lo(s4.y), half_hi(s4.y)};
+  constexpr float kSm = group_scale_mul(FMT);
+  const float sr[4] = {kSm * half_lo(s4.x), kSm * half_hi(s4.x), kSm * half_lo(s4.y), kSm * half_hi(s4.y)};
 #pragma unroll
   for (int nt = 0; nt < NT8; ++nt) {
     const uint4 xr = lds128(xs + nt * 2048);
-    const uint32_t b0 = FMT == MOE_FMT_INT1 ? hmul2(xr.x, act_mul(FMT, 0)) : xr.x, b1 = hmul2(xr.y, act_mul(FMT, 1));
+    const uint32_t b0 = xr.x, b1 = hmul2(xr.y, act_mul(FMT, 1));  // act_mul(FMT, 0) == 1
     const uint32_t b2 = FMT == MOE_FMT_INT4 ? xr.z : hmul2(xr.z, act_mul(FMT, 2));
     const uint32_t b3 = hmul2(xr.w, act_mul(FMT, 3));
     const float d0 = offset_term(FMT) * ldsf(gs + nt * 128), d1 = offset_term(FMT) * ldsf(gs + nt * 128 + 16);
@@ -415,9 +420,11 @@ __device__ __forceinline__ void load_item(ItemSrc<NMAT>& s, int it, int total, i
 
 // Epilogue of one output (row r, weight row n) from the matrices' sums v[m]
 // (integer formats: already multiplied by 2^24).  Gate/up returns h as stored
-// (fp16-rounded for integer layers), for the group sums of the down GEMV.
+// (fp16-rounded for integer layers), for the group sums of the down GEMV, and
+// sets `range` when that fp16 h overflowed.
 template <int NMAT>
-__device__ __forceinline__ float store_output(const GemvArgs& a, int r, int n, const float* v, const float* ts) {
+__device__ __forceinline__ float store_output(const GemvArgs& a, int r, int n, const float* v, const float* ts,
+                                              bool& range) {
   if (NMAT == 2) {
     float gv = v[0], uv = v[1];
     if (a.row_scale) {
@@ -428,7 +435,13 @@ __device__ __forceinline__ float store_output(const GemvArgs& a, int r, int n, c
       reinterpret_cast<float*>(a.out)[(size_t)r * a.N + n] = h;
       return h;
     }
+    if (a.xinv) {
+      const float xi = a.xinv[r];
+      gv *= xi;
+      uv *= xi;
+    }
     const __half h = __float2half_rn(__fdividef(gv, 1.0f + __expf(-gv)) * uv);
+    range |= __hisinf(h) != 0;
     reinterpret_cast<__half*>(a.out)[(size_t)r * a.N + n] = h;
     return __half2float(h);
   }
@@ -436,6 +449,11 @@ __device__ __forceinline__ float store_output(const GemvArgs& a, int r, int n, c
   if (a.row_scale) o *= a.row_scale[r] * ts[0];
   reinterpret_cast<float*>(a.out)[(size_t)r * a.N + n] = o;
   return o;
+}
+
+// Record an SwiGLU output beyond fp16 range (the first error is kept).
+__device__ __forceinline__ void report_range(int32_t* status) {
+  if (status) atomicCAS(status, 0, (int32_t)MOE_ERR_RANGE);
 }
 
 template <int NMAT, int NT8, bool I1>
@@ -595,6 +613,7 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
       }
       // lane outputs: weight row nl = 32s + 4g + 2t + (j >> 1), token row nt*8 + 2c + (j & 1)
       if (ok && a.P == 1) {
+        bool range = false;
 #pragma unroll
         for (int nt = 0; nt < NT8; ++nt) {
           float hs[2] = {0.0f, 0.0f};  // this lane's part of the group sums of h for tokens 2c, 2c+1
@@ -608,7 +627,7 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m) v[m] = acc[m][t][nt][j] * fscale[m];
                 hs[j & 1] += store_output<NMAT>(a, row0 + tk, w.nb * kBlockRows + 32 * s + 4 * g + 2 * t + (j >> 1),
-                                                v, ts);
+                                                v, ts, range);
               }
             }
           if (a.out_sum) {  // warp s owns the 32 weight rows of one down-projection input group
@@ -625,6 +644,7 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
             }
           }
         }
+        if (range) report_range(a.status);
       } else if (ok) {
 #pragma unroll
         for (int t = 0; t < 2; ++t)
@@ -678,7 +698,9 @@ __global__ void __launch_bounds__(256) gemv_fixup_kernel(GemvArgs a, const int32
       for (int q = 0; q < a.P; ++q) sum += a.part[(((size_t)q * a.R + r) * NMAT + m) * a.N + n];
       v[m] = sum;
     }
-    float h = store_output<NMAT>(a, r, n, v, ts);
+    bool range = false;
+    float h = store_output<NMAT>(a, r, n, v, ts, range);
+    if (range) report_range(a.status);
     if (a.out_sum) {
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) h += __shfl_xor_sync(0xffffffffu, h, o);
@@ -854,6 +876,7 @@ cudaError_t launch_expert_gemv(const uint8_t* packed, uint64_t packed_bytes, con
     act = ws.xs;
     sums = fp4 ? nullptr : ws.xsum;
     g.row_scale = fp4 ? ws.sx : nullptr;
+    g.xinv = fp4 ? nullptr : ws.xinv;
     g.out = ws.h;
     g.out_sum = fp4 ? nullptr : ws.hsum;
   } else {

@@ -140,6 +140,7 @@ struct Workspace {
   int counter_len;
   float* xsum;         // [T*k][H/32] group sums of the gathered fp16 activations (integer layers)
   float* hsum;         // [T*k][F/32] group sums of the fp16 SwiGLU outputs (integer layers)
+  float* xinv;         // [T*k] integer layers: 2^e undoing the power-of-two prescale of a row's x
 };
 
 }  // namespace moe

@@ -180,18 +180,51 @@ __device__ __forceinline__ void zero_counters(int32_t* counters, int n) {
   for (int i = threadIdx.x; i < n; i += blockDim.x) counters[i] = 0;
 }
 
+// Power-of-two prescale that brings a row with max |value| m into fp16 range:
+// 1 while m < 2^15, else 2^-e with m * 2^-e in [2^14, 2^15).  Scaling by a power
+// of two is exact (values far below m may round into the fp16 subnormals, an
+// error far below the row's largest term).
+__device__ __forceinline__ int prescale_exp(float m) {
+  if (!(m >= 32768.0f)) return 0;
+  return (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127 - 14;
+}
+
 // Gather x rows into expert-sorted order as fp16 (integer-format layers), with
 // the sum of every group of 32 fp16 values (fp32) for the decode GEMV's code
-// offset term (xsum may be null).  blockDim.x is a multiple of 32 and H of 128,
-// so the four threads of a group sit in one warp at every step.
-__global__ void gather_f16_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm,
-                                  int R, int H, int k, __half* __restrict__ xs, float* __restrict__ xsum,
-                                  int32_t* counters, int n_counters) {
+// offset term (xsum may be null).  bf16 covers a far wider range than fp16, so
+// a token whose max |x| reaches 2^15 is stored as x * 2^-e and its row's
+// xinv = 2^e restores the scale after the gate/up sums (xinv = 1 otherwise, and
+// the stored values are exactly fp16(x)).  blockDim.x is 128 and H a multiple
+// of 128, so the four threads of a group sit in one warp at every step.
+__global__ void __launch_bounds__(128) gather_f16_kernel(const __nv_bfloat16* __restrict__ x,
+                                                         const int32_t* __restrict__ perm, int R, int H, int k,
+                                                         __half* __restrict__ xs, float* __restrict__ xsum,
+                                                         float* __restrict__ xinv, int32_t* counters,
+                                                         int n_counters) {
+  __shared__ float s_max[4];
   if (blockIdx.x == 0 && blockIdx.y == 0) zero_counters(counters, n_counters);
   const int r = blockIdx.x;
   const int t = perm[r] / k;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
   uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)r * H);
+  // max |x| of the whole token row (every column block reads it; the second
+  // block's reads hit the cache)
+  float m = 0.0f;
+  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
+    const uint4 v = __ldg(src + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      m = fmaxf(m, fmaxf(__uint_as_float((w[i] << 16) & 0x7FFF0000u), __uint_as_float(w[i] & 0x7FFF0000u)));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
+  const int e = prescale_exp(m);
+  const float sc = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e (e <= 114)
+  if (xinv && blockIdx.y == 0 && threadIdx.x == 0) xinv[r] = __uint_as_float((uint32_t)(127 + e) << 23);
   for (int c = blockIdx.y * blockDim.x + threadIdx.x; c < H / 8; c += gridDim.y * blockDim.x) {
     const uint4 v = __ldg(src + c);
     const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v);
@@ -200,9 +233,14 @@ __global__ void gather_f16_kernel(const __nv_bfloat16* __restrict__ x, const int
     float sum = 0.0f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      h2[i] = __float22half2_rn(__bfloat1622float2(b2[i]));
-      const float2 f = __half22float2(h2[i]);
-      sum += f.x + f.y;
+      float2 f = __bfloat1622float2(b2[i]);
+      if (e) {
+        f.x *= sc;
+        f.y *= sc;
+      }
+      h2[i] = __float22half2_rn(f);
+      const float2 g = __half22float2(h2[i]);
+      sum += g.x + g.y;
     }
     dst[c] = o;
     const unsigned act = __activemask();  // whole groups of four lanes (H/8 is a multiple of 16)
@@ -337,8 +375,8 @@ cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4,
   } else {
     int ny = R < 512 ? (H / 8 + 127) / 128 : 1;  // column blocks: more parallelism for few rows
     if (ny > 8) ny = 8;
-    gather_f16_kernel<<<dim3(R, ny), 128, 0, stream>>>(x, ws.perm, R, H, k, (__half*)ws.xs, ws.xsum, ws.counters,
-                                                       ws.counter_len);
+    gather_f16_kernel<<<dim3(R, ny), 128, 0, stream>>>(x, ws.perm, R, H, k, (__half*)ws.xs, ws.xsum, ws.xinv,
+                                                       ws.counters, ws.counter_len);
   }
   return cudaGetLastError();
 }

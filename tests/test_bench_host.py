@@ -19,10 +19,10 @@ def test_code_hash_ignores_comments_and_layout_only():
 
 def test_traffic_summary_matches_or_is_null():
     # the summary is used only when its hash equals the current sources'; otherwise null
-    t = bench.ncu_traffic("gateup_prefill_mixtral")
+    t = bench.ncu_traffic("gateup_prefill_large")
     import json
     d = json.load(open(bench.TRAFFIC_FILE))
     if d["csrc_hash"] == bench.csrc_hash():
-        assert t == d["kernels"]["gateup_prefill_mixtral"]["dram_bytes_per_launch"]
+        assert t == d["kernels"]["gateup_prefill_large"]["dram_bytes_per_launch"]
     else:
         assert t is None

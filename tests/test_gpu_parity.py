@@ -95,13 +95,15 @@ def check_layer(L, T, tokens=None, bias=None, router_zero=False, max_ties=None):
         np.testing.assert_array_equal(g["xq"].reshape(T, L.H), xq)
         np.testing.assert_array_equal(g["sx"], sx)
 
+    if callable(tokens):
+        tokens = tokens(g["perm"], g["counts"], k)
     tokens = np.arange(T) if tokens is None else np.asarray(tokens)
     experts = np.unique(np.concatenate([idx_o[tokens].ravel(), idx_g[tokens].ravel()]))
     buf = hp.oracle_pack(L, experts)
     y_ref, _, _ = hp.oracle_forward_rows(buf, x_bits, Wr_h, b_h, k, tokens=tokens,
                                          idx_override=idx_g if ties else None, fp4=L.fp4)
     ratio = hp.check_output(g["y"][torch.from_numpy(tokens).cuda()], y_ref)
-    return dict(ties=len(ties), err_ratio=ratio, counts=g["counts"])
+    return dict(ties=len(ties), err_ratio=ratio, counts=g["counts"], n_tokens=len(tokens))
 
 
 # ------------------------------------------------------------------ generator / packing
@@ -399,6 +401,60 @@ def test_forward_zero_expert():
     hp.check_output(g["y"], y_ref)
 
 
+def _x_device(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+@pytest.mark.parametrize("T", [9, 600])
+def test_forward_x_beyond_fp16_range(T):
+    # bf16 x reaches far beyond fp16.  Planted |x| of 1e5, 3e6 and 131008 in column 17 of three
+    # tokens: those tokens' rows are prescaled by a power of two before the fp16 conversion and
+    # rescaled after the gate/up sums.  Inputs 0..31 (the quantization group of column 17) of
+    # every gate, up and router row are zero, so the group scales are 0 (the 1-bit sign code has
+    # no zero code) and the SwiGLU outputs and routing stay ordinary.  1-bit matrices are
+    # included (their decode path once doubled the activations).  T=9 runs the decode GEMV,
+    # T=600 the tcgen05 GEMMs.
+    E, H, F, k = 6, 256, 256, 2
+    fmt = np.array([[4, 4, 4], [2, 2, 2], [1, 1, 1], [4, 2, 1], [1, 2, 4], [3, 3, 3]], np.uint8)
+    Wh = np.stack([W.expert_w(e, H, F) for e in range(E)])
+    Wh[:, 0].reshape(E, F, H)[:, :, :32] = 0.0
+    Wh[:, 1].reshape(E, F, H)[:, :, :32] = 0.0
+    layer_fmt = fmt.reshape(-1)
+    packed = moe.alloc_packed(moe.pack_layout(E, H, F, layer_fmt)[0])
+    moe.moe_pack(torch.from_numpy(Wh).cuda(), 0, E, H, F, layer_fmt, packed)
+    layer = moe.PackedLayer(E, H, F, layer_fmt, packed)
+    Wr_h = W.router_w(E, H)
+    Wr_h[:, :32] = 0.0
+    x_bits = W.x_bf16_bits(T, H).copy()
+    big = {0: 1e5, 3: -3e6, T - 1: 65504.0 * 2}
+    for t, v in big.items():
+        x_bits[t, 17] = gen.f32_to_bf16_bits(np.array([v], np.float32))[0]
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = moe.moe_layer_forward(_x_device(x_bits), torch.from_numpy(Wr_h).cuda(), None, layer, k,
+                              debug={"status": st})
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    buf = orc.pack_layer(Wh, 0, E, H, F, layer_fmt)
+    y_ref, _, _ = hp.oracle_forward_rows(buf, x_bits, Wr_h, None, k)
+    hp.check_output(y, y_ref)
+
+
+@pytest.mark.parametrize("T", [9, 600])
+def test_swiglu_overflow_reports_range(T):
+    # x at 3000 sigma: h = silu(g) * u lands far beyond fp16 in an integer layer, which stores h
+    # in fp16.  The call must write MOE_ERR_RANGE to the status word, and the next ordinary call
+    # on the same context must be clean and exact.
+    L = custom("hrange", T, 256, 256, 4, 2, [[4, 4, 4], [3, 2, 4], [2, 2, 2], [4, 3, 1]])
+    layer = hp.gpu_pack(L)
+    x = W.device_x(T, L.H) * 3000.0
+    Wr, b = W.device_router(L)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    moe.moe_layer_forward(x, Wr, b, layer, L.k, debug={"status": st})
+    torch.cuda.synchronize()
+    assert _lib.STATUS[int(st.item())] == "MOE_ERR_RANGE"
+    check_layer(L, T)
+
+
 def test_forward_deterministic_and_empty_batch():
     L = W.layer("tiny")
     layer = hp.gpu_pack(L)
@@ -453,12 +509,38 @@ def test_stage_events_record():
 
 
 # ------------------------------------------------------------------ forward, the five layers
+def strata(halves=True, extra=0, seed=0):
+    """Token sample for a full-size batch, taken from the GPU's own permutation: for every
+    expert, every 256-row chunk the tcgen05 GEMM walks, and (halves) each half of a chunk's
+    rows (the two CTAs of a pair), the tokens of the first and last row; plus `extra` seeded
+    random tokens.  Every expert with rows is compared, at the chunk and CTA-half edges where
+    offset or ragged-tail mistakes would show."""
+    def pick(perm, counts, k):
+        T = len(perm) // k
+        rows, off = [], 0
+        for c in counts:
+            c = int(c)
+            for c0 in range(0, c, 256):
+                n = min(256, c - c0)
+                nmma = min(256, (n + 15) // 16 * 16)
+                parts = [(0, min(n, nmma // 2)), (nmma // 2, n)] if halves else [(0, n)]
+                for a, b in parts:
+                    if b > a:
+                        rows += [off + c0 + a, off + c0 + b - 1]
+            off += c
+        tok = set(int(perm[r]) // k for r in rows)
+        if extra:
+            tok |= set(np.random.default_rng(seed).choice(T, min(T, extra), replace=False).tolist())
+        return np.array(sorted(tok))
+    return pick
+
+
 CONFIG_RUNS = [
     ("mixtral", 1, None), ("mixtral", 8, None), ("mixtral", 64, None),
-    ("hotcold", 32, None), ("nvfp4", 16, None), ("large", 64, [0, 1, 2, 63]),
-    ("mixtral", 2048, [0, 1, 1000, 2047]), ("hotcold", 4096, [0, 4095]),
-    ("nvfp4", 8192, [0, 8191]), ("large", 8192, [0, 8191]),
-    ("graded", 32, None), ("graded", 4096, [0, 1, 2047, 4095]),
+    ("hotcold", 32, None), ("nvfp4", 16, None), ("large", 64, None),
+    ("mixtral", 2048, strata(extra=200)), ("hotcold", 4096, strata(extra=256)),
+    ("nvfp4", 8192, strata(extra=256)), ("large", 8192, strata(halves=False, extra=16)),
+    ("graded", 32, None), ("graded", 4096, strata(extra=128)),
 ]
 
 
@@ -466,4 +548,4 @@ CONFIG_RUNS = [
 def test_forward_config(name, T, tokens):
     L = W.layer(name)
     r = check_layer(L, T, tokens=tokens)
-    print(f"{name} T={T}: near-ties {r['ties']}, err/max {r['err_ratio']:.3g}")
+    print(f"{name} T={T}: near-ties {r['ties']}, err/max {r['err_ratio']:.3g}, tokens compared {r['n_tokens']}")
