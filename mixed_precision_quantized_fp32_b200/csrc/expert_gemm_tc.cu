@@ -145,17 +145,18 @@ __device__ __forceinline__ void e2m1x8_to_f16(uint32_t w, uint32_t* o) {
 }
 
 // Eight inputs (chunk c = inputs 8c..8c+7 of the staged group) of weight row n
-// as four fp16 pairs in natural order.  codes: the group's words [word][128
-// rows]; scales: [128] fp16 (integer) or [2 blocks][128] e4m3 (NVFP4).  The
-// format is a template parameter so a stage's chunks are straight-line code.
+// as four fp16 pairs in natural order.  codes: shared address of the group's
+// words [word][128 rows]; scales: shared address of [128] fp16 (integer) or
+// [2 blocks][128] e4m3 (NVFP4).  The format is a template parameter so a
+// stage's chunks are straight-line code.
 template <int FMT>
-__device__ __forceinline__ uint4 dequant_chunk(const uint32_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                                              int n, int c) {
+__device__ __forceinline__ uint4 dequant_chunk(uint32_t codes, uint32_t scales, int n, int c) {
   uint32_t v[4];
   if (FMT == MOE_FMT_NVFP4) {
-    const __half_raw sr = __nv_cvt_fp8_to_halfraw(scales[(c >> 1) * 128 + n], __NV_E4M3);  // exact
+    const __half_raw sr =
+        __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)ptx::lds_u8(scales + (c >> 1) * 128 + n), __NV_E4M3);  // exact
     const uint32_t p = (uint32_t)sr.x | ((uint32_t)sr.x << 16);
-    e2m1x8_to_f16(codes[c * 128 + n], v);
+    e2m1x8_to_f16(ptx::lds_u32(codes + 4 * (c * 128 + n)), v);
 #pragma unroll
     for (int b = 0; b < 4; ++b) v[b] = h2mul(v[b], p);  // exact: <= 6 significant bits
   } else {
@@ -163,7 +164,7 @@ __device__ __forceinline__ uint4 dequant_chunk(const uint32_t* __restrict__ code
     // the mantissa of 1024.0 reads as 1024 + f*u; one FMA with 1/f and
     // -(1024/f + offset) gives q = u - offset exactly, then one multiply by the
     // group scale rounds s*q once.
-    const uint32_t s = reinterpret_cast<const uint16_t*>(scales)[n];
+    const uint32_t s = ptx::lds_u16(scales + 2 * n);
     const uint32_t s2 = s | (s << 16);
     constexpr uint32_t kMagic = 0x64006400u;
     if (FMT == MOE_FMT_INT1) {
@@ -172,13 +173,13 @@ __device__ __forceinline__ uint4 dequant_chunk(const uint32_t* __restrict__ code
       // gives s*(2u - 1) = +-s in one rounding
       constexpr uint32_t kMul1[4] = {0x3C003C00u, 0x38003800u, 0x34003400u, 0x30003000u};  // 2^-j
       constexpr uint32_t kSub1[4] = {0xE400E400u, 0xE000E000u, 0xDC00DC00u, 0xD800D800u};  // -1024*2^-j
-      const uint32_t w = codes[n] >> (4 * c);
+      const uint32_t w = ptx::lds_u32(codes + 4 * n) >> (4 * c);
       const uint32_t s2x2 = h2mul(s2, 0x40004000u), neg_s2 = s2 ^ 0x80008000u;
 #pragma unroll
       for (int j = 0; j < 4; ++j)
         v[j] = h2fma(h2fma((w & (0x00010001u << j)) | kMagic, kMul1[j], kSub1[j]), s2x2, neg_s2);
     } else if (FMT == MOE_FMT_INT4) {
-      const uint32_t w = codes[c * 128 + n], w8 = w >> 8;
+      const uint32_t w = ptx::lds_u32(codes + 4 * (c * 128 + n)), w8 = w >> 8;
       v[0] = h2mul(h2fma((w & 0x000F000Fu) | kMagic, 0x3C003C00u, 0xE408E408u), s2);   // u - 8
       v[1] = h2mul(h2fma((w & 0x00F000F0u) | kMagic, 0x2C002C00u, 0xD480D480u), s2);   // 16u / 16 + 64 - 72
       v[2] = h2mul(h2fma((w8 & 0x000F000Fu) | kMagic, 0x3C003C00u, 0xE408E408u), s2);
@@ -190,10 +191,10 @@ __device__ __forceinline__ uint4 dequant_chunk(const uint32_t* __restrict__ code
       constexpr uint32_t kMul[4] = {0x3C003C00u, 0x34003400u, 0x2C002C00u, 0x24002400u};        // 4^-j
       constexpr uint32_t kSub2[4] = {0xE402E402u, 0xDC08DC08u, 0xD420D420u, 0xCC80CC80u};       // -(1024/4^j + 2)
       constexpr uint32_t kSub3[4] = {0xE404E404u, 0xDC10DC10u, 0xD440D440u, 0xCD00CD00u};       // -(1024/4^j + 4)
-      const uint32_t lo = codes[(c >> 1) * 128 + n] >> (8 * (c & 1));
+      const uint32_t lo = ptx::lds_u32(codes + 4 * ((c >> 1) * 128 + n)) >> (8 * (c & 1));
       uint32_t hh = 0u;
       if (FMT == MOE_FMT_INT3) {
-        const uint32_t hw = codes[2 * 128 + n];
+        const uint32_t hw = ptx::lds_u32(codes + 4 * (2 * 128 + n));
         hh = __funnelshift_r(hw, hw, (uint32_t)(8 * (c >> 1) + (c & 1) + 30) & 31u);
       }
 #pragma unroll
@@ -235,7 +236,7 @@ __device__ __forceinline__ uint64_t scale_stage_offset(int mt, int g, int K, int
 // them to the tensor core and release the stage to the MMA warp.  Returns
 // false if a bounded wait gave up.
 template <int NMAT, bool CG2, int F0, int F1>
-__device__ __noinline__ bool dequant_item(const Ring R, long long wait, uint8_t* smem, uint64_t* load_full,
+__device__ __noinline__ bool dequant_item(const Ring R, long long wait, uint32_t smem, uint64_t* load_full,
                                           uint64_t* a_full, volatile int* abort_flag, int ksteps, int n, int u0,
                                           int& stage, uint32_t& phase, int& gstage, unsigned long long* trace) {
   using C = TcCfg<NMAT, CG2>;
@@ -246,25 +247,24 @@ __device__ __noinline__ bool dequant_item(const Ring R, long long wait, uint8_t*
   for (int ks = 0; ks < ksteps; ++ks) {
     if (!__all_sync(0xffffffffu, ptx::mbar_wait(&load_full[stage], phase, abort_flag, wait))) return false;
     if (threadIdx.x == 0) trace_stamp(trace, 2, gstage);
-    uint8_t* sb = smem + stage * R.stage_bytes;
+    const uint32_t sb = smem + (uint32_t)(stage * R.stage_bytes);  // shared address of the stage
     uint4 v[kUnits];
 #pragma unroll
     for (int i = 0; i < kUnits; ++i) {
       const int m = i % NMAT, cg = cg0 + i / NMAT, g = cg >> 2;
-      const uint8_t* scales = sb + R.off_scales + m * C::kScaleBytes + g * 256;
+      const uint32_t scales = sb + (uint32_t)(R.off_scales + m * C::kScaleBytes + g * 256);
       if (m == 0) {
-        const uint32_t* codes = reinterpret_cast<const uint32_t*>(sb + C::kOffCodes) + g * fmt_words(F0) * 128;
+        const uint32_t codes = sb + (uint32_t)(C::kOffCodes + g * fmt_words(F0) * 512);
         v[i] = dequant_chunk<F0>(codes, scales, n, cg & 3);
       } else {
-        const uint32_t* codes = reinterpret_cast<const uint32_t*>(sb + C::kOffCodes + R.code_bytes) +
-                                g * fmt_words(F1) * 128;
+        const uint32_t codes = sb + (uint32_t)(C::kOffCodes + R.code_bytes + g * fmt_words(F1) * 512);
         v[i] = dequant_chunk<F1>(codes, scales, n, cg & 3);
       }
     }
 #pragma unroll
     for (int i = 0; i < kUnits; ++i) {
       const int m = i % NMAT, cg = cg0 + i / NMAT;
-      *reinterpret_cast<uint4*>(sb + C::kOffA + m * C::kABytes + tile_offset(n, cg)) = v[i];
+      ptx::sts_v4(sb + (uint32_t)(C::kOffA + m * C::kABytes + tile_offset(n, cg)), v[i]);
     }
     ptx::fence_proxy_async_smem();
     __syncwarp();
@@ -288,7 +288,7 @@ __device__ __noinline__ bool dequant_item(const Ring R, long long wait, uint8_t*
 // meets 1-bit matrices; their cases are compiled only into the I1 kernels, so the
 // kernels for layers without them keep their size and register allocation.
 template <int NMAT, bool CG2, bool I1, int F0>
-__device__ __forceinline__ bool dequant_item_f1(int f1, const Ring R, long long wait, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
+__device__ __forceinline__ bool dequant_item_f1(int f1, const Ring R, long long wait, uint32_t smem, uint64_t* load_full, uint64_t* a_full,
                                                 volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
                                                 uint32_t& phase, int& gstage, unsigned long long* trace) {
   if (NMAT == 1) return dequant_item<NMAT, CG2, F0, F0>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
@@ -303,7 +303,7 @@ __device__ __forceinline__ bool dequant_item_f1(int f1, const Ring R, long long 
   }
 }
 template <int NMAT, bool CG2, bool I1>
-__device__ __forceinline__ bool dequant_item_any(int f0, int f1, const Ring R, long long wait, uint8_t* smem, uint64_t* load_full, uint64_t* a_full,
+__device__ __forceinline__ bool dequant_item_any(int f0, int f1, const Ring R, long long wait, uint32_t smem, uint64_t* load_full, uint64_t* a_full,
                                                  volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
                                                  uint32_t& phase, int& gstage, unsigned long long* trace) {
   if constexpr (I1) {
@@ -322,7 +322,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
   using C = TcCfg<NMAT, CG2>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  // 1024-byte aligned base, derived from the shared array by pointer arithmetic (an
+  // integer round trip would turn every access through it into a generic one)
+  uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
   const Ring R = a.ring;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + R.stages * R.stage_bytes);
   uint64_t* load_full = bars;
@@ -539,7 +541,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         fmt[m] = L.fmt[i];
         tsc[m] = fmt[m] == MOE_FMT_NVFP4 ? L.tscale[i] : 1.0f;
       }
-      if (!dequant_item_any<NMAT, CG2, I1>(fmt[0], fmt[NMAT - 1], a.ring, a.wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage,
+      if (!dequant_item_any<NMAT, CG2, I1>(fmt[0], fmt[NMAT - 1], a.ring, a.wait, ptx::smem_u32(smem), load_full, a_full, abort_flag, ksteps, n, u0, stage,
                                   phase, gstage, a.trace)) {
         ok = false;
         break;

@@ -112,10 +112,11 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       "l"((uint64_t)map), "r"(x), "r"(y), "r"(z), "r"(ptx::smem_u32(bar))
       : "memory");
 }
-__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
-__device__ __forceinline__ uint2 lds64(const uint8_t* p) { return *reinterpret_cast<const uint2*>(p); }
-__device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
-__device__ __forceinline__ float ldsf(const uint8_t* p) { return *reinterpret_cast<const float*>(p); }
+// shared-space loads through 32-bit shared addresses
+__device__ __forceinline__ uint4 lds128(uint32_t a) { return ptx::lds_v4(a); }
+__device__ __forceinline__ uint2 lds64(uint32_t a) { return ptx::lds_v2(a); }
+__device__ __forceinline__ uint32_t lds32(uint32_t a) { return ptx::lds_u32(a); }
+__device__ __forceinline__ float ldsf(uint32_t a) { return ptx::lds_f32(a); }
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsumers) : "memory"); }
 
 // Bounded wait that ignores the abort flag (used to drain copies before exit).
@@ -173,19 +174,20 @@ __host__ __device__ constexpr float group_scale_mul(int fmt) { return fmt == MOE
 
 // Address of the 16-byte chunk of rows 4g..4g+3 in word-row z of a code box
 // (lines of 128 bytes: line = 2z + slice; 128-byte swizzle: chunk ^= line % 8).
-__device__ __forceinline__ const uint8_t* code_chunk(const uint8_t* box, int z, int y, int g) {
+__device__ __forceinline__ uint32_t code_chunk(uint32_t box, int z, int y, int g) {
   const int line = 2 * z + y;
-  return box + line * 128 + ((g ^ (line & 7)) << 4);
+  return box + (uint32_t)(line * 128 + ((g ^ (line & 7)) << 4));
 }
 
 // One group (kg) of one matrix: unpack the lane's rows, run the MMAs for every
-// token tile and accumulate.  box: this warp's code box; sc: the matrix's scale
-// tile; xs: the lane's 16 activation bytes of the group in token tile 0 (token
-// tiles follow at 8 rows x 256 bytes); gs: the group sum of token 2c in token
-// tile 0 (token 2c+1 follows at +16 bytes, tile nt at nt * 128 bytes).
+// token tile and accumulate.  All addresses are shared-window addresses.  box:
+// this warp's code box; sc: the matrix's scale tile; xs: the lane's 16
+// activation bytes of the group in token tile 0 (token tiles follow at 8 rows x
+// 256 bytes); gs: the group sum of token 2c in token tile 0 (token 2c+1 follows
+// at +16 bytes, tile nt at nt * 128 bytes).
 template <int FMT, int NT8>
-__device__ __forceinline__ void group_mma(const uint8_t* box, const uint8_t* sc, int kg, int y, int s, int g, int c,
-                                          const uint8_t* xs, const uint8_t* gs, float (&acc)[2][NT8][4]) {
+__device__ __forceinline__ void group_mma(uint32_t box, uint32_t sc, int kg, int y, int s, int g, int c,
+                                          uint32_t xs, uint32_t gs, float (&acc)[2][NT8][4]) {
   uint32_t p[4][4];   // [row i][pair j]
   if (FMT == MOE_FMT_NVFP4) {
     const uint4 w = lds128(code_chunk(box, 4 * kg + c, y, g));
@@ -306,11 +308,11 @@ __device__ __forceinline__ void consume_tiles(const StageLayout& L, uint8_t* sme
       ok = false;
     if (threadIdx.x == 0) gtrace(tr, 2, gtile);
     if (ok) {
-      const uint8_t* sb = smem + stage * L.bytes;
+      const uint32_t sb = ptx::smem_u32(smem) + (uint32_t)(stage * L.bytes);
 #pragma unroll
       for (int kg = 0; kg < 4; ++kg) {
-        const uint8_t* xs = sb + L.x_off + g * 256 + (32 * kg + 8 * c) * 2;
-        const uint8_t* gs = sb + L.sum_off + (2 * c) * 16 + kg * 4;
+        const uint32_t xs = sb + (uint32_t)(L.x_off + g * 256 + (32 * kg + 8 * c) * 2);
+        const uint32_t gs = sb + (uint32_t)(L.sum_off + (2 * c) * 16 + kg * 4);
         group_mma<F0, NT8>(sb + L.code_off[0] + (s >> 1) * L.box[0], sb + L.scale_off[0], kg, s & 1, s, g, c, xs,
                            gs, acc[0]);
         if (NMAT == 2)
@@ -465,7 +467,8 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
                                                                    const __grid_constant__ CUtensorMap tm_s,
                                                                    const GemvArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  // 1024-byte aligned base, derived from the shared array by pointer arithmetic
+  uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
   const StageLayout& SL = a.st;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SL.stages * SL.bytes);
   uint64_t* empty = full + kMaxStages;
