@@ -60,7 +60,7 @@ Plan make_plan(int T, int k, int E) {
   const long long active = R < E ? R : E;
   const long long avg = active > 0 ? (R + active - 1) / active : 0;
   p.tc = avg > 32 && R >= 256;
-  p.chunk_rows = p.tc ? 256 : 8;
+  p.chunk_rows = p.tc ? kTcChunkRows : 8;
   p.max_chunks = (int)(E + (R + p.chunk_rows - 1) / p.chunk_rows);
   return p;
 }

@@ -9,16 +9,20 @@
 //   * persistent clusters of two CTAs (one CTA per SM) walk (token chunk, weight
 //     tiles) work items; chunk = up to 256 consecutive expert-sorted rows of one
 //     expert; each CTA owns 128-row weight tiles (gate + up, or two down tiles);
-//   * warp 16 (one lane) streams each 64-input stage (two quantization groups):
-//     this CTA's half of the chunk's token rows with a 2D TMA load (128-byte
-//     swizzle) and the packed codes + scales of its weight tiles with 1D bulk
-//     copies (never multicast); the ring is as deep as the widest code format
-//     of the launch allows;
+//   * two rings of shared-memory slots per CTA: raw slots hold a stage's packed
+//     codes + scales (64 inputs = two quantization groups) and are freed as soon
+//     as they are dequantized, so their copies run many stages ahead; operand
+//     slots hold the activation tile and the dequantized weight tiles the tensor
+//     core reads, and are freed by the MMA commit;
+//   * warp 16 (one lane) streams the codes and scales of this CTA's weight tiles
+//     into the raw ring with 1D bulk copies; warp 18 (one lane) loads this CTA's
+//     half of the chunk's token rows into the operand ring with a 2D TMA load
+//     (128-byte swizzle); no copy is multicast;
 //   * warps 0-15 turn codes into fp16 operands (exponent-bias unpack: a code u
 //     OR'ed into the mantissa of 1024.0 gives 1024+u exactly; one subtract
-//     and one multiply by the group scale) written straight into the swizzled
-//     K-major layout the tensor core reads, then arrive on the even CTA's
-//     barrier;
+//     and one multiply by the group scale), release the raw slot, and write
+//     the operands straight into the swizzled K-major layout the tensor core
+//     reads, then arrive on the even CTA's barrier;
 //   * warp 17 of the even CTA (one lane) issues tcgen05.mma.cta_group::2
 //     M=256 (128 weight rows from each CTA) x N<=256 (token rows, half from
 //     each CTA) x K=16 and commits to both CTAs' mbarriers;
@@ -42,7 +46,7 @@ namespace moe {
 namespace {
 
 constexpr int kTcBM = 128;   // weight rows per work item (MMA M)
-constexpr int kTcBN = 256;   // token rows per work item (max MMA N)
+constexpr int kTcBN = kTcChunkRows;  // token rows per work item (max MMA N)
 #ifndef MOE_TC_BK
 #define MOE_TC_BK 64
 #endif
@@ -56,16 +60,19 @@ static_assert(kTcBK == 32 || kTcBK == 64, "stage depth");
 constexpr int kDeqWarps = MOE_TC_DEQ_WARPS;  // dequantize + epilogue warps (8 or 16)
 static_assert(kDeqWarps == 8 || kDeqWarps == 16, "dequant warps");
 constexpr int kThreadsPerRow = kDeqWarps * 32 / 128;
-constexpr int kTmaWarp = kDeqWarps, kMmaWarp = kDeqWarps + 1;
-constexpr int kTcThreads = 32 * (kDeqWarps + 2);
+constexpr int kRawWarp = kDeqWarps, kMmaWarp = kDeqWarps + 1, kBWarp = kDeqWarps + 2;
+constexpr int kTcThreads = 32 * (kDeqWarps + 3);
 constexpr long long kWaitLimit = 4000000000LL;  // clock cycles, ~2 s
-constexpr int kPrefetchAhead = 4;                 // stages of packed codes warmed in L2 ahead of their copy
 
 // CG2: the work item runs on a pair of CTAs (one cluster) with cta_group::2
 // MMAs, each CTA holding half of the activation tile's token rows.
-// Stage layout: activation tile, NMAT dequantized weight tiles, NMAT code slots,
-// NMAT scale slots.  The code slot is sized for the widest format the launch
-// meets (Ring), so narrow layers get a deeper ring.
+// Two rings per CTA:
+//  * raw slots: the packed codes and scales of NMAT weight tiles for one stage,
+//    freed as soon as the dequant warps have read them, so copies run many
+//    stages ahead;
+//  * operand slots: the activation tile and the NMAT dequantized weight tiles
+//    the tensor core reads, freed by the MMA commit.
+// The code slot is sized for the widest format the launch meets (Ring).
 template <int NMAT, bool CG2 = false>
 struct TcCfg {
   static constexpr int kBRows = CG2 ? kTcBN / 2 : kTcBN;
@@ -74,31 +81,33 @@ struct TcCfg {
   static constexpr int kScaleBytes = kGroups * 256;   // one fp16 group or two e4m3 blocks x 128 rows
   static constexpr int kOffB = 0;
   static constexpr int kOffA = kBBytes;
-  static constexpr int kOffCodes = kOffA + NMAT * kABytes;
+  static constexpr int kOpBytes = kBBytes + NMAT * kABytes;  // one operand slot (a multiple of 1024)
 };
-constexpr int kMaxStages = 8;
-constexpr int kBarBytes = 256;                       // 3 barriers per stage + 2 + TMEM slot + flag
+constexpr int kMaxRaw = 16, kMaxOp = 4;
+constexpr int kBarBytes = 512;                       // barriers, TMEM slot and abort flag
 constexpr int kSmemMax = 232448;                     // opt-in shared memory per CTA
-static_assert(3 * 8 * kMaxStages + 32 <= kBarBytes, "barrier area");
+static_assert(8 * (2 * kMaxRaw + 3 * kMaxOp + 2) + 16 <= kBarBytes, "barrier area");
 
 struct Ring {
-  int stages;       // stages in the ring (<= kMaxStages)
-  int stage_bytes;  // one stage, a multiple of 1024
+  int op_slots;     // operand slots (<= kMaxOp)
+  int raw_slots;    // raw slots (<= kMaxRaw)
   int code_bytes;   // one matrix's code slot: kGroups x 512 bytes per code word of the widest format
-  int off_scales;   // scale slots
+  int raw_bytes;    // one raw slot: NMAT code slots, then NMAT scale slots
+  int off_raw;      // offset of the raw ring (after the operand slots)
 };
 
 template <int NMAT, bool CG2>
 Ring make_ring(int max_words) {
   using C = TcCfg<NMAT, CG2>;
   Ring r;
+  r.op_slots = CG2 ? 3 : 2;
   r.code_bytes = kGroups * 512 * max_words;
-  r.off_scales = C::kOffCodes + NMAT * r.code_bytes;
-  r.stage_bytes = (r.off_scales + NMAT * C::kScaleBytes + 1023) / 1024 * 1024;
-  r.stages = min(kMaxStages, (kSmemMax - kBarBytes - 1024) / r.stage_bytes);
+  r.raw_bytes = (NMAT * (r.code_bytes + C::kScaleBytes) + 127) / 128 * 128;
+  r.off_raw = r.op_slots * C::kOpBytes;
+  r.raw_slots = min(kMaxRaw, (kSmemMax - kBarBytes - 1024 - r.off_raw) / r.raw_bytes);
   return r;
 }
-inline int ring_smem(const Ring& r) { return r.stages * r.stage_bytes + kBarBytes + 1024; }
+inline int ring_smem(const Ring& r) { return r.off_raw + r.raw_slots * r.raw_bytes + kBarBytes + 1024; }
 
 struct TcArgs {
   const uint8_t* packed;
@@ -231,89 +240,128 @@ __device__ __forceinline__ uint64_t scale_stage_offset(int mt, int g, int K, int
   return ((uint64_t)mt * (uint64_t)(K >> 5) + (uint64_t)g) * 256u;
 }
 
+// Position of a role in the two rings: raw slot and phase, operand slot and
+// phase, and the global stage counter (trace index).
+struct Cursor {
+  int rs;
+  uint32_t rph;
+  int os;
+  uint32_t oph;
+  int g;
+};
+
 // Dequantize every stage of one work item (formats F0 = first matrix, F1 =
-// second): wait for the stage's codes, convert this thread's units, publish
-// them to the tensor core and release the stage to the MMA warp.  Returns
-// false if a bounded wait gave up.
+// second): wait for the stage's codes in a raw slot, convert this thread's units
+// to registers and release the raw slot, wait for the operand slot to be free
+// (its previous MMAs done) and this CTA's activation tile to land, write the
+// units in the tensor core's layout and arrive on the operand slot's barrier
+// (the even CTA's, for a pair).  Returns false if a bounded wait gave up.
 template <int NMAT, bool CG2, int F0, int F1>
-__device__ __noinline__ bool dequant_item(const Ring R, long long wait, uint32_t smem, uint64_t* load_full,
-                                          uint64_t* a_full, volatile int* abort_flag, int ksteps, int n, int u0,
-                                          int& stage, uint32_t& phase, int& gstage, unsigned long long* trace) {
+__device__ __noinline__ bool dequant_item(const Ring R, long long wait, uint32_t smem, uint64_t* bars,
+                                          volatile int* abort_flag, int ksteps, int n, int u0, Cursor& cursor,
+                                          unsigned long long* trace) {
   using C = TcCfg<NMAT, CG2>;
   constexpr int kUnits = NMAT * kGroups * 4 / kThreadsPerRow;
   static_assert(NMAT == 1 || kUnits % 2 == 0, "units must alternate matrices evenly");
+  uint64_t* raw_full = bars;
+  uint64_t* raw_empty = bars + kMaxRaw;
+  uint64_t* b_full = bars + 2 * kMaxRaw;
+  uint64_t* a_full = b_full + kMaxOp;
+  uint64_t* op_empty = a_full + kMaxOp;
   const int lane = threadIdx.x & 31;
   const int cg0 = u0 / NMAT;
+  // the cursor lives in registers for the loop (a reference would be re-read after every
+  // shared-memory store)
+  int rs = cursor.rs, os = cursor.os, g = cursor.g;
+  uint32_t rph = cursor.rph, oph = cursor.oph;
+  bool ok = true;
   for (int ks = 0; ks < ksteps; ++ks) {
-    if (!__all_sync(0xffffffffu, ptx::mbar_wait(&load_full[stage], phase, abort_flag, wait))) return false;
-    if (threadIdx.x == 0) trace_stamp(trace, 2, gstage);
-    const uint32_t sb = smem + (uint32_t)(stage * R.stage_bytes);  // shared address of the stage
+    if (!__all_sync(0xffffffffu, ptx::mbar_wait(&raw_full[rs], rph, abort_flag, wait))) {
+      ok = false;
+      break;
+    }
+    if (threadIdx.x == 0) trace_stamp(trace, 2, g);
+    const uint32_t rb = smem + (uint32_t)(R.off_raw + rs * R.raw_bytes);  // shared address of the raw slot
     uint4 v[kUnits];
 #pragma unroll
     for (int i = 0; i < kUnits; ++i) {
-      const int m = i % NMAT, cg = cg0 + i / NMAT, g = cg >> 2;
-      const uint32_t scales = sb + (uint32_t)(R.off_scales + m * C::kScaleBytes + g * 256);
+      const int m = i % NMAT, cg = cg0 + i / NMAT, gr = cg >> 2;
+      const uint32_t scales = rb + (uint32_t)(NMAT * R.code_bytes + m * C::kScaleBytes + gr * 256);
       if (m == 0) {
-        const uint32_t codes = sb + (uint32_t)(C::kOffCodes + g * fmt_words(F0) * 512);
-        v[i] = dequant_chunk<F0>(codes, scales, n, cg & 3);
+        v[i] = dequant_chunk<F0>(rb + (uint32_t)(gr * fmt_words(F0) * 512), scales, n, cg & 3);
       } else {
-        const uint32_t codes = sb + (uint32_t)(C::kOffCodes + R.code_bytes + g * fmt_words(F1) * 512);
-        v[i] = dequant_chunk<F1>(codes, scales, n, cg & 3);
+        v[i] = dequant_chunk<F1>(rb + (uint32_t)(R.code_bytes + gr * fmt_words(F1) * 512), scales, n, cg & 3);
       }
     }
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&raw_empty[rs]);  // release orders this warp's reads before it
+    if (++rs == R.raw_slots) {
+      rs = 0;
+      rph ^= 1u;
+    }
+    // the operand slot's previous MMAs are done, and this CTA's activation tile has landed
+    if (!__all_sync(0xffffffffu, ptx::mbar_wait(&op_empty[os], oph ^ 1u, abort_flag, wait) &&
+                                     ptx::mbar_wait(&b_full[os], oph, abort_flag, wait))) {
+      ok = false;
+      break;
+    }
+    const uint32_t ob = smem + (uint32_t)(os * C::kOpBytes);
 #pragma unroll
     for (int i = 0; i < kUnits; ++i) {
       const int m = i % NMAT, cg = cg0 + i / NMAT;
-      ptx::sts_v4(sb + (uint32_t)(C::kOffA + m * C::kABytes + tile_offset(n, cg)), v[i]);
+      ptx::sts_v4(ob + (uint32_t)(C::kOffA + m * C::kABytes + tile_offset(n, cg)), v[i]);
     }
     ptx::fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
       if (CG2)
-        ptx::mbar_arrive_cluster(&a_full[stage], 0);  // the even CTA issues the pair's MMAs
+        ptx::mbar_arrive_cluster(&a_full[os], 0);  // the even CTA issues the pair's MMAs
       else
-        ptx::mbar_arrive(&a_full[stage]);
+        ptx::mbar_arrive(&a_full[os]);
     }
-    if (threadIdx.x == 0) trace_stamp(trace, 3, gstage);
-    ++gstage;
-    if (++stage == R.stages) {
-      stage = 0;
-      phase ^= 1u;
+    if (threadIdx.x == 0) trace_stamp(trace, 3, g);
+    ++g;
+    if (++os == R.op_slots) {
+      os = 0;
+      oph ^= 1u;
     }
   }
-  return true;
+  cursor = Cursor{rs, rph, os, oph, g};
+  return ok;
 }
 
 // Runtime format pair -> the matching dequant_item instantiation.  I1: the launch
 // meets 1-bit matrices; their cases are compiled only into the I1 kernels, so the
 // kernels for layers without them keep their size and register allocation.
 template <int NMAT, bool CG2, bool I1, int F0>
-__device__ __forceinline__ bool dequant_item_f1(int f1, const Ring R, long long wait, uint32_t smem, uint64_t* load_full, uint64_t* a_full,
-                                                volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
-                                                uint32_t& phase, int& gstage, unsigned long long* trace) {
-  if (NMAT == 1) return dequant_item<NMAT, CG2, F0, F0>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+__device__ __forceinline__ bool dequant_item_f1(int f1, const Ring R, long long wait, uint32_t smem, uint64_t* bars,
+                                                volatile int* abort_flag, int ksteps, int n, int u0, Cursor& cur,
+                                                unsigned long long* trace) {
+  if (NMAT == 1) return dequant_item<NMAT, CG2, F0, F0>(R, wait, smem, bars, abort_flag, ksteps, n, u0, cur, trace);
   if constexpr (I1) {
-    if (f1 == MOE_FMT_INT1) return dequant_item<NMAT, CG2, F0, MOE_FMT_INT1>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    if (f1 == MOE_FMT_INT1)
+      return dequant_item<NMAT, CG2, F0, MOE_FMT_INT1>(R, wait, smem, bars, abort_flag, ksteps, n, u0, cur, trace);
   }
   switch (f1) {
-    case MOE_FMT_INT2: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT2>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    case MOE_FMT_INT3: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT3>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    case MOE_FMT_INT4: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT4>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    default: return dequant_item<NMAT, CG2, F0, MOE_FMT_NVFP4>(R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT2: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT2>(R, wait, smem, bars, abort_flag, ksteps, n, u0, cur, trace);
+    case MOE_FMT_INT3: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT3>(R, wait, smem, bars, abort_flag, ksteps, n, u0, cur, trace);
+    case MOE_FMT_INT4: return dequant_item<NMAT, CG2, F0, MOE_FMT_INT4>(R, wait, smem, bars, abort_flag, ksteps, n, u0, cur, trace);
+    default: return dequant_item<NMAT, CG2, F0, MOE_FMT_NVFP4>(R, wait, smem, bars, abort_flag, ksteps, n, u0, cur, trace);
   }
 }
 template <int NMAT, bool CG2, bool I1>
-__device__ __forceinline__ bool dequant_item_any(int f0, int f1, const Ring R, long long wait, uint32_t smem, uint64_t* load_full, uint64_t* a_full,
-                                                 volatile int* abort_flag, int ksteps, int n, int u0, int& stage,
-                                                 uint32_t& phase, int& gstage, unsigned long long* trace) {
+__device__ __forceinline__ bool dequant_item_any(int f0, int f1, const Ring R, long long wait, uint32_t smem,
+                                                 uint64_t* bars, volatile int* abort_flag, int ksteps, int n, int u0,
+                                                 Cursor& cur, unsigned long long* trace) {
   if constexpr (I1) {
-    if (f0 == MOE_FMT_INT1) return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_INT1>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    if (f0 == MOE_FMT_INT1)
+      return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_INT1>(f1, R, wait, smem, bars, abort_flag, ksteps, n, u0, cur, trace);
   }
   switch (f0) {
-    case MOE_FMT_INT2: return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_INT2>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    case MOE_FMT_INT3: return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_INT3>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    case MOE_FMT_INT4: return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_INT4>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
-    default: return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_NVFP4>(f1, R, wait, smem, load_full, a_full, abort_flag, ksteps, n, u0, stage, phase, gstage, trace);
+    case MOE_FMT_INT2: return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_INT2>(f1, R, wait, smem, bars, abort_flag, ksteps, n, u0, cur, trace);
+    case MOE_FMT_INT3: return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_INT3>(f1, R, wait, smem, bars, abort_flag, ksteps, n, u0, cur, trace);
+    case MOE_FMT_INT4: return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_INT4>(f1, R, wait, smem, bars, abort_flag, ksteps, n, u0, cur, trace);
+    default: return dequant_item_f1<NMAT, CG2, I1, MOE_FMT_NVFP4>(f1, R, wait, smem, bars, abort_flag, ksteps, n, u0, cur, trace);
   }
 }
 
@@ -326,11 +374,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // integer round trip would turn every access through it into a generic one)
   uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
   const Ring R = a.ring;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + R.stages * R.stage_bytes);
-  uint64_t* load_full = bars;
-  uint64_t* a_full = bars + R.stages;
-  uint64_t* stage_empty = bars + 2 * R.stages;
-  uint64_t* acc_full = bars + 3 * R.stages;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + R.off_raw + R.raw_slots * R.raw_bytes);
+  uint64_t* raw_full = bars;                 // [kMaxRaw] codes + scales landed (tx count)
+  uint64_t* raw_empty = bars + kMaxRaw;      // [kMaxRaw] this CTA's dequant warps have read them
+  uint64_t* b_full = bars + 2 * kMaxRaw;     // [kMaxOp] this CTA's activation tile landed (tx count)
+  uint64_t* a_full = b_full + kMaxOp;        // [kMaxOp] dequant warps of the pair wrote the weight tiles
+  uint64_t* op_empty = a_full + kMaxOp;      // [kMaxOp] the MMAs reading the slot are done
+  uint64_t* acc_full = op_empty + kMaxOp;
   uint64_t* acc_empty = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -343,10 +393,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t rank = CG2 ? ptx::cluster_ctarank() : 0u;
   constexpr int kPairCtas = CG2 ? 2 : 1;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < R.stages; ++s) {
-      ptx::mbar_init(&load_full[s], 1);
+    for (int s = 0; s < R.raw_slots; ++s) {
+      ptx::mbar_init(&raw_full[s], 1);
+      ptx::mbar_init(&raw_empty[s], kDeqWarps);  // this CTA's dequant warps
+    }
+    for (int s = 0; s < R.op_slots; ++s) {
+      ptx::mbar_init(&b_full[s], 1);
       ptx::mbar_init(&a_full[s], kDeqWarps * kPairCtas);  // one arrival per dequant warp of the pair
-      ptx::mbar_init(&stage_empty[s], 1);
+      ptx::mbar_init(&op_empty[s], 1);
     }
     ptx::mbar_init(acc_full, 1);
     ptx::mbar_init(acc_empty, kDeqWarps * kPairCtas);
@@ -362,7 +416,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ptx::tmem_relinquish();
     }
   }
-  if (warp == kTmaWarp && lane == 0) ptx::prefetch_tmap(&tmap_b);
+  if (warp == kBWarp && lane == 0) ptx::prefetch_tmap(&tmap_b);
   ptx::tc_fence_before();
   __syncthreads();
   if (CG2) ptx::cluster_sync();  // the peer's barriers are initialised before any remote arrival
@@ -386,22 +440,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort_flag, a.wait)) != 0;
   };
 
-  if (warp == kTmaWarp) {
-    int stage = 0, gstage = 0;
-    uint32_t phase = 0;
-    uint32_t issued = 0, issued_phase = 0;  // per stage: a load was armed, and its parity
+  if (warp == kRawWarp) {
+    // ---------------------------------------------------------- packed codes + scales
+    int rs = 0, g = 0;
+    uint32_t rph = 0;
+    uint32_t issued = 0, issued_phase = 0;  // per raw slot: a load was armed, and its parity
     for (int t = first; t < total && ok; t += stride) {
       const int c = t / m_tiles, mt = (t % m_tiles) * kPairCtas + (int)rank;
       const int e = a.chunks[3 * c];
-      // this CTA's token rows of the MMA's N = nmma columns: the first or second half
-      const int nmma = min(kTcBN, (a.chunks[3 * c + 2] + 15) & ~15);
-      const int row0 = a.chunks[3 * c + 1] + (int)rank * (nmma / 2);
       // A weight tile's codes (and scales) are contiguous along K, so each stage's
       // slice is the tile base plus ks times a fixed stride.
       const uint8_t* cptr[NMAT];
       const uint8_t* sptr[NMAT];
       uint32_t cbytes[NMAT];
-      uint32_t bytes = C::kBBytes;
+      uint32_t bytes = 0;
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) {
         const int i = e * 3 + a.proj + (a.pair ? 0 : m);
@@ -413,49 +465,81 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         bytes += cbytes[m] + (uint32_t)C::kScaleBytes;
       }
       for (int ks = 0; ks < ksteps; ++ks) {
-        if (lane == 0 && ks + kPrefetchAhead < ksteps) {  // warm L2 with the codes a few stages ahead
-#pragma unroll
-          for (int m = 0; m < NMAT; ++m)
-            ptx::prefetch_l2(cptr[m] + (size_t)(ks + kPrefetchAhead) * cbytes[m], cbytes[m]);
-        }
-        if (!wait_all(&stage_empty[stage], phase ^ 1u)) {
+        if (!wait_all(&raw_empty[rs], rph ^ 1u)) {
           ok = false;
           break;
         }
         if (lane == 0 && !a.withhold) {
-          trace_stamp(a.trace, 0, gstage);
-          uint8_t* sb = smem + stage * R.stage_bytes;
-          ptx::mbar_arrive_expect_tx(&load_full[stage], bytes);
-          ptx::tma_load_2d(sb + C::kOffB, &tmap_b, ks * kTcBK, row0, &load_full[stage]);
+          trace_stamp(a.trace, 0, g);
+          uint8_t* rb = smem + R.off_raw + rs * R.raw_bytes;
+          ptx::mbar_arrive_expect_tx(&raw_full[rs], bytes);
 #pragma unroll
           for (int m = 0; m < NMAT; ++m) {
-            ptx::bulk_load(sb + C::kOffCodes + m * R.code_bytes, cptr[m] + (size_t)ks * cbytes[m], cbytes[m],
-                           &load_full[stage]);
-            ptx::bulk_load(sb + R.off_scales + m * C::kScaleBytes, sptr[m] + (size_t)ks * C::kScaleBytes,
-                           (uint32_t)C::kScaleBytes, &load_full[stage]);
+            ptx::bulk_load(rb + m * R.code_bytes, cptr[m] + (size_t)ks * cbytes[m], cbytes[m], &raw_full[rs]);
+            ptx::bulk_load(rb + NMAT * R.code_bytes + m * C::kScaleBytes, sptr[m] + (size_t)ks * C::kScaleBytes,
+                           (uint32_t)C::kScaleBytes, &raw_full[rs]);
           }
-          trace_stamp(a.trace, 1, gstage);
+          trace_stamp(a.trace, 1, g);
         }
-        ++gstage;
+        ++g;
         __syncwarp();
         if (!a.withhold) {
-          issued |= 1u << stage;
-          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          issued |= 1u << rs;
+          issued_phase = (issued_phase & ~(1u << rs)) | (rph << rs);
         }
-        if (++stage == R.stages) {
-          stage = 0;
-          phase ^= 1u;
+        if (++rs == R.raw_slots) {
+          rs = 0;
+          rph ^= 1u;
         }
       }
     }
     // never leave while a copy may still be landing in shared memory
-    for (int s = 0; s < R.stages; ++s)
-      if (issued & (1u << s)) ptx::mbar_drain(&load_full[s], (issued_phase >> s) & 1u, kWaitLimit / 4);
+    for (int s2 = 0; s2 < R.raw_slots; ++s2)
+      if (issued & (1u << s2)) ptx::mbar_drain(&raw_full[s2], (issued_phase >> s2) & 1u, kWaitLimit / 4);
+    __syncwarp();
+  } else if (warp == kBWarp) {
+    // ---------------------------------------------------------- activation tiles
+    int os = 0;
+    uint32_t oph = 0;
+    uint32_t issued = 0, issued_phase = 0;  // per operand slot: a load was armed, and its parity
+    for (int t = first; t < total && ok; t += stride) {
+      const int c = t / m_tiles;
+      // this CTA's token rows of the MMA's N = nmma columns: the first or second half
+      const int nmma = min(kTcBN, (a.chunks[3 * c + 2] + 15) & ~15);
+      const int row0 = a.chunks[3 * c + 1] + (int)rank * (nmma / 2);
+      for (int ks = 0; ks < ksteps; ++ks) {
+        if (!wait_all(&op_empty[os], oph ^ 1u)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0 && !a.withhold) {
+          ptx::mbar_arrive_expect_tx(&b_full[os], (uint32_t)C::kBBytes);
+          ptx::tma_load_2d(smem + os * C::kOpBytes + C::kOffB, &tmap_b, ks * kTcBK, row0, &b_full[os]);
+        }
+        __syncwarp();
+        if (!a.withhold) {
+          issued |= 1u << os;
+          issued_phase = (issued_phase & ~(1u << os)) | (oph << os);
+        }
+        if (++os == R.op_slots) {
+          os = 0;
+          oph ^= 1u;
+        }
+      }
+    }
+    for (int s2 = 0; s2 < R.op_slots; ++s2)
+      if (issued & (1u << s2)) ptx::mbar_drain(&b_full[s2], (issued_phase >> s2) & 1u, kWaitLimit / 4);
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    int stage = 0, gstage = 0;
-    uint32_t phase = 0, acc_phase = 0;
+    // ---------------------------------------------------------- MMA issue (even CTA)
+    int os = 0, g = 0;
+    uint32_t oph = 0, acc_phase = 0;
+    // Shared-memory descriptors of operand slot 0, built once: a slot, a weight tile
+    // and a K=16 step only add to the 14-bit start-address field (16-byte units;
+    // every shared address here is below 256 KB, so the field never carries).
     const uint32_t sbase = ptx::smem_u32(smem);
+    const uint64_t dA0 = tile_desc(sbase + C::kOffA), dB0 = tile_desc(sbase + C::kOffB);
+    constexpr uint64_t kSlotStep = C::kOpBytes >> 4, kTileStep = C::kABytes >> 4, kKStep = 32 >> 4;
     bool committed = false;
     for (int t = first; t < total && ok && rank == 0; t += stride) {
       const int c = t / m_tiles;
@@ -469,37 +553,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       acc_phase ^= 1u;
       ptx::tc_fence_after();
       for (int ks = 0; ks < ksteps; ++ks) {
-        if (!wait_all(&a_full[stage], phase) || !wait_all(&load_full[stage], phase)) {
+        if (!wait_all(&a_full[os], oph)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        if (lane == 0) trace_stamp(a.trace, 4, gstage);
+        if (lane == 0) trace_stamp(a.trace, 4, g);
         if (lane == 0) {
-          const uint32_t st = sbase + (uint32_t)(stage * R.stage_bytes);
+          const uint64_t so = (uint64_t)os * kSlotStep;
+          const uint64_t da = dA0 + so, db = dB0 + so;
+          const uint32_t acc0 = ks != 0;
 #pragma unroll
           for (int m = 0; m < NMAT; ++m)
 #pragma unroll
             for (int k16 = 0; k16 < kTcBK / 16; ++k16) {
-              const uint64_t ad = tile_desc(st + C::kOffA + m * C::kABytes + k16 * 32);
-              const uint64_t bd = tile_desc(st + C::kOffB + k16 * 32);
+              const uint64_t ad = da + (uint64_t)m * kTileStep + (uint64_t)k16 * kKStep;
+              const uint64_t bd = db + (uint64_t)k16 * kKStep;
               if (CG2)
-                ptx::mma2_f16_ss(tmem + (uint32_t)(m * 256), ad, bd, idesc, (ks | k16) != 0);
+                ptx::mma2_f16_ss(tmem + (uint32_t)(m * 256), ad, bd, idesc, k16 ? 1u : acc0);
               else
-                ptx::mma_f16_ss(tmem + (uint32_t)(m * 256), ad, bd, idesc, (ks | k16) != 0);
+                ptx::mma_f16_ss(tmem + (uint32_t)(m * 256), ad, bd, idesc, k16 ? 1u : acc0);
             }
           if (CG2)
-            ptx::mma2_commit_mc(&stage_empty[stage], 0x3);
+            ptx::mma2_commit_mc(&op_empty[os], 0x3);
           else
-            ptx::mma_commit(&stage_empty[stage]);
-          trace_stamp(a.trace, 5, gstage);
+            ptx::mma_commit(&op_empty[os]);
+          trace_stamp(a.trace, 5, g);
         }
-        ++gstage;
+        ++g;
         __syncwarp();
         committed = true;
-        if (++stage == R.stages) {
-          stage = 0;
-          phase ^= 1u;
+        if (++os == R.op_slots) {
+          os = 0;
+          oph ^= 1u;
         }
       }
       if (!ok) break;
@@ -512,9 +598,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
     }
     if (committed) {  // the last commit lands once every MMA issued by this CTA has completed
-      const int last = (stage + R.stages - 1) % R.stages;
-      const uint32_t par = (stage == 0) ? (phase ^ 1u) : phase;
-      ptx::mbar_drain(&stage_empty[last], par, kWaitLimit / 4);
+      const int last = (os + R.op_slots - 1) % R.op_slots;
+      const uint32_t par = (os == 0) ? (oph ^ 1u) : oph;
+      ptx::mbar_drain(&op_empty[last], par, kWaitLimit / 4);
     }
     __syncwarp();
   } else {
@@ -528,8 +614,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int q = warp & 3, cq = warp >> 2;               // epilogue: TMEM lane quarter, column group
     constexpr int kUnits = NMAT * kGroups * 4 / kThreadsPerRow;
     const int u0 = sel * kUnits;
-    int stage = 0, gstage = 0, item = 0;
-    uint32_t phase = 0, acc_phase = 0;
+    Cursor cur{0, 0u, 0, 0u, 0};
+    int item = 0;
+    uint32_t acc_phase = 0;
     for (int t = first; t < total && ok; t += stride, ++item) {
       const int c = t / m_tiles, mt = (t % m_tiles) * kPairCtas + (int)rank;
       const int e = a.chunks[3 * c], row0 = a.chunks[3 * c + 1], rows = a.chunks[3 * c + 2];
@@ -541,8 +628,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         fmt[m] = L.fmt[i];
         tsc[m] = fmt[m] == MOE_FMT_NVFP4 ? L.tscale[i] : 1.0f;
       }
-      if (!dequant_item_any<NMAT, CG2, I1>(fmt[0], fmt[NMAT - 1], a.ring, a.wait, ptx::smem_u32(smem), load_full, a_full, abort_flag, ksteps, n, u0, stage,
-                                  phase, gstage, a.trace)) {
+      if (!dequant_item_any<NMAT, CG2, I1>(fmt[0], fmt[NMAT - 1], a.ring, a.wait, ptx::smem_u32(smem), bars,
+                                           abort_flag, ksteps, n, u0, cur, a.trace)) {
         ok = false;
         break;
       }
@@ -660,7 +747,7 @@ template <int NMAT, bool CG2, bool I1>
 cudaError_t launch_tc(TcArgs a, int max_words, const void* act, int rows_total, cudaStream_t stream) {
   using C = TcCfg<NMAT, CG2>;
   a.ring = make_ring<NMAT, CG2>(max_words);
-  if (a.ring.stages < 3) return cudaErrorInvalidConfiguration;
+  if (a.ring.raw_slots < 2) return cudaErrorInvalidConfiguration;
   const int smem = ring_smem(a.ring);
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;

@@ -30,6 +30,9 @@ struct GemmHooks {
   uint32_t wait_cycles;  // pipeline wait budget, 0: default
 };
 
+// Token rows per work chunk of the tcgen05 expert GEMMs (the MMA's largest N).
+constexpr int kTcChunkRows = 256;
+
 cudaError_t launch_expert_gemm_tc(const uint8_t* packed, const uint8_t* fmt_host, int E, int H, int F, int T, int k,
                                   bool fp4, bool gateup, const Workspace& ws, int32_t* status, uint64_t* trace,
                                   GemmHooks hooks, cudaStream_t stream);
