@@ -559,7 +559,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         ptx::tc_fence_after();
         if (lane == 0) trace_stamp(a.trace, 4, g);
-        if (lane == 0) {
+        {
+          // the whole warp runs this with uniform operands; one elected lane issues
           const uint64_t so = (uint64_t)os * kSlotStep;
           const uint64_t da = dA0 + so, db = dB0 + so;
           const uint32_t acc0 = ks != 0;
@@ -570,15 +571,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const uint64_t ad = da + (uint64_t)m * kTileStep + (uint64_t)k16 * kKStep;
               const uint64_t bd = db + (uint64_t)k16 * kKStep;
               if (CG2)
-                ptx::mma2_f16_ss(tmem + (uint32_t)(m * 256), ad, bd, idesc, k16 ? 1u : acc0);
+                ptx::mma2_f16_ss_warp(tmem + (uint32_t)(m * 256), ad, bd, idesc, k16 ? 1u : acc0);
               else
-                ptx::mma_f16_ss(tmem + (uint32_t)(m * 256), ad, bd, idesc, k16 ? 1u : acc0);
+                ptx::mma_f16_ss_warp(tmem + (uint32_t)(m * 256), ad, bd, idesc, k16 ? 1u : acc0);
             }
           if (CG2)
-            ptx::mma2_commit_mc(&op_empty[os], 0x3);
+            ptx::mma2_commit_mc_warp(&op_empty[os], 0x3);
           else
-            ptx::mma_commit(&op_empty[os]);
-          trace_stamp(a.trace, 5, g);
+            ptx::mma_commit_warp(&op_empty[os]);
+          if (lane == 0) trace_stamp(a.trace, 5, g);
         }
         ++g;
         __syncwarp();
@@ -589,12 +590,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       if (!ok) break;
-      if (lane == 0) {
-        if (CG2)
-          ptx::mma2_commit_mc(acc_full, 0x3);
-        else
-          ptx::mma_commit(acc_full);
-      }
+      if (CG2)
+        ptx::mma2_commit_mc_warp(acc_full, 0x3);
+      else
+        ptx::mma_commit_warp(acc_full);
       __syncwarp();
     }
     if (committed) {  // the last commit lands once every MMA issued by this CTA has completed
