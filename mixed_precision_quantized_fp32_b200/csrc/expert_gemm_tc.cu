@@ -66,45 +66,53 @@ constexpr long long kWaitLimit = 4000000000LL;  // clock cycles, ~2 s
 
 // CG2: the work item runs on a pair of CTAs (one cluster) with cta_group::2
 // MMAs, each CTA holding half of the activation tile's token rows.
-// Two rings per CTA:
+// Three rings of shared-memory slots per CTA:
 //  * raw slots: the packed codes and scales of NMAT weight tiles for one stage,
-//    freed as soon as the dequant warps have read them, so copies run many
+//    freed as soon as the dequant warps have read them, so their copies run many
 //    stages ahead;
-//  * operand slots: the activation tile and the NMAT dequantized weight tiles
-//    the tensor core reads, freed by the MMA commit.
-// The code slot is sized for the widest format the launch meets (Ring).
+//  * A slots: the NMAT dequantized weight tiles the tensor core reads;
+//  * B slots: the activation tile; its own ring, so activation loads are issued
+//    several stages ahead instead of waiting for a weight-tile slot to free.
+// A and B slots are freed by the MMA commit.  The code slot is sized for the
+// widest format the launch meets (Ring).
 template <int NMAT, bool CG2 = false>
 struct TcCfg {
   static constexpr int kBRows = CG2 ? kTcBN / 2 : kTcBN;
-  static constexpr int kBBytes = kBRows * kRowBytes;  // activation tile (this CTA's rows)
+  static constexpr int kBBytes = kBRows * kRowBytes;  // activation tile (this CTA's rows), one B slot
   static constexpr int kABytes = kTcBM * kRowBytes;   // dequantized weight tile
+  static constexpr int kASlotBytes = NMAT * kABytes;  // one A slot
   static constexpr int kScaleBytes = kGroups * 256;   // one fp16 group or two e4m3 blocks x 128 rows
-  static constexpr int kOffB = 0;
-  static constexpr int kOffA = kBBytes;
-  static constexpr int kOpBytes = kBBytes + NMAT * kABytes;  // one operand slot (a multiple of 1024)
 };
-constexpr int kMaxRaw = 16, kMaxOp = 4;
-constexpr int kBarBytes = 512;                       // barriers, TMEM slot and abort flag
+constexpr int kMaxRaw = 16, kMaxA = 4, kMaxB = 8;
+constexpr int kBarBytes = 640;                       // barriers, TMEM slot and abort flag
 constexpr int kSmemMax = 232448;                     // opt-in shared memory per CTA
-static_assert(8 * (2 * kMaxRaw + 3 * kMaxOp + 2) + 16 <= kBarBytes, "barrier area");
+static_assert(8 * (2 * kMaxRaw + 2 * kMaxA + 3 * kMaxB + 2) + 16 <= kBarBytes, "barrier area");
 
 struct Ring {
-  int op_slots;     // operand slots (<= kMaxOp)
+  int a_slots;      // weight-tile slots (<= kMaxA)
+  int b_slots;      // activation-tile slots (<= kMaxB)
   int raw_slots;    // raw slots (<= kMaxRaw)
   int code_bytes;   // one matrix's code slot: kGroups x 512 bytes per code word of the widest format
   int raw_bytes;    // one raw slot: NMAT code slots, then NMAT scale slots
-  int off_raw;      // offset of the raw ring (after the operand slots)
+  int off_b;        // offset of the B ring (after the A slots)
+  int off_raw;      // offset of the raw ring (after the B slots)
 };
 
 template <int NMAT, bool CG2>
 Ring make_ring(int max_words) {
   using C = TcCfg<NMAT, CG2>;
   Ring r;
-  r.op_slots = CG2 ? 3 : 2;
+  r.a_slots = CG2 ? 3 : 2;
+  r.b_slots = CG2 ? 5 : 3;
   r.code_bytes = kGroups * 512 * max_words;
   r.raw_bytes = (NMAT * (r.code_bytes + C::kScaleBytes) + 127) / 128 * 128;
-  r.off_raw = r.op_slots * C::kOpBytes;
-  r.raw_slots = min(kMaxRaw, (kSmemMax - kBarBytes - 1024 - r.off_raw) / r.raw_bytes);
+  for (;;) {
+    r.off_b = r.a_slots * C::kASlotBytes;
+    r.off_raw = r.off_b + r.b_slots * C::kBBytes;
+    r.raw_slots = min(kMaxRaw, (kSmemMax - kBarBytes - 1024 - r.off_raw) / r.raw_bytes);
+    if (r.raw_slots >= 4 || r.b_slots <= 2) break;
+    --r.b_slots;  // keep the raw ring at least 4 deep
+  }
   return r;
 }
 inline int ring_smem(const Ring& r) { return r.off_raw + r.raw_slots * r.raw_bytes + kBarBytes + 1024; }
@@ -240,22 +248,48 @@ __device__ __forceinline__ uint64_t scale_stage_offset(int mt, int g, int K, int
   return ((uint64_t)mt * (uint64_t)(K >> 5) + (uint64_t)g) * 256u;
 }
 
-// Position of a role in the two rings: raw slot and phase, operand slot and
-// phase, and the global stage counter (trace index).
+// The mbarriers after the rings.
+struct Bars {
+  uint64_t* raw_full;   // [kMaxRaw] codes + scales landed (tx count)
+  uint64_t* raw_empty;  // [kMaxRaw] this CTA's dequant warps have read them
+  uint64_t* a_full;     // [kMaxA] the dequant warps of the pair wrote the weight tiles (the even CTA's counts)
+  uint64_t* a_empty;    // [kMaxA] the MMAs reading the weight tiles are done
+  uint64_t* b_full;     // [kMaxB] this CTA's activation tile landed (tx count)
+  uint64_t* b_empty;    // [kMaxB] the MMAs reading the activation tile are done
+  uint64_t* b_peer;     // [kMaxB] (even CTA) the odd CTA's activation tile landed
+  uint64_t* acc_full;
+  uint64_t* acc_empty;
+};
+__device__ __forceinline__ Bars bars_at(uint64_t* b) {
+  Bars r;
+  r.raw_full = b;
+  r.raw_empty = b + kMaxRaw;
+  r.a_full = b + 2 * kMaxRaw;
+  r.a_empty = r.a_full + kMaxA;
+  r.b_full = r.a_empty + kMaxA;
+  r.b_empty = r.b_full + kMaxB;
+  r.b_peer = r.b_empty + kMaxB;
+  r.acc_full = r.b_peer + kMaxB;
+  r.acc_empty = r.acc_full + 1;
+  return r;
+}
+
+// Position of the dequant warps in the raw and A rings, and the global stage
+// counter (trace index).
 struct Cursor {
   int rs;
   uint32_t rph;
-  int os;
-  uint32_t oph;
+  int as;
+  uint32_t aph;
   int g;
 };
 
 // Dequantize every stage of one work item (formats F0 = first matrix, F1 =
 // second): wait for the stage's codes in a raw slot, convert this thread's units
-// to registers and release the raw slot, wait for the operand slot to be free
-// (its previous MMAs done) and this CTA's activation tile to land, write the
-// units in the tensor core's layout and arrive on the operand slot's barrier
-// (the even CTA's, for a pair).  Returns false if a bounded wait gave up.
+// to registers and release the raw slot, wait for the A slot to be free (its
+// previous MMAs done), write the units in the tensor core's layout and arrive on
+// the A slot's barrier (the even CTA's, for a pair).  Returns false if a bounded
+// wait gave up.
 template <int NMAT, bool CG2, int F0, int F1>
 __device__ __noinline__ bool dequant_item(const Ring R, long long wait, uint32_t smem, uint64_t* bars,
                                           volatile int* abort_flag, int ksteps, int n, int u0, Cursor& cursor,
@@ -263,20 +297,16 @@ __device__ __noinline__ bool dequant_item(const Ring R, long long wait, uint32_t
   using C = TcCfg<NMAT, CG2>;
   constexpr int kUnits = NMAT * kGroups * 4 / kThreadsPerRow;
   static_assert(NMAT == 1 || kUnits % 2 == 0, "units must alternate matrices evenly");
-  uint64_t* raw_full = bars;
-  uint64_t* raw_empty = bars + kMaxRaw;
-  uint64_t* b_full = bars + 2 * kMaxRaw;
-  uint64_t* a_full = b_full + kMaxOp;
-  uint64_t* op_empty = a_full + kMaxOp;
+  const Bars B = bars_at(bars);
   const int lane = threadIdx.x & 31;
   const int cg0 = u0 / NMAT;
   // the cursor lives in registers for the loop (a reference would be re-read after every
   // shared-memory store)
-  int rs = cursor.rs, os = cursor.os, g = cursor.g;
-  uint32_t rph = cursor.rph, oph = cursor.oph;
+  int rs = cursor.rs, as = cursor.as, g = cursor.g;
+  uint32_t rph = cursor.rph, aph = cursor.aph;
   bool ok = true;
   for (int ks = 0; ks < ksteps; ++ks) {
-    if (!__all_sync(0xffffffffu, ptx::mbar_wait(&raw_full[rs], rph, abort_flag, wait))) {
+    if (!__all_sync(0xffffffffu, ptx::mbar_wait(&B.raw_full[rs], rph, abort_flag, wait))) {
       ok = false;
       break;
     }
@@ -294,39 +324,38 @@ __device__ __noinline__ bool dequant_item(const Ring R, long long wait, uint32_t
       }
     }
     __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(&raw_empty[rs]);  // release orders this warp's reads before it
+    if (lane == 0) ptx::mbar_arrive(&B.raw_empty[rs]);  // release orders this warp's reads before it
     if (++rs == R.raw_slots) {
       rs = 0;
       rph ^= 1u;
     }
-    // the operand slot's previous MMAs are done, and this CTA's activation tile has landed
-    if (!__all_sync(0xffffffffu, ptx::mbar_wait(&op_empty[os], oph ^ 1u, abort_flag, wait) &&
-                                     ptx::mbar_wait(&b_full[os], oph, abort_flag, wait))) {
+    // the A slot's previous MMAs are done
+    if (!__all_sync(0xffffffffu, ptx::mbar_wait(&B.a_empty[as], aph ^ 1u, abort_flag, wait))) {
       ok = false;
       break;
     }
-    const uint32_t ob = smem + (uint32_t)(os * C::kOpBytes);
+    const uint32_t ab = smem + (uint32_t)(as * C::kASlotBytes);
 #pragma unroll
     for (int i = 0; i < kUnits; ++i) {
       const int m = i % NMAT, cg = cg0 + i / NMAT;
-      ptx::sts_v4(ob + (uint32_t)(C::kOffA + m * C::kABytes + tile_offset(n, cg)), v[i]);
+      ptx::sts_v4(ab + (uint32_t)(m * C::kABytes + tile_offset(n, cg)), v[i]);
     }
     ptx::fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
       if (CG2)
-        ptx::mbar_arrive_cluster(&a_full[os], 0);  // the even CTA issues the pair's MMAs
+        ptx::mbar_arrive_cluster(&B.a_full[as], 0);  // the even CTA issues the pair's MMAs
       else
-        ptx::mbar_arrive(&a_full[os]);
+        ptx::mbar_arrive(&B.a_full[as]);
     }
     if (threadIdx.x == 0) trace_stamp(trace, 3, g);
     ++g;
-    if (++os == R.op_slots) {
-      os = 0;
-      oph ^= 1u;
+    if (++as == R.a_slots) {
+      as = 0;
+      aph ^= 1u;
     }
   }
-  cursor = Cursor{rs, rph, os, oph, g};
+  cursor = Cursor{rs, rph, as, aph, g};
   return ok;
 }
 
@@ -375,14 +404,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
   const Ring R = a.ring;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + R.off_raw + R.raw_slots * R.raw_bytes);
-  uint64_t* raw_full = bars;                 // [kMaxRaw] codes + scales landed (tx count)
-  uint64_t* raw_empty = bars + kMaxRaw;      // [kMaxRaw] this CTA's dequant warps have read them
-  uint64_t* b_full = bars + 2 * kMaxRaw;     // [kMaxOp] this CTA's activation tile landed (tx count)
-  uint64_t* a_full = b_full + kMaxOp;        // [kMaxOp] dequant warps of the pair wrote the weight tiles
-  uint64_t* op_empty = a_full + kMaxOp;      // [kMaxOp] the MMAs reading the slot are done
-  uint64_t* acc_full = op_empty + kMaxOp;
-  uint64_t* acc_empty = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  const Bars B = bars_at(bars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(B.acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -394,16 +417,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr int kPairCtas = CG2 ? 2 : 1;
   if (threadIdx.x == 0) {
     for (int s = 0; s < R.raw_slots; ++s) {
-      ptx::mbar_init(&raw_full[s], 1);
-      ptx::mbar_init(&raw_empty[s], kDeqWarps);  // this CTA's dequant warps
+      ptx::mbar_init(&B.raw_full[s], 1);
+      ptx::mbar_init(&B.raw_empty[s], kDeqWarps);  // this CTA's dequant warps
     }
-    for (int s = 0; s < R.op_slots; ++s) {
-      ptx::mbar_init(&b_full[s], 1);
-      ptx::mbar_init(&a_full[s], kDeqWarps * kPairCtas);  // one arrival per dequant warp of the pair
-      ptx::mbar_init(&op_empty[s], 1);
+    for (int s = 0; s < R.a_slots; ++s) {
+      ptx::mbar_init(&B.a_full[s], kDeqWarps * kPairCtas);  // one arrival per dequant warp of the pair
+      ptx::mbar_init(&B.a_empty[s], 1);
     }
-    ptx::mbar_init(acc_full, 1);
-    ptx::mbar_init(acc_empty, kDeqWarps * kPairCtas);
+    for (int s = 0; s < R.b_slots; ++s) {
+      ptx::mbar_init(&B.b_full[s], 1);
+      ptx::mbar_init(&B.b_empty[s], 1);
+      ptx::mbar_init(&B.b_peer[s], 1);
+    }
+    ptx::mbar_init(B.acc_full, 1);
+    ptx::mbar_init(B.acc_empty, kDeqWarps * kPairCtas);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -465,19 +492,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         bytes += cbytes[m] + (uint32_t)C::kScaleBytes;
       }
       for (int ks = 0; ks < ksteps; ++ks) {
-        if (!wait_all(&raw_empty[rs], rph ^ 1u)) {
+        if (!wait_all(&B.raw_empty[rs], rph ^ 1u)) {
           ok = false;
           break;
         }
         if (lane == 0 && !a.withhold) {
           trace_stamp(a.trace, 0, g);
           uint8_t* rb = smem + R.off_raw + rs * R.raw_bytes;
-          ptx::mbar_arrive_expect_tx(&raw_full[rs], bytes);
+          ptx::mbar_arrive_expect_tx(&B.raw_full[rs], bytes);
 #pragma unroll
           for (int m = 0; m < NMAT; ++m) {
-            ptx::bulk_load(rb + m * R.code_bytes, cptr[m] + (size_t)ks * cbytes[m], cbytes[m], &raw_full[rs]);
+            ptx::bulk_load(rb + m * R.code_bytes, cptr[m] + (size_t)ks * cbytes[m], cbytes[m], &B.raw_full[rs]);
             ptx::bulk_load(rb + NMAT * R.code_bytes + m * C::kScaleBytes, sptr[m] + (size_t)ks * C::kScaleBytes,
-                           (uint32_t)C::kScaleBytes, &raw_full[rs]);
+                           (uint32_t)C::kScaleBytes, &B.raw_full[rs]);
           }
           trace_stamp(a.trace, 1, g);
         }
@@ -495,65 +522,86 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     // never leave while a copy may still be landing in shared memory
     for (int s2 = 0; s2 < R.raw_slots; ++s2)
-      if (issued & (1u << s2)) ptx::mbar_drain(&raw_full[s2], (issued_phase >> s2) & 1u, kWaitLimit / 4);
+      if (issued & (1u << s2)) ptx::mbar_drain(&B.raw_full[s2], (issued_phase >> s2) & 1u, kWaitLimit / 4);
     __syncwarp();
   } else if (warp == kBWarp) {
     // ---------------------------------------------------------- activation tiles
-    int os = 0;
-    uint32_t oph = 0;
-    uint32_t issued = 0, issued_phase = 0;  // per operand slot: a load was armed, and its parity
+    int bs = 0;
+    uint32_t bph = 0;
+    uint32_t issued = 0, issued_phase = 0;  // per B slot: a load was armed, and its parity
     for (int t = first; t < total && ok; t += stride) {
       const int c = t / m_tiles;
       // this CTA's token rows of the MMA's N = nmma columns: the first or second half
       const int nmma = min(kTcBN, (a.chunks[3 * c + 2] + 15) & ~15);
       const int row0 = a.chunks[3 * c + 1] + (int)rank * (nmma / 2);
       for (int ks = 0; ks < ksteps; ++ks) {
-        if (!wait_all(&op_empty[os], oph ^ 1u)) {
+        if (!wait_all(&B.b_empty[bs], bph ^ 1u)) {
           ok = false;
           break;
         }
         if (lane == 0 && !a.withhold) {
-          ptx::mbar_arrive_expect_tx(&b_full[os], (uint32_t)C::kBBytes);
-          ptx::tma_load_2d(smem + os * C::kOpBytes + C::kOffB, &tmap_b, ks * kTcBK, row0, &b_full[os]);
+          ptx::mbar_arrive_expect_tx(&B.b_full[bs], (uint32_t)C::kBBytes);
+          ptx::tma_load_2d(smem + R.off_b + bs * C::kBBytes, &tmap_b, ks * kTcBK, row0, &B.b_full[bs]);
         }
         __syncwarp();
         if (!a.withhold) {
-          issued |= 1u << os;
-          issued_phase = (issued_phase & ~(1u << os)) | (oph << os);
+          issued |= 1u << bs;
+          issued_phase = (issued_phase & ~(1u << bs)) | (bph << bs);
         }
-        if (++os == R.op_slots) {
-          os = 0;
-          oph ^= 1u;
+        if (++bs == R.b_slots) {
+          bs = 0;
+          bph ^= 1u;
         }
       }
     }
-    for (int s2 = 0; s2 < R.op_slots; ++s2)
-      if (issued & (1u << s2)) ptx::mbar_drain(&b_full[s2], (issued_phase >> s2) & 1u, kWaitLimit / 4);
+    for (int s2 = 0; s2 < R.b_slots; ++s2)
+      if (issued & (1u << s2)) ptx::mbar_drain(&B.b_full[s2], (issued_phase >> s2) & 1u, kWaitLimit / 4);
     __syncwarp();
+  } else if (warp == kMmaWarp && rank != 0) {
+    // ---------------------------------------------------------- odd CTA: report its activation tiles
+    // The even CTA's MMAs read this CTA's half of every activation tile; once it has
+    // landed, say so on the even CTA's barrier.
+    int bs = 0;
+    uint32_t bph = 0;
+    for (int t = first; t < total && ok; t += stride)
+      for (int ks = 0; ks < ksteps; ++ks) {
+        if (!wait_all(&B.b_full[bs], bph)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) ptx::mbar_arrive_cluster(&B.b_peer[bs], 0);
+        __syncwarp();
+        if (++bs == R.b_slots) {
+          bs = 0;
+          bph ^= 1u;
+        }
+      }
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------- MMA issue (even CTA)
-    int os = 0, g = 0;
-    uint32_t oph = 0, acc_phase = 0;
-    // Shared-memory descriptors of operand slot 0, built once: a slot, a weight tile
-    // and a K=16 step only add to the 14-bit start-address field (16-byte units;
-    // every shared address here is below 256 KB, so the field never carries).
+    int as = 0, bs = 0, g = 0;
+    uint32_t aph = 0, bph = 0, acc_phase = 0;
+    // Shared-memory descriptors of slot 0, built once: a slot, a weight tile and a
+    // K=16 step only add to the 14-bit start-address field (16-byte units; every
+    // shared address here is below 256 KB, so the field never carries).
     const uint32_t sbase = ptx::smem_u32(smem);
-    const uint64_t dA0 = tile_desc(sbase + C::kOffA), dB0 = tile_desc(sbase + C::kOffB);
-    constexpr uint64_t kSlotStep = C::kOpBytes >> 4, kTileStep = C::kABytes >> 4, kKStep = 32 >> 4;
+    const uint64_t dA0 = tile_desc(sbase), dB0 = tile_desc(sbase + (uint32_t)R.off_b);
+    constexpr uint64_t kASlotStep = C::kASlotBytes >> 4, kBSlotStep = C::kBBytes >> 4;
+    constexpr uint64_t kTileStep = C::kABytes >> 4, kKStep = 32 >> 4;
     bool committed = false;
-    for (int t = first; t < total && ok && rank == 0; t += stride) {
+    for (int t = first; t < total && ok; t += stride) {
       const int c = t / m_tiles;
       const int rows = a.chunks[3 * c + 2];
       const int nmma = min(kTcBN, (rows + 15) & ~15);
       const uint32_t idesc = ptx::idesc_f16_f32(kTcBM * kPairCtas, nmma);
-      if (!wait_all(acc_empty, acc_phase ^ 1u)) {
+      if (!wait_all(B.acc_empty, acc_phase ^ 1u)) {
         ok = false;
         break;
       }
       acc_phase ^= 1u;
       ptx::tc_fence_after();
       for (int ks = 0; ks < ksteps; ++ks) {
-        if (!wait_all(&a_full[os], oph)) {
+        if (!wait_all(&B.a_full[as], aph) || !wait_all(&B.b_full[bs], bph) ||
+            (CG2 && !wait_all(&B.b_peer[bs], bph))) {
           ok = false;
           break;
         }
@@ -561,8 +609,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) trace_stamp(a.trace, 4, g);
         {
           // the whole warp runs this with uniform operands; one elected lane issues
-          const uint64_t so = (uint64_t)os * kSlotStep;
-          const uint64_t da = dA0 + so, db = dB0 + so;
+          const uint64_t da = dA0 + (uint64_t)as * kASlotStep, db = dB0 + (uint64_t)bs * kBSlotStep;
           const uint32_t acc0 = ks != 0;
 #pragma unroll
           for (int m = 0; m < NMAT; ++m)
@@ -575,31 +622,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               else
                 ptx::mma_f16_ss_warp(tmem + (uint32_t)(m * 256), ad, bd, idesc, k16 ? 1u : acc0);
             }
-          if (CG2)
-            ptx::mma2_commit_mc_warp(&op_empty[os], 0x3);
-          else
-            ptx::mma_commit_warp(&op_empty[os]);
+          if (CG2) {
+            ptx::mma2_commit_mc_warp(&B.a_empty[as], 0x3);
+            ptx::mma2_commit_mc_warp(&B.b_empty[bs], 0x3);
+          } else {
+            ptx::mma_commit_warp(&B.a_empty[as]);
+            ptx::mma_commit_warp(&B.b_empty[bs]);
+          }
           if (lane == 0) trace_stamp(a.trace, 5, g);
         }
         ++g;
         __syncwarp();
         committed = true;
-        if (++os == R.op_slots) {
-          os = 0;
-          oph ^= 1u;
+        if (++as == R.a_slots) {
+          as = 0;
+          aph ^= 1u;
+        }
+        if (++bs == R.b_slots) {
+          bs = 0;
+          bph ^= 1u;
         }
       }
       if (!ok) break;
       if (CG2)
-        ptx::mma2_commit_mc_warp(acc_full, 0x3);
+        ptx::mma2_commit_mc_warp(B.acc_full, 0x3);
       else
-        ptx::mma_commit_warp(acc_full);
+        ptx::mma_commit_warp(B.acc_full);
       __syncwarp();
     }
     if (committed) {  // the last commit lands once every MMA issued by this CTA has completed
-      const int last = (os + R.op_slots - 1) % R.op_slots;
-      const uint32_t par = (os == 0) ? (oph ^ 1u) : oph;
-      ptx::mbar_drain(&op_empty[last], par, kWaitLimit / 4);
+      const int last = (bs + R.b_slots - 1) % R.b_slots;
+      const uint32_t par = (bs == 0) ? (bph ^ 1u) : bph;
+      ptx::mbar_drain(&B.b_empty[last], par, kWaitLimit / 4);
     }
     __syncwarp();
   } else {
@@ -633,7 +687,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         break;
       }
       if (!ok) break;
-      if (!wait_all(acc_full, acc_phase)) {
+      if (!wait_all(B.acc_full, acc_phase)) {
         ok = false;
         break;
       }
@@ -691,9 +745,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
       if (lane == 0) {
         if (CG2)
-          ptx::mbar_arrive_cluster(acc_empty, 0);
+          ptx::mbar_arrive_cluster(B.acc_empty, 0);
         else
-          ptx::mbar_arrive(acc_empty);
+          ptx::mbar_arrive(B.acc_empty);
       }
       if (threadIdx.x == 0) trace_stamp(a.trace, 7, item);
     }
