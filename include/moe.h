@@ -158,12 +158,27 @@ MOE_API moe_status moe_pack(const float* W, int32_t e0, int32_t ne, int32_t E, i
                     const uint8_t* fmt, void* out, uint64_t out_bytes, uint64_t* bytes_out,
                     uint64_t* code_off, uint64_t* scale_off, cudaStream_t stream);
 
+/* Activation formats of an NVFP4 layer's expert GEMMs (moe_weights.act). */
+enum {
+  MOE_ACT_FP8 = 0,    /* per-token dynamic FP8: x per token and the SwiGLU output h per row as
+                         e4m3 codes with scale amax/448 (MoE mixed-precision page, sec. 2.1) */
+  MOE_ACT_NVFP4 = 1   /* NVFP4 activations: x per token and h per row take the weights' NVFP4
+                         rule with the row as the tensor (s = amax/2688 in fp32, 1 for an
+                         all-zero row; e4m3 block scale per 16 = e4m3(blockmax/(6*s)); e2m1
+                         codes = e2m1(a/(sb*s)), 0 where sb = 0).  Prefill batches then run the
+                         block-scaled FP4 tensor-core MMA (tcgen05.mma kind::mxf4nvf4) on the
+                         codes and block scales of both operands, with s and the weights'
+                         tensor scale applied to the sums. */
+};
+
 /* A packed layer as moe_layer_forward reads it. */
 typedef struct {
   int32_t E, H, F;
   const uint8_t* fmt;   /* HOST [E*3]: must equal the fmt the buffer was packed with */
   const void* packed;   /* DEVICE, 256-byte aligned, written by moe_pack */
   uint64_t packed_bytes;
+  int32_t act;          /* MOE_ACT_*: activation format of an NVFP4 layer; 0 for integer layers
+                           (MOE_ERR_FORMAT otherwise) */
 } moe_weights;
 
 /* Optional outputs of moe_layer_forward; every pointer is DEVICE and nullable. */
@@ -201,6 +216,10 @@ typedef struct {
   uint32_t wait_cycles;   /* budget of the expert GEMMs' waits on their pipelines, in clock cycles;
                              0: the default (~1-2 s).  Waits for copies still in flight at exit keep
                              the default. */
+  uint8_t* xsb;       /* [T*H/16] MOE_ACT_NVFP4: e4m3 block scales of x (xq then holds one e2m1 code
+                         per byte, sx the row scales amax/2688) */
+  uint8_t* hsb;       /* [T*k*F/16] MOE_ACT_NVFP4: e4m3 block scales of h, sorted rows (hq: one e2m1
+                         code per byte; sh: row scales) */
 } moe_debug;
 
 #define MOE_TRACE_EVENTS 8
@@ -229,11 +248,14 @@ typedef struct {
  *   3. counts per expert, exclusive offsets and a stable permutation (rows of
  *      one expert in ascending token order);
  *   4. NVFP4 layers only: per-token dynamic FP8 e4m3 codes of x with scale
- *      amax/448 (MoE mixed-precision page sec. 2.1);
+ *      amax/448 (MoE mixed-precision page sec. 2.1), or with act =
+ *      MOE_ACT_NVFP4 per-token NVFP4 codes and block scales;
  *   5. per expert: h = silu(Wg x) * (Wu x) with fp32 accumulation on
  *      dequantized weights (integer formats: fp16 operands, weights rounded
- *      once to fp16 as s*q; NVFP4: exact bf16 operands, scales applied after
- *      the sum); NVFP4 layers then quantize each h row to e4m3 (amax/448);
+ *      once to fp16 as s*q; NVFP4: exact fp16 operands, scales applied after
+ *      the sum; NVFP4 activations in prefill: the block-scaled FP4 MMA on the
+ *      codes); NVFP4 layers then quantize each h row to e4m3 (amax/448), or
+ *      to NVFP4 with act = MOE_ACT_NVFP4;
  *   6. o = Wd h per row; y[t] = bf16( sum_j w[t][j] * o[row(t,j)] ) summed in
  *      fp32 in ascending j.
  * Integer-format layers run their expert GEMMs on fp16 operands.  A token

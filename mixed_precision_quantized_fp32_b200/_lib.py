@@ -13,6 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmoe_b200.so")
 
 MOE_STAGE_EVENTS = 8
+ACT_FP8, ACT_NVFP4 = 0, 1  # moe_weights.act
 MOE_TRACE_EVENTS = 8
 MOE_TRACE_STAGES = 1024
 
@@ -28,7 +29,7 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 
 class MoeWeights(C.Structure):
     _fields_ = [("E", C.c_int32), ("H", C.c_int32), ("F", C.c_int32), ("fmt", C.c_void_p),
-                ("packed", C.c_void_p), ("packed_bytes", C.c_uint64)]
+                ("packed", C.c_void_p), ("packed_bytes", C.c_uint64), ("act", C.c_int32)]
 
 
 class MoeDebug(C.Structure):
@@ -36,7 +37,8 @@ class MoeDebug(C.Structure):
                 ("inv", C.c_void_p), ("counts", C.c_void_p), ("xq", C.c_void_p), ("sx", C.c_void_p),
                 ("hq", C.c_void_p), ("sh", C.c_void_p), ("status", C.c_void_p),
                 ("stage_events", C.c_void_p), ("trace", C.c_void_p),
-                ("test_withhold", C.c_uint32), ("wait_cycles", C.c_uint32)]
+                ("test_withhold", C.c_uint32), ("wait_cycles", C.c_uint32), ("xsb", C.c_void_p),
+                ("hsb", C.c_void_p)]
 
 
 class MoeError(RuntimeError):

@@ -76,10 +76,11 @@ class PackedLayer:
     F: int
     fmt: np.ndarray       # host uint8 [E*3]
     packed: torch.Tensor  # cuda uint8, 256-byte aligned
+    act: int = 0          # NVFP4 layers: activation format (ACT_FP8 or ACT_NVFP4)
 
     def weights_struct(self) -> MoeWeights:
         return MoeWeights(self.E, self.H, self.F, self.fmt.ctypes.data, self.packed.data_ptr(),
-                          self.packed.numel())
+                          self.packed.numel(), self.act)
 
 
 def workspace_bytes(layer: PackedLayer, T: int, k: int) -> int:
@@ -91,7 +92,8 @@ def workspace_bytes(layer: PackedLayer, T: int, k: int) -> int:
     return int(need.value)
 
 
-DEBUG_FIELDS = ("topk_idx", "topk_w", "perm", "inv", "counts", "xq", "sx", "hq", "sh", "status", "trace")
+DEBUG_FIELDS = ("topk_idx", "topk_w", "perm", "inv", "counts", "xq", "sx", "hq", "sh", "status", "trace", "xsb",
+                "hsb")
 DEBUG_INTS = ("test_withhold", "wait_cycles")  # plain integers, see moe_debug in moe.h
 
 

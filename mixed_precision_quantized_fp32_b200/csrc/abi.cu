@@ -53,20 +53,22 @@ struct Plan {
 // Few rows per expert (decode): chunks of 8 rows on the streaming GEMV (warp
 // MMA); an expert with more rows gets several chunks, which read the same weight
 // tiles close in time (the second read hits L2).  Many rows per expert
-// (prefill): 256-row chunks on the tcgen05 kernel.
-Plan make_plan(int T, int k, int E) {
+// (prefill): 256-row chunks on the tcgen05 kernel (128 on the block-scaled FP4
+// kernel of NVFP4 activations).
+Plan make_plan(int T, int k, int E, bool act4) {
   Plan p;
   const long long R = (long long)T * k;
   const long long active = R < E ? R : E;
   const long long avg = active > 0 ? (R + active - 1) / active : 0;
   p.tc = avg > 32 && R >= 256;
-  p.chunk_rows = p.tc ? kTcChunkRows : 8;
+  p.chunk_rows = p.tc ? (act4 ? kFp4ChunkRows : kTcChunkRows) : 8;
   p.max_chunks = (int)(E + (R + p.chunk_rows - 1) / p.chunk_rows);
   return p;
 }
 
 // Carve the workspace; with base == nullptr only the size is computed.
-uint64_t carve(uint8_t* base, int T, int k, int E, int H, int F, bool fp4, const Plan& plan, Workspace* w) {
+uint64_t carve(uint8_t* base, int T, int k, int E, int H, int F, bool fp4, bool act4, const Plan& plan,
+               Workspace* w) {
   const uint64_t R = (uint64_t)T * k;
   const uint64_t nblk = (R + 1023) / 1024;
   uint64_t pos = 0;
@@ -95,12 +97,31 @@ uint64_t carve(uint8_t* base, int T, int k, int E, int H, int F, bool fp4, const
     ws.sx = (float*)take((uint64_t)T * 4);
   }
   if (!fp4) ws.xinv = (float*)take(R * 4);
-  ws.xs = take(R * H * 2);
-  ws.h = take(R * F * (fp4 ? 4 : 2));
-  if (fp4) {
-    ws.hb = take(R * F * 2);
-    ws.hq = (uint8_t*)take(R * F);
+  if (act4) {
+    // NVFP4 activations: block scales of x per token; prefill gathers codes + scales,
+    // decode gathers fp16 block values
+    ws.ldx = (H / 16 + 15) / 16 * 16;
+    ws.ldh = (F / 16 + 15) / 16 * 16;
+    ws.xsf = (uint8_t*)take((uint64_t)T * ws.ldx);
+    if (plan.tc) {
+      ws.xs4 = (uint8_t*)take(R * H / 2);
+      ws.xsf4 = (uint8_t*)take(R * ws.ldx);
+      ws.hs4 = (uint8_t*)take(R * F / 2);
+      ws.hsf4 = (uint8_t*)take(R * ws.ldh);
+    } else {
+      ws.xs = take(R * H * 2);
+      ws.hb = take(R * F * 2);
+    }
+    ws.h = take(R * F * 4);
     ws.sh = (float*)take(R * 4);
+  } else {
+    ws.xs = take(R * H * 2);
+    ws.h = take(R * F * (fp4 ? 4 : 2));
+    if (fp4) {
+      ws.hb = take(R * F * 2);
+      ws.hq = (uint8_t*)take(R * F);
+      ws.sh = (float*)take(R * 4);
+    }
   }
   ws.o = (float*)take(R * H * 4);
   if (!plan.tc) {
@@ -156,8 +177,11 @@ extern "C" moe_status moe_layer_forward(const void* x, int32_t T, const float* r
   const int kind = layer_kind(E, w->fmt);
   if (kind < 0) return MOE_ERR_FORMAT;
   const bool fp4 = kind == 1;
-  const Plan plan = make_plan(T, k, E);
-  const uint64_t need = carve(nullptr, T, k, E, H, F, fp4, plan, nullptr);
+  if (w->act != MOE_ACT_FP8 && w->act != MOE_ACT_NVFP4) return MOE_ERR_ARG;
+  if (w->act == MOE_ACT_NVFP4 && !fp4) return MOE_ERR_FORMAT;  // NVFP4 activations need an NVFP4 layer
+  const bool act4 = w->act == MOE_ACT_NVFP4;
+  const Plan plan = make_plan(T, k, E, act4);
+  const uint64_t need = carve(nullptr, T, k, E, H, F, fp4, act4, plan, nullptr);
   if (!ws) {
     if (!ws_bytes_out) return MOE_ERR_ARG;
     *ws_bytes_out = need;
@@ -177,7 +201,7 @@ extern "C" moe_status moe_layer_forward(const void* x, int32_t T, const float* r
   if (ds != MOE_OK) return ds;
 
   Workspace wsp;
-  carve((uint8_t*)ws, T, k, E, H, F, fp4, plan, &wsp);
+  carve((uint8_t*)ws, T, k, E, H, F, fp4, act4, plan, &wsp);
   moe_debug d{};
   if (dbg) d = *dbg;
   const __nv_bfloat16* xb = (const __nv_bfloat16*)x;
@@ -193,11 +217,16 @@ extern "C" moe_status moe_layer_forward(const void* x, int32_t T, const float* r
   if (launch_permute(T, k, E, plan.chunk_rows, wsp, d.counts, d.perm, d.inv, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (!mark(2)) return MOE_ERR_CUDA;
-  if (launch_gather(xb, T, H, k, fp4, wsp, d.xq, d.sx, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (act4) {
+    if (launch_gather_nvfp4(xb, T, H, k, plan.tc, wsp, d.xq, d.xsb, d.sx, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  } else if (launch_gather(xb, T, H, k, fp4, wsp, d.xq, d.sx, stream) != cudaSuccess) {
+    return MOE_ERR_CUDA;
+  }
   if (!mark(3)) return MOE_ERR_CUDA;
   int32_t* status = d.status ? d.status : wsp.status;
   auto gemm = [&](bool gateup) -> cudaError_t {
     const GemmHooks hooks{d.test_withhold, d.wait_cycles};
+    if (act4 && plan.tc) return launch_expert_gemm_fp4(packed, E, H, F, T, k, gateup, wsp, status, hooks, stream);
     return plan.tc ? launch_expert_gemm_tc(packed, w->fmt, E, H, F, T, k, fp4, gateup, wsp, status, d.trace, hooks,
                                            stream)
                    : launch_expert_gemv(packed, w->packed_bytes, w->fmt, E, H, F, T * k, k, fp4, gateup,
@@ -206,7 +235,11 @@ extern "C" moe_status moe_layer_forward(const void* x, int32_t T, const float* r
   };
   if (gemm(true) != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(4)) return MOE_ERR_CUDA;
-  if (fp4 && launch_act_quant_h(T * k, F, wsp, d.hq, d.sh, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (act4) {
+    if (launch_act_quant_h_nvfp4(T * k, F, plan.tc, wsp, d.hq, d.hsb, d.sh, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  } else if (fp4 && launch_act_quant_h(T * k, F, wsp, d.hq, d.sh, stream) != cudaSuccess) {
+    return MOE_ERR_CUDA;
+  }
   if (!mark(5)) return MOE_ERR_CUDA;
   if (gemm(false) != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(6)) return MOE_ERR_CUDA;

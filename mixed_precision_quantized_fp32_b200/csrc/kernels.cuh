@@ -30,8 +30,10 @@ struct GemmHooks {
   uint32_t wait_cycles;  // pipeline wait budget, 0: default
 };
 
-// Token rows per work chunk of the tcgen05 expert GEMMs (the MMA's largest N).
+// Token rows per work chunk of the tcgen05 expert GEMMs (the MMA's largest N):
+// fp16-operand GEMM, and the block-scaled FP4 GEMM of NVFP4 activations.
 constexpr int kTcChunkRows = 256;
+constexpr int kFp4ChunkRows = 128;
 
 cudaError_t launch_expert_gemm_tc(const uint8_t* packed, const uint8_t* fmt_host, int E, int H, int F, int T, int k,
                                   bool fp4, bool gateup, const Workspace& ws, int32_t* status, uint64_t* trace,
@@ -45,6 +47,16 @@ cudaError_t launch_expert_gemv(const uint8_t* packed, uint64_t packed_bytes, con
                                int F, int R, int k, bool fp4, bool gateup, int max_chunks, int chunk_rows,
                                const Workspace& ws, int32_t* status, uint64_t* trace, GemmHooks hooks,
                                cudaStream_t stream);
+
+// NVFP4 activations: per-token codes of x and their gather into sorted rows
+// (prefill: codes + block scales; decode: fp16 block values), and per-row codes of h.
+cudaError_t launch_gather_nvfp4(const __nv_bfloat16* x, int T, int H, int k, bool tc, const Workspace& ws,
+                                uint8_t* dbg_xq, uint8_t* dbg_xsb, float* dbg_sx, cudaStream_t stream);
+cudaError_t launch_act_quant_h_nvfp4(int R, int F, bool tc, const Workspace& ws, uint8_t* dbg_hq, uint8_t* dbg_hsb,
+                                     float* dbg_sh, cudaStream_t stream);
+// Block-scaled FP4 expert GEMM (prefill of NVFP4 layers with NVFP4 activations).
+cudaError_t launch_expert_gemm_fp4(const uint8_t* packed, int E, int H, int F, int T, int k, bool gateup,
+                                   const Workspace& ws, int32_t* status, GemmHooks hooks, cudaStream_t stream);
 
 cudaError_t launch_combine(int T, int k, int H, const Workspace& ws, __nv_bfloat16* y, cudaStream_t stream);
 

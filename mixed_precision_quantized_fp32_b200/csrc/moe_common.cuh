@@ -141,6 +141,13 @@ struct Workspace {
   float* xsum;         // [T*k][H/32] group sums of the gathered fp16 activations (integer layers)
   float* hsum;         // [T*k][F/32] group sums of the fp16 SwiGLU outputs (integer layers)
   float* xinv;         // [T*k] integer layers: 2^e undoing the power-of-two prescale of a row's x
+  // NVFP4 activations (moe_weights.act = MOE_ACT_NVFP4); xq then holds packed e2m1 codes [T][H/2]
+  int ldx, ldh;        // row pitch of the block-scale arrays of x and h (bytes, a multiple of 16)
+  uint8_t* xsf;        // [T][ldx] e4m3 block scales of x per token
+  uint8_t* xs4;        // [T*k][H/2] gathered codes of x (prefill)
+  uint8_t* xsf4;       // [T*k][ldx] gathered block scales of x (prefill)
+  uint8_t* hs4;        // [T*k][F/2] codes of h (prefill)
+  uint8_t* hsf4;       // [T*k][ldh] block scales of h (prefill)
 };
 
 }  // namespace moe

@@ -129,6 +129,39 @@ def oracle_forward_rows(layer_buf, x_bits, Wr, b, k, tokens=None, idx_override=N
     return y, idx, w
 
 
+def oracle_forward_rows_act4(layer_buf, x_bits, Wr, b, k, tokens=None, idx_override=None):
+    """As oracle_forward_rows for an NVFP4 layer with NVFP4 activations (the oracle's
+    NVFP4-activation mode, oracle/nvfp4_act.py): x per token and h per row quantized to
+    e2m1 codes with e4m3 block scales, products on the block values, the row and
+    tensor scales applied to the sums."""
+    from oracle import nvfp4_act as na
+    T = x_bits.shape[0]
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens)
+    xt = x_bits[tokens]
+    logits = orc.router(xt, Wr, b)
+    idx, w = orc.topk_softmax(logits, k)
+    if idx_override is not None:
+        idx = np.ascontiguousarray(idx_override[tokens], np.int32)
+        sel = np.take_along_axis(logits, idx, 1).astype(np.float64)
+        ex = np.exp(sel - sel.max(1, keepdims=True))
+        w = (ex / ex.sum(1, keepdims=True)).astype(np.float32)
+        order = np.argsort(-sel, axis=1, kind="stable")
+        idx = np.take_along_axis(idx, order, 1)
+        w = np.take_along_axis(w, order, 1)
+    xv, xsb, xs = na.quant_rows(gen.bf16_bits_to_f32(xt))
+    a = na.block_values(xv, xsb)
+    H = x_bits.shape[1]
+    y = np.zeros((len(tokens), H))
+    for e in np.unique(idx):
+        ts, js = np.nonzero(idx == e)
+        h = orc.gateup(layer_buf, int(e), a[ts], xs[ts].astype(np.float64))
+        hv, hsb, hs = na.quant_rows(h.astype(np.float32))
+        o = orc.down(layer_buf, int(e), na.block_values(hv, hsb), hs.astype(np.float64))
+        for r, (t, j) in enumerate(zip(ts, js)):
+            y[t] += float(w[t, j]) * o[r]
+    return y, idx, w
+
+
 def check_output(y_gpu_bf16, y_ref):
     """|y_gpu - y_ref| <= TOL * max|y_ref|; returns the error ratio."""
     import torch

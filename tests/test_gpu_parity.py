@@ -34,7 +34,7 @@ def custom(name, T, H, F, E, k, fmt, bias=None):
     return L
 
 
-def run_gpu(L, layer, T, x=None, Wr=None, b=None, k=None):
+def run_gpu(L, layer, T, x=None, Wr=None, b=None, k=None, act=0):
     k = k or L.k
     x = W.device_x(T, L.H) if x is None else x
     if Wr is None:
@@ -51,6 +51,9 @@ def run_gpu(L, layer, T, x=None, Wr=None, b=None, k=None):
                    sx=torch.empty(T, dtype=torch.float32, device="cuda"),
                    hq=torch.empty(R * L.F, dtype=torch.uint8, device="cuda"),
                    sh=torch.empty(R, dtype=torch.float32, device="cuda"))
+    if act:
+        dbg.update(xsb=torch.empty(T * L.H // 16, dtype=torch.uint8, device="cuda"),
+                   hsb=torch.empty(R * L.F // 16, dtype=torch.uint8, device="cuda"))
     # y inside a guard band: 4 KiB of a sentinel (exact in bf16) on each side must survive the call
     G, SENTINEL = 2048, -12288.0
     buf = torch.full((T * L.H + 2 * G,), SENTINEL, dtype=torch.bfloat16, device="cuda")
@@ -65,17 +68,20 @@ def run_gpu(L, layer, T, x=None, Wr=None, b=None, k=None):
     return out
 
 
-def check_layer(L, T, tokens=None, bias=None, router_zero=False, max_ties=None):
+def check_layer(L, T, tokens=None, bias=None, router_zero=False, max_ties=None, act=0):
     """Full parity of one layer / batch.  tokens: the subset whose outputs are
-    compared against the oracle (default all)."""
+    compared against the oracle (default all).  act: the activation format of an
+    NVFP4 layer (moe.ACT_NVFP4: the oracle's NVFP4-activation mode)."""
     k = L.k
     layer = hp.gpu_pack_cached(L) if L.name in W.NAMES else hp.gpu_pack(L)
+    if act:
+        layer = moe.PackedLayer(layer.E, layer.H, layer.F, layer.fmt, layer.packed, act)
     x_bits = W.x_bf16_bits(T, L.H)
     Wr_h = np.zeros((L.E, L.H), np.float32) if router_zero else W.router_w(L.E, L.H)
     b_h = bias if bias is not None else L.bias
     Wr = torch.from_numpy(Wr_h).cuda()
     b = None if b_h is None else torch.from_numpy(np.asarray(b_h, np.float32)).cuda()
-    g = run_gpu(L, layer, T, Wr=Wr, b=b)
+    g = run_gpu(L, layer, T, Wr=Wr, b=b, act=act)
 
     logits, idx_o, w_o = hp.oracle_route(x_bits, Wr_h, b_h, k)
     idx_g = g["topk_idx"].reshape(T, k)
@@ -90,7 +96,13 @@ def check_layer(L, T, tokens=None, bias=None, router_zero=False, max_ties=None):
     np.testing.assert_array_equal(g["counts"], counts)
     np.testing.assert_array_equal(g["perm"], perm)
     np.testing.assert_array_equal(g["inv"], inv)
-    if L.fp4:
+    if L.fp4 and act:
+        from oracle import nvfp4_act as na
+        xv, xsb, xs = na.quant_rows(gen.bf16_bits_to_f32(x_bits))
+        np.testing.assert_array_equal(g["xq"].reshape(T, L.H), xv)
+        np.testing.assert_array_equal(g["xsb"].reshape(T, L.H // 16), xsb)
+        np.testing.assert_array_equal(g["sx"], xs)
+    elif L.fp4:
         xq, sx = orc.act_quant_e4m3(gen.bf16_bits_to_f32(x_bits))
         np.testing.assert_array_equal(g["xq"].reshape(T, L.H), xq)
         np.testing.assert_array_equal(g["sx"], sx)
@@ -100,8 +112,12 @@ def check_layer(L, T, tokens=None, bias=None, router_zero=False, max_ties=None):
     tokens = np.arange(T) if tokens is None else np.asarray(tokens)
     experts = np.unique(np.concatenate([idx_o[tokens].ravel(), idx_g[tokens].ravel()]))
     buf = hp.oracle_pack(L, experts)
-    y_ref, _, _ = hp.oracle_forward_rows(buf, x_bits, Wr_h, b_h, k, tokens=tokens,
-                                         idx_override=idx_g if ties else None, fp4=L.fp4)
+    if act:
+        y_ref, _, _ = hp.oracle_forward_rows_act4(buf, x_bits, Wr_h, b_h, k, tokens=tokens,
+                                                  idx_override=idx_g if ties else None)
+    else:
+        y_ref, _, _ = hp.oracle_forward_rows(buf, x_bits, Wr_h, b_h, k, tokens=tokens,
+                                             idx_override=idx_g if ties else None, fp4=L.fp4)
     ratio = hp.check_output(g["y"][torch.from_numpy(tokens).cuda()], y_ref)
     return dict(ties=len(ties), err_ratio=ratio, counts=g["counts"], n_tokens=len(tokens))
 
@@ -506,6 +522,75 @@ def test_stage_events_record():
     torch.cuda.synchronize()
     times = [ev[i].elapsed_time(ev[i + 1]) for i in range(len(ev) - 1)]
     assert all(t >= 0 for t in times) and ev[0].elapsed_time(ev[-1]) > 0
+
+
+# ------------------------------------------------------------------ NVFP4 activations (block-scaled FP4 MMA)
+@pytest.mark.parametrize("T", [9, 300])
+def test_nvfp4_activations_small(T):
+    # x and h quantized to NVFP4 (e2m1 + e4m3 per 16 + fp32 row scale): x codes, block scales
+    # and row scales bit-exact, outputs within the bound.  T=9 runs the decode GEMV on fp16
+    # block values, T=300 the block-scaled FP4 tcgen05 GEMM (chunks of up to 128 rows).
+    L = custom("act4", T, 256, 384, 6, 2, [[16, 16, 16]] * 6)
+    check_layer(L, T, act=moe.ACT_NVFP4)
+
+
+@pytest.mark.parametrize("T", [7, 260])
+def test_nvfp4_activations_half_stages_odd_tiles(T):
+    # H = 384 and F = 640: the FP4 GEMM's last 256-input stage holds one 128-input tile
+    # (K % 256 = 128) for both GEMMs, and the down projection has three 128-row tiles (the
+    # last item holds one tile).
+    L = custom("act4odd", T, 384, 640, 5, 2, [[16, 16, 16]] * 5)
+    check_layer(L, T, act=moe.ACT_NVFP4)
+
+
+def test_nvfp4_activations_down_stage_refeed():
+    # the GPU's NVFP4 codes of h (row scale, block scales, codes) fed into the oracle's down
+    # stage: output parity of the down GEMM + combine alone; the h codes themselves depend on
+    # summation order and are counted (at most 1% may differ)
+    from oracle import nvfp4_act as na
+    T, k = 300, 2
+    L = custom("act4refeed", T, 256, 256, 4, k, [[16, 16, 16]] * 4)
+    layer = hp.gpu_pack(L)
+    layer = moe.PackedLayer(layer.E, layer.H, layer.F, layer.fmt, layer.packed, moe.ACT_NVFP4)
+    g = run_gpu(L, layer, T, act=moe.ACT_NVFP4)
+    x_bits = W.x_bf16_bits(T, L.H)
+    buf = hp.oracle_pack(L, range(L.E))
+    idx = g["topk_idx"].reshape(T, k)
+    counts, offsets, perm, inv = orc.permute(idx.astype(np.int32), L.E)
+    hq = g["hq"].reshape(T * k, L.F)
+    hsb = g["hsb"].reshape(T * k, L.F // 16)
+    sh = g["sh"]
+    o = np.zeros((T * k, L.H))
+    for e in range(L.E):
+        r0, r1 = offsets[e], offsets[e + 1]
+        if r1 > r0:
+            o[r0:r1] = orc.down(buf, e, na.block_values(hq[r0:r1], hsb[r0:r1]), sh[r0:r1].astype(np.float64))
+    w = g["topk_w"].reshape(T, k)
+    y_ref = np.zeros((T, L.H))
+    for t in range(T):
+        for j in range(k):
+            y_ref[t] += float(w[t, j]) * o[inv[t * k + j]]
+    hp.check_output(g["y"], y_ref)
+    xv, xsb, xs = na.quant_rows(gen.bf16_bits_to_f32(x_bits))
+    a = na.block_values(xv, xsb)
+    n_diff = 0
+    for e in range(L.E):
+        r0, r1 = offsets[e], offsets[e + 1]
+        if r1 > r0:
+            ts = perm[r0:r1] // k
+            h = orc.gateup(buf, e, a[ts], xs[ts].astype(np.float64))
+            hv, _, _ = na.quant_rows(h.astype(np.float32))
+            n_diff += int(np.count_nonzero(hv != hq[r0:r1]))
+    assert n_diff <= 0.01 * hq.size, f"{n_diff} of {hq.size} h codes differ"
+
+
+@pytest.mark.parametrize("T", [16, 8192])
+def test_forward_nvfp4_layer_nvfp4_activations(T):
+    # the 256-expert top-6 NVFP4 layer with NVFP4 activations: decode T=16 (all tokens) and
+    # prefill T=8192 (every expert's first and last rows plus 256 seeded tokens)
+    L = W.layer("nvfp4")
+    r = check_layer(L, T, tokens=strata(halves=False, extra=256) if T > 64 else None, act=moe.ACT_NVFP4)
+    print(f"nvfp4 act4 T={T}: near-ties {r['ties']}, err/max {r['err_ratio']:.3g}, tokens compared {r['n_tokens']}")
 
 
 # ------------------------------------------------------------------ forward, the five layers
