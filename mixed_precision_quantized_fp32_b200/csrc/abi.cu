@@ -226,7 +226,8 @@ extern "C" moe_status moe_layer_forward(const void* x, int32_t T, const float* r
   int32_t* status = d.status ? d.status : wsp.status;
   auto gemm = [&](bool gateup) -> cudaError_t {
     const GemmHooks hooks{d.test_withhold, d.wait_cycles};
-    if (act4 && plan.tc) return launch_expert_gemm_fp4(packed, E, H, F, T, k, gateup, wsp, status, hooks, stream);
+    if (act4 && plan.tc)
+      return launch_expert_gemm_fp4(packed, E, H, F, T, k, gateup, wsp, status, d.trace, hooks, stream);
     return plan.tc ? launch_expert_gemm_tc(packed, w->fmt, E, H, F, T, k, fp4, gateup, wsp, status, d.trace, hooks,
                                            stream)
                    : launch_expert_gemv(packed, w->packed_bytes, w->fmt, E, H, F, T * k, k, fp4, gateup,

@@ -68,9 +68,15 @@ struct F4Args {
   int topk;
   float* out;               // gate/up: h [rows][F]; down: o [rows][H]
   int32_t* status;
+  unsigned long long* trace;  // diagnostics: clock64 stamps of CTA 0 (or null)
   long long wait;
   int withhold;
 };
+
+// Stamp event `ev` of index `i` (CTA 0 only, first MOE_TRACE_STAGES indices).
+__device__ __forceinline__ void f4_trace(unsigned long long* tr, int ev, int i) {
+  if (tr && blockIdx.x == 0 && i < MOE_TRACE_STAGES) tr[ev * MOE_TRACE_STAGES + i] = (unsigned long long)clock64();
+}
 
 __device__ __forceinline__ int swz128(int row, int chunk) {
   return (row >> 3) * 1024 + (row & 7) * 128 + ((chunk ^ (row & 7)) << 4);
@@ -158,7 +164,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
   };
 
   if (warp == kF4LoadWarp) {
-    int s = 0;
+    int s = 0, g = 0;
     uint32_t ph = 0, issued = 0, issued_phase = 0;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const int c = t / m_items, mi = t % m_items;
@@ -180,6 +186,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         }
         const int nt = min(2, ktiles - 2 * ks);  // 128-input tiles in this stage
         if (lane == 0 && !a.withhold) {
+          f4_trace(a.trace, 0, g);
           uint8_t* sb = smem + s * kF4SlotBytes;
           const uint32_t bytes = (uint32_t)nmat * (uint32_t)nt * 9216u + 16384u + 2048u;  // codes + scales, B, B scales
           ptx::mbar_arrive_expect_tx(&full[s], bytes);
@@ -191,7 +198,9 @@ __global__ void __launch_bounds__(kF4Threads, 1)
           }
           ptx::tma_load_2d(sb + kF4OffB, &tmap_b, ks * 128, row0, &full[s]);
           ptx::tma_load_2d(sb + kF4OffSfbRaw, &tmap_sfb, ks * 16, row0, &full[s]);
+          f4_trace(a.trace, 1, g);
         }
+        ++g;
         __syncwarp();
         if (!a.withhold) {
           issued |= 1u << s;
@@ -207,7 +216,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       if (issued & (1u << s2)) ptx::mbar_drain(&full[s2], (issued_phase >> s2) & 1u, kF4WaitLimit / 4);
     __syncwarp();
   } else if (warp == kF4MmaWarp) {
-    int s = 0;
+    int s = 0, g = 0;
     uint32_t ph = 0, acc_phase = 0;
     const uint32_t sb0 = ptx::smem_u32(smem);
     bool committed = false;
@@ -227,6 +236,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
           break;
         }
         ptx::tc_fence_after();
+        if (lane == 0) f4_trace(a.trace, 4, g);
         const uint32_t sb = sb0 + (uint32_t)(s * kF4SlotBytes);
         // this stage's scale atoms to TMEM (after the previous stage's MMAs, in issue order)
 #pragma unroll
@@ -244,6 +254,8 @@ __global__ void __launch_bounds__(kF4Threads, 1)
             mma_fp4_warp(tmem + (uint32_t)(m * kF4BN), da + (uint64_t)(m * (16384 >> 4) + 2 * j), db + (uint64_t)(2 * j),
                          idesc, tmem + kF4TmemSfa + 16u * m + 4u * j, tmem + kF4TmemSfb + 4u * j, j ? 1u : acc0);
         ptx::mma_commit_warp(&empty[s]);
+        if (lane == 0) f4_trace(a.trace, 5, g);
+        ++g;
         __syncwarp();
         committed = true;
         if (++s == kF4Slots) {
@@ -263,7 +275,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
   } else {
     // ---------------------------------------------------------- rearrange + epilogue (warps 0-7)
     const int n = threadIdx.x & 127, half = threadIdx.x >> 7;  // weight row (or token row), which 128-input tile
-    int s = 0;
+    int s = 0, g = 0, item = 0;
     uint32_t ph = 0, acc_phase = 0;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const int c = t / m_items, mi = t % m_items;
@@ -274,6 +286,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
           ok = false;
           break;
         }
+        if (threadIdx.x == 0) f4_trace(a.trace, 2, g);
         const int nt = min(2, ktiles - 2 * ks);
         const bool have = half < nt;  // this thread's 128-input tile exists
         const uint32_t sb = ptx::smem_u32(smem) + (uint32_t)(s * kF4SlotBytes);
@@ -331,6 +344,8 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         ptx::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&ready[s]);
+        if (threadIdx.x == 0) f4_trace(a.trace, 3, g);
+        ++g;
         if (++s == kF4Slots) {
           s = 0;
           ph ^= 1u;
@@ -343,37 +358,55 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       }
       acc_phase ^= 1u;
       ptx::tc_fence_after();
-      // epilogue: warp w reads TMEM lane quarter w%4, columns [64*(w/4), +64)
+      if (threadIdx.x == 0) f4_trace(a.trace, 6, item);
+      // epilogue: warp w reads TMEM lane quarter w%4, columns (tokens) [64*(w/4), +64)
       const int q = warp & 3, ch = warp >> 2;
       const int nrow0 = (gate_up ? mi : 2 * mi) * kF4BM + q * 32 + lane;
       float ts[2];
 #pragma unroll
       for (int m = 0; m < 2; ++m) ts[m] = L.tscale[e * 3 + (gate_up ? m : 2)];
+      // the warp's 64 token scales, two per lane, loaded before any store (they are
+      // broadcast with shuffles below)
+      float scl[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int tok = ch * 64 + 32 * u + lane;
+        scl[u] = 0.0f;
+        if (tok < rows) {
+          const int r = row0 + tok;
+          scl[u] = gate_up ? a.row_scale[a.perm[r] / a.topk] : a.row_scale[r];
+        }
+      }
+      float* __restrict__ out = a.out;
       const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
       for (int cb = ch * 64; cb < ch * 64 + 64 && cb < rows; cb += 16) {
         uint32_t r0[16], r1[16];
         ptx::tmem_ld16(lane_base + (uint32_t)cb, r0);
         ptx::tmem_ld16(lane_base + (uint32_t)(kF4BN + cb), r1);
         ptx::tmem_ld_wait();
+        const int u = (cb - ch * 64) >> 5;  // which of the lane's two scales (warp-uniform)
+        const float su = u ? scl[1] : scl[0];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int tok = cb + j;
-          if (tok >= rows) break;
-          const int r = row0 + tok;
+          const float sc = __shfl_sync(0xffffffffu, su, (tok - ch * 64) & 31);
+          if (tok >= rows) continue;
+          const size_t o = (size_t)(row0 + tok) * a.N + nrow0;
           if (gate_up) {
-            const float sx = a.row_scale[a.perm[r] / a.topk];
-            const float g = __uint_as_float(r0[j]) * (sx * ts[0]), u = __uint_as_float(r1[j]) * (sx * ts[1]);
-            a.out[(size_t)r * a.N + nrow0] = __fdividef(g, 1.0f + __expf(-g)) * u;
+            const float g = __uint_as_float(r0[j]) * (sc * ts[0]), uu = __uint_as_float(r1[j]) * (sc * ts[1]);
+            out[o] = __fdividef(g, 1.0f + __expf(-g)) * uu;
           } else {
-            const float sc = a.row_scale[r] * ts[0];
-            a.out[(size_t)r * a.N + nrow0] = __uint_as_float(r0[j]) * sc;
-            if (nmat == 2) a.out[(size_t)r * a.N + nrow0 + kF4BM] = __uint_as_float(r1[j]) * sc;
+            const float f = sc * ts[0];
+            out[o] = __uint_as_float(r0[j]) * f;
+            if (nmat == 2) out[o + kF4BM] = __uint_as_float(r1[j]) * f;
           }
         }
       }
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(acc_empty);
+      if (threadIdx.x == 0) f4_trace(a.trace, 7, item);
+      ++item;
     }
   }
 
@@ -429,8 +462,10 @@ bool encode_bytes_map(CUtensorMap* map, const void* base, int rows, int cols, in
 }  // namespace
 
 cudaError_t launch_expert_gemm_fp4(const uint8_t* packed, int E, int H, int F, int T, int k, bool gateup,
-                                   const Workspace& ws, int32_t* status, GemmHooks hooks, cudaStream_t stream) {
+                                   const Workspace& ws, int32_t* status, uint64_t* trace, GemmHooks hooks,
+                                   cudaStream_t stream) {
   F4Args a{};
+  a.trace = gateup ? reinterpret_cast<unsigned long long*>(trace) : nullptr;
   a.packed = packed;
   a.E = E;
   a.H = H;

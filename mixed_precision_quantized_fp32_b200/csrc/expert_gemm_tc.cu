@@ -697,46 +697,70 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int nrow = (a.pair ? 2 * mt : mt) * kTcBM + q * 32 + lane;
       const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
       bool range = false;  // an fp16 SwiGLU output overflowed
-      for (int cb = cq * kColsPerWarp; cb < cq * kColsPerWarp + kColsPerWarp && cb < rows; cb += 16) {
-        uint32_t r0[16], r1[16];
-        ptx::tmem_ld16(lane_base + (uint32_t)cb, r0);
-        if (NMAT == 2) ptx::tmem_ld16(lane_base + 256u + (uint32_t)cb, r1);
-        ptx::tmem_ld_wait();
+      if (a.row_scale) {
+        // NVFP4 layers: the row scales of the warp's kColsPerWarp tokens (gate/up: the
+        // token's sx through perm; down: the row's sh), two per lane, loaded before any
+        // store and broadcast with shuffles -- loaded inside the store loop, each would
+        // wait for the stores before it.
+        static_assert(kColsPerWarp == 64, "two token scales per lane");
+        float fac[2] = {0.0f, 0.0f};
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int tok = cb + j;
-          if (tok >= rows) break;
-          const int r = row0 + tok;
-          if (NMAT == 2 && a.pair) {  // two weight tiles of the down matrix: rows nrow and nrow + 128
-            float o0 = __uint_as_float(r0[j]), o1 = __uint_as_float(r1[j]);
-            if (a.row_scale) {
-              const float sc = a.row_scale[r] * tsc[0];
-              o0 *= sc;
-              o1 *= sc;
-            }
-            reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = o0;
-            reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow + kTcBM] = o1;
-          } else if (NMAT == 2) {
-            float g = __uint_as_float(r0[j]), u = __uint_as_float(r1[j]);
-            if (a.row_scale) {
-              const float sx = a.row_scale[a.perm[r] / a.topk];
-              g *= sx * tsc[0];
-              u *= sx * tsc[1];
-              reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = __fdividef(g, 1.0f + __expf(-g)) * u;
+        for (int u2 = 0; u2 < 2; ++u2) {
+          const int tok = cq * kColsPerWarp + 32 * u2 + lane;
+          if (tok < rows) {
+            const int r = row0 + tok;
+            fac[u2] = (NMAT == 2 && !a.pair) ? a.row_scale[a.perm[r] / a.topk] : a.row_scale[r];
+          }
+        }
+        float* __restrict__ out = reinterpret_cast<float*>(a.out);
+        for (int cb = cq * kColsPerWarp; cb < cq * kColsPerWarp + kColsPerWarp && cb < rows; cb += 16) {
+          uint32_t r0[16], r1[16];
+          ptx::tmem_ld16(lane_base + (uint32_t)cb, r0);
+          if (NMAT == 2) ptx::tmem_ld16(lane_base + 256u + (uint32_t)cb, r1);
+          ptx::tmem_ld_wait();
+          const float fu = ((cb - cq * kColsPerWarp) >> 5) ? fac[1] : fac[0];  // warp-uniform choice
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int tok = cb + j;
+            const float f = __shfl_sync(0xffffffffu, fu, (tok - cq * kColsPerWarp) & 31);
+            if (tok >= rows) continue;
+            const size_t o = (size_t)(row0 + tok) * a.N + nrow;
+            if (NMAT == 2 && a.pair) {  // two weight tiles of the down matrix: rows nrow and nrow + 128
+              const float sc = f * tsc[0];
+              out[o] = __uint_as_float(r0[j]) * sc;
+              out[o + kTcBM] = __uint_as_float(r1[j]) * sc;
+            } else if (NMAT == 2) {
+              const float g = __uint_as_float(r0[j]) * (f * tsc[0]), u = __uint_as_float(r1[j]) * (f * tsc[1]);
+              out[o] = __fdividef(g, 1.0f + __expf(-g)) * u;
             } else {
-              if (a.xinv) {
-                const float xi = a.xinv[r];
-                g *= xi;
-                u *= xi;
-              }
+              out[o] = __uint_as_float(r0[j]) * (f * tsc[0]);
+            }
+          }
+        }
+      } else {
+        // integer layers: SwiGLU into fp16 h (gate/up) or fp32 o (down)
+        for (int cb = cq * kColsPerWarp; cb < cq * kColsPerWarp + kColsPerWarp && cb < rows; cb += 16) {
+          uint32_t r0[16], r1[16];
+          ptx::tmem_ld16(lane_base + (uint32_t)cb, r0);
+          if (NMAT == 2) ptx::tmem_ld16(lane_base + 256u + (uint32_t)cb, r1);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int tok = cb + j;
+            if (tok >= rows) break;
+            const int r = row0 + tok;
+            if (NMAT == 2 && a.pair) {  // two weight tiles of the down matrix: rows nrow and nrow + 128
+              reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = __uint_as_float(r0[j]);
+              reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow + kTcBM] = __uint_as_float(r1[j]);
+            } else if (NMAT == 2) {
+              const float xi = a.xinv[r];  // 2^e: exact, 1 unless the token was prescaled
+              const float g = __uint_as_float(r0[j]) * xi, u = __uint_as_float(r1[j]) * xi;
               const __half h = __float2half_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
               range |= __hisinf(h) != 0;
               reinterpret_cast<__half*>(a.out)[(size_t)r * a.N + nrow] = h;
+            } else {
+              reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = __uint_as_float(r0[j]);
             }
-          } else {
-            float o = __uint_as_float(r0[j]);
-            if (a.row_scale) o *= a.row_scale[r] * tsc[0];
-            reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = o;
           }
         }
       }

@@ -56,7 +56,8 @@ cudaError_t launch_act_quant_h_nvfp4(int R, int F, bool tc, const Workspace& ws,
                                      float* dbg_sh, cudaStream_t stream);
 // Block-scaled FP4 expert GEMM (prefill of NVFP4 layers with NVFP4 activations).
 cudaError_t launch_expert_gemm_fp4(const uint8_t* packed, int E, int H, int F, int T, int k, bool gateup,
-                                   const Workspace& ws, int32_t* status, GemmHooks hooks, cudaStream_t stream);
+                                   const Workspace& ws, int32_t* status, uint64_t* trace, GemmHooks hooks,
+                                   cudaStream_t stream);
 
 cudaError_t launch_combine(int T, int k, int H, const Workspace& ws, __nv_bfloat16* y, cudaStream_t stream);
 
