@@ -80,7 +80,13 @@ enum {
   MOE_FMT_INT2 = 2,   /* symmetric codes {-1,0,1}, fp16 scale per 32 inputs */
   MOE_FMT_INT3 = 3,   /* symmetric codes [-3,3],   fp16 scale per 32 inputs */
   MOE_FMT_INT4 = 4,   /* symmetric codes [-7,7],   fp16 scale per 32 inputs */
-  MOE_FMT_NVFP4 = 16  /* e2m1 codes, e4m3 scale per 16 inputs, fp32 scale per matrix */
+  MOE_FMT_NVFP4 = 16, /* e2m1 codes, e4m3 scale per 16 inputs, fp32 scale per matrix */
+  MOE_FMT_OUTLIERS = 0x80  /* flag OR'ed onto a format code: the matrix keeps its top 0.05% of
+                              weights by |w| (floor(N*K*5/10000), ties to the lower row-major
+                              index) in an fp16 side list; they are zeroed before the group
+                              quantization and their residual w - dequant(w) is added back in the
+                              expert GEMMs (MoE mixed-precision page sec. 4.2, tip 2).  Integer
+                              and NVFP4 matrices with FP8 activations. */
 };
 
 /*
@@ -88,10 +94,12 @@ enum {
  *
  * Header, 16384 bytes:
  *   [0]     u32 magic 0x51454F4D        [4]  u32 version 1
- *   [8]     i32 E   [12] i32 H   [16] i32 F   [20..32) zero
- *   [32]    u8  fmt[768]        formats of (expert e, projection p) at e*3+p,
- *                               p = 0 gate [F x H], 1 up [F x H], 2 down [H x F];
- *                               entries past E*3 are zero
+ *   [8]     i32 E   [12] i32 H   [16] i32 F
+ *   [20]    u32 flags           bit 0: the layer has an outlier section (else 0)
+ *   [24]    u64 out_sec         byte offset of the outlier section (0 if none)
+ *   [32]    u8  fmt[768]        base formats (without MOE_FMT_OUTLIERS) of (expert e,
+ *                               projection p) at e*3+p, p = 0 gate [F x H], 1 up [F x H],
+ *                               2 down [H x F]; entries past E*3 are zero
  *   [800]   u64 code_off[768]   byte offset of each matrix's codes
  *   [6944]  u64 scale_off[768]  byte offset of each matrix's scales
  *   [13088] f32 tscale[768]     NVFP4 per-matrix scale (0 for integer formats)
@@ -134,6 +142,21 @@ enum {
  *          P = 8*(c/2) + c%2 + 2j and code 2m+1 at bit 16+P
  *   NVFP4: codes 8w..8w+7 in word w, code 8w+i at bits 4i..4i+3.
  * Scale layout: [N/128][K/gs][128] (gs = 32 integer, 16 NVFP4).
+ *
+ * Outlier section (present when any fmt code carries MOE_FMT_OUTLIERS), at the
+ * first 256-byte boundary after the last expert section:
+ *   u64 side_off[768]       byte offset of each matrix's side list (0 if none)
+ *   u32 scratch[64 + 65536] selection state of moe_pack (contents unspecified)
+ * then, from the next 256-byte boundary, one side list per opted-in matrix in
+ * (expert, projection) order, each on a 256-byte boundary:
+ *   u32 row_ptr[N+1]        row n's entries are [row_ptr[n], row_ptr[n+1])
+ *   u32 entry[n_out]        column | (fp16 residual bits << 16), in (row, column)
+ *                           order; n_out = floor(N*K*5/10000)
+ * The residual is w - dequant at that position, taken in double and rounded
+ * once to fp16: w itself for every format with a zero code, w - s for the
+ * 1-bit sign code (a zeroed weight reads +s).  The layer computes with
+ * dequant(codes) + residual.  The quantization above then sees the matrix with
+ * its outliers set to 0 (group scales, NVFP4 sT and block scales included).
  */
 
 /*
@@ -148,7 +171,9 @@ enum {
  *   (DEVICE, 256-byte aligned, out_bytes >= the queried size), so a layer too
  *   large to stage in fp32 can be packed a few experts at a time.
  *   W: DEVICE fp32 [ne][3][H*F] -- gate [F][H], up [F][H], down [H][F],
- *   row-major, 16-byte aligned.  fmt: HOST u8 [E*3].
+ *   row-major, 16-byte aligned.  fmt: HOST u8 [E*3], a format code per matrix,
+ *   optionally OR'ed with MOE_FMT_OUTLIERS.  moe_layer_forward must be given the
+ *   same codes (flags included) as moe_pack.
  * Shapes: 1 <= E <= 256; H, F multiples of 128 (up to 32768).
  * Errors: MOE_ERR_ARG (null W/fmt/bytes_out, bad e0/ne), MOE_ERR_SHAPE,
  *   MOE_ERR_FORMAT, MOE_ERR_ALIGN, MOE_ERR_WORKSPACE (out_bytes too small),
@@ -264,7 +289,10 @@ typedef struct {
  * x is accepted.  The SwiGLU output h is stored in fp16: an |h| that rounds
  * beyond 65504 writes MOE_ERR_RANGE to moe_debug.status (y is then not
  * finite).  NVFP4 layers scale x and h per row and have no such limit.
- * Layers must be all-NVFP4 or all-integer (MOE_ERR_FORMAT).
+ * Layers must be all-NVFP4 or all-integer (MOE_ERR_FORMAT).  Matrices packed
+ * with MOE_FMT_OUTLIERS add their side lists' residuals to the GEMM sums in
+ * the epilogues (fp32, the row's activations as the GEMM reads them); with
+ * MOE_ACT_NVFP4 activations such a layer is rejected (MOE_ERR_FORMAT).
  * Errors: MOE_ERR_ARG, MOE_ERR_ALIGN, MOE_ERR_SHAPE, MOE_ERR_FORMAT,
  *   MOE_ERR_WORKSPACE, MOE_ERR_UNSUPPORTED_DEVICE, MOE_ERR_CUDA.
  */

@@ -13,7 +13,8 @@ import torch
 from . import _lib
 from ._lib import MoeDebug, MoeError, MoeWeights, check
 
-FMT_INT2, FMT_INT3, FMT_INT4, FMT_NVFP4 = 2, 3, 4, 16
+FMT_INT1, FMT_INT2, FMT_INT3, FMT_INT4, FMT_NVFP4 = 1, 2, 3, 4, 16
+FMT_OUTLIERS = 0x80  # or-ed into a format code: the matrix keeps its top 0.05% |w| in an fp16 side list
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:

@@ -34,6 +34,7 @@ bool shape_ok(int E, int H, int F) {
 }
 
 // Layer kind: 0 = all integer, 1 = all NVFP4, -1 = unknown code or a mix.
+// fmt: base formats.
 int layer_kind(int E, const uint8_t* fmt) {
   int n_fp4 = 0;
   for (int i = 0; i < 3 * E; ++i) {
@@ -140,6 +141,30 @@ uint64_t carve(uint8_t* base, int T, int k, int E, int H, int F, bool fp4, bool 
   return pos;
 }
 
+// The caller's format codes split into base formats (what the kernels decode) and
+// whether any matrix keeps an outlier side list.  Returns false on an unknown flag.
+bool split_fmt(int E, const uint8_t* fmt, uint8_t* base, bool* any_out) {
+  *any_out = false;
+  for (int i = 0; i < 3 * E; ++i) {
+    if (fmt[i] & ~(MOE_FMT_OUTLIERS | 0x1F)) return false;
+    base[i] = (uint8_t)fmt_base(fmt[i]);
+    *any_out |= fmt_outliers(fmt[i]);
+  }
+  return true;
+}
+
+// Full layout: expert sections (base formats) then the outlier section.
+bool full_layout(int E, int H, int F, const uint8_t* fmt, uint64_t* co, uint64_t* so, uint64_t* side,
+                 uint64_t* out_sec, uint64_t* total) {
+  uint8_t base[3 * kMaxE];
+  bool any = false;
+  if (!split_fmt(E, fmt, base, &any)) return false;
+  uint64_t end = 0;
+  if (!layer_layout(E, H, F, base, co, so, &end)) return false;
+  *out_sec = outlier_layout(E, H, F, fmt, end, side, total);
+  return true;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -150,8 +175,8 @@ extern "C" moe_status moe_pack(const float* W, int32_t e0, int32_t ne, int32_t E
                                uint64_t* code_off, uint64_t* scale_off, cudaStream_t stream) {
   if (!fmt) return MOE_ERR_ARG;
   if (!shape_ok(E, H, F)) return MOE_ERR_SHAPE;
-  uint64_t co[3 * kMaxE], so[3 * kMaxE], total = 0;
-  if (!layer_layout(E, H, F, fmt, co, so, &total)) return MOE_ERR_FORMAT;
+  uint64_t co[3 * kMaxE], so[3 * kMaxE], side[3 * kMaxE], total = 0, out_sec = 0;
+  if (!full_layout(E, H, F, fmt, co, so, side, &out_sec, &total)) return MOE_ERR_FORMAT;
   if (code_off) std::memcpy(code_off, co, sizeof(uint64_t) * 3 * E);
   if (scale_off) std::memcpy(scale_off, so, sizeof(uint64_t) * 3 * E);
   if (bytes_out) *bytes_out = total;
@@ -162,7 +187,8 @@ extern "C" moe_status moe_pack(const float* W, int32_t e0, int32_t ne, int32_t E
   if (out_bytes < total) return MOE_ERR_WORKSPACE;
   const moe_status ds = check_device();
   if (ds != MOE_OK) return ds;
-  if (launch_pack(W, e0, ne, E, H, F, fmt, (uint8_t*)out, co, so, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_pack(W, e0, ne, E, H, F, fmt, (uint8_t*)out, co, so, out_sec, side, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return MOE_OK;
 }
 
@@ -174,11 +200,15 @@ extern "C" moe_status moe_layer_forward(const void* x, int32_t T, const float* r
   if (!shape_ok(E, H, F)) return MOE_ERR_SHAPE;
   if (T < 0 || k < 1 || k > kMaxK || k > E) return MOE_ERR_SHAPE;
   if ((long long)T * k > (1LL << 20)) return MOE_ERR_SHAPE;
-  const int kind = layer_kind(E, w->fmt);
+  uint8_t fmt[3 * kMaxE];  // base formats
+  bool outliers = false;
+  if (!split_fmt(E, w->fmt, fmt, &outliers)) return MOE_ERR_FORMAT;
+  const int kind = layer_kind(E, fmt);
   if (kind < 0) return MOE_ERR_FORMAT;
   const bool fp4 = kind == 1;
   if (w->act != MOE_ACT_FP8 && w->act != MOE_ACT_NVFP4) return MOE_ERR_ARG;
   if (w->act == MOE_ACT_NVFP4 && !fp4) return MOE_ERR_FORMAT;  // NVFP4 activations need an NVFP4 layer
+  if (w->act == MOE_ACT_NVFP4 && outliers) return MOE_ERR_FORMAT;  // side lists: FP8 activations only
   const bool act4 = w->act == MOE_ACT_NVFP4;
   const Plan plan = make_plan(T, k, E, act4);
   const uint64_t need = carve(nullptr, T, k, E, H, F, fp4, act4, plan, nullptr);
@@ -193,8 +223,8 @@ extern "C" moe_status moe_layer_forward(const void* x, int32_t T, const float* r
   if (!aligned(x, 16) || !aligned(y, 16) || !aligned(router_w, 16) || !aligned(w->packed, 256) ||
       !aligned(ws, 256))
     return MOE_ERR_ALIGN;
-  uint64_t total = 0;
-  if (!layer_layout(E, H, F, w->fmt, nullptr, nullptr, &total)) return MOE_ERR_FORMAT;
+  uint64_t co[3 * kMaxE], so[3 * kMaxE], side[3 * kMaxE], total = 0, out_sec = 0;
+  if (!full_layout(E, H, F, w->fmt, co, so, side, &out_sec, &total)) return MOE_ERR_FORMAT;
   if (w->packed_bytes < total) return MOE_ERR_WORKSPACE;
   if (ws_bytes < need) return MOE_ERR_WORKSPACE;
   const moe_status ds = check_device();
@@ -228,11 +258,11 @@ extern "C" moe_status moe_layer_forward(const void* x, int32_t T, const float* r
     const GemmHooks hooks{d.test_withhold, d.wait_cycles};
     if (act4 && plan.tc)
       return launch_expert_gemm_fp4(packed, E, H, F, T, k, gateup, wsp, status, d.trace, hooks, stream);
-    return plan.tc ? launch_expert_gemm_tc(packed, w->fmt, E, H, F, T, k, fp4, gateup, wsp, status, d.trace, hooks,
-                                           stream)
-                   : launch_expert_gemv(packed, w->packed_bytes, w->fmt, E, H, F, T * k, k, fp4, gateup,
+    return plan.tc ? launch_expert_gemm_tc(packed, fmt, E, H, F, T, k, fp4, gateup, wsp, status, d.trace, hooks,
+                                           outliers, stream)
+                   : launch_expert_gemv(packed, w->packed_bytes, fmt, E, H, F, T * k, k, fp4, gateup,
                                         plan.max_chunks, plan.chunk_rows, wsp, status, gateup ? d.trace : nullptr,
-                                        hooks, stream);
+                                        hooks, outliers, stream);
   };
   if (gemm(true) != cudaSuccess) return MOE_ERR_CUDA;
   if (!mark(4)) return MOE_ERR_CUDA;

@@ -35,6 +35,7 @@
 // status word.  Copies and MMAs still in flight are waited for, and the pair
 // meets at a cluster barrier, before TMEM is freed and the CTAs return.
 #include <algorithm>
+#include <type_traits>
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
@@ -128,6 +129,7 @@ struct TcArgs {
   const int32_t* chunk_count;
   const float* row_scale;  // NVFP4: gate/up -> per-token sx, down -> per-row sh; null for integer layers
   const float* xinv;       // integer gate/up: per-row 2^e undoing the activations' prescale (null otherwise)
+  const __half* act16;     // the fp16 activations [rows][K] (the residual term of outlier side lists)
   const int32_t* perm;
   int topk;
   void* out;               // gate/up: h [rows][F] (fp16, or fp32 for NVFP4); down: o fp32 [rows][H]
@@ -394,7 +396,8 @@ __device__ __forceinline__ bool dequant_item_any(int f0, int f1, const Ring R, l
   }
 }
 
-template <int NMAT, bool CG2, bool I1>
+// OUT: the layer has outlier side lists (their residuals are added in the epilogue)
+template <int NMAT, bool CG2, bool I1, bool OUT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
   using C = TcCfg<NMAT, CG2>;
@@ -458,6 +461,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int stride = CG2 ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int ksteps = a.K / kTcBK;
   const LayerHdr L = hdr_view(a.packed, a.E, a.H, a.F);
+  const LayerHdr LS = OUT ? hdr_view_side(a.packed, a.E, a.H, a.F) : L;  // with the side-list table
   bool ok = true;
 
   // Every role runs its loop with whole warps: waits are taken by all lanes and
@@ -725,7 +729,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const float f = __shfl_sync(0xffffffffu, fu, (tok - cq * kColsPerWarp) & 31);
             if (tok >= rows) continue;
             const size_t o = (size_t)(row0 + tok) * a.N + nrow;
-            if (NMAT == 2 && a.pair) {  // two weight tiles of the down matrix: rows nrow and nrow + 128
+            if (OUT) {  // residuals of the side lists, in the units of the fp16 activations
+              const __half* av = a.act16 + (size_t)(row0 + tok) * a.K;
+              const int i0 = e * 3 + a.proj;
+              float d0, d1 = 0.0f;
+              if (NMAT == 2 && a.pair) {
+                d0 = outlier_dot(LS, i0, a.N, nrow, av);
+                d1 = outlier_dot(LS, i0, a.N, nrow + kTcBM, av);
+                out[o] = (__uint_as_float(r0[j]) * tsc[0] + d0) * f;
+                out[o + kTcBM] = (__uint_as_float(r1[j]) * tsc[0] + d1) * f;
+              } else if (NMAT == 2) {
+                d0 = outlier_dot(LS, i0, a.N, nrow, av);
+                d1 = outlier_dot(LS, i0 + 1, a.N, nrow, av);
+                const float g = (__uint_as_float(r0[j]) * tsc[0] + d0) * f, u = (__uint_as_float(r1[j]) * tsc[1] + d1) * f;
+                out[o] = __fdividef(g, 1.0f + __expf(-g)) * u;
+              } else {
+                out[o] = (__uint_as_float(r0[j]) * tsc[0] + outlier_dot(LS, i0, a.N, nrow, av)) * f;
+              }
+            } else if (NMAT == 2 && a.pair) {  // two weight tiles of the down matrix: rows nrow and nrow + 128
               const float sc = f * tsc[0];
               out[o] = __uint_as_float(r0[j]) * sc;
               out[o + kTcBM] = __uint_as_float(r1[j]) * sc;
@@ -749,17 +770,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int tok = cb + j;
             if (tok >= rows) break;
             const int r = row0 + tok;
+            float d0 = 0.0f, d1 = 0.0f;  // residuals of the side lists, in the units of the fp16 activations
+            if (OUT) {
+              const __half* av = a.act16 + (size_t)r * a.K;
+              const int i0 = e * 3 + a.proj;
+              d0 = outlier_dot(LS, i0, a.N, nrow, av);
+              if (NMAT == 2) d1 = a.pair ? outlier_dot(LS, i0, a.N, nrow + kTcBM, av) : outlier_dot(LS, i0 + 1, a.N, nrow, av);
+            }
             if (NMAT == 2 && a.pair) {  // two weight tiles of the down matrix: rows nrow and nrow + 128
-              reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = __uint_as_float(r0[j]);
-              reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow + kTcBM] = __uint_as_float(r1[j]);
+              reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = __uint_as_float(r0[j]) + d0;
+              reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow + kTcBM] = __uint_as_float(r1[j]) + d1;
             } else if (NMAT == 2) {
               const float xi = a.xinv[r];  // 2^e: exact, 1 unless the token was prescaled
-              const float g = __uint_as_float(r0[j]) * xi, u = __uint_as_float(r1[j]) * xi;
+              const float g = (__uint_as_float(r0[j]) + d0) * xi, u = (__uint_as_float(r1[j]) + d1) * xi;
               const __half h = __float2half_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
               range |= __hisinf(h) != 0;
               reinterpret_cast<__half*>(a.out)[(size_t)r * a.N + nrow] = h;
             } else {
-              reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = __uint_as_float(r0[j]);
+              reinterpret_cast<float*>(a.out)[(size_t)r * a.N + nrow] = __uint_as_float(r0[j]) + d0;
             }
           }
         }
@@ -820,9 +848,10 @@ int sm_count() {
   return n[dev];
 }
 
-template <int NMAT, bool CG2, bool I1>
+template <int NMAT, bool CG2, bool I1, bool OUT>
 cudaError_t launch_tc(TcArgs a, int max_words, const void* act, int rows_total, cudaStream_t stream) {
   using C = TcCfg<NMAT, CG2>;
+  a.act16 = static_cast<const __half*>(act);
   a.ring = make_ring<NMAT, CG2>(max_words);
   if (a.ring.raw_slots < 2) return cudaErrorInvalidConfiguration;
   const int smem = ring_smem(a.ring);
@@ -838,7 +867,7 @@ cudaError_t launch_tc(TcArgs a, int max_words, const void* act, int rows_total, 
           CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  auto kern = expert_gemm_tc_kernel<NMAT, CG2, I1>;
+  auto kern = expert_gemm_tc_kernel<NMAT, CG2, I1, OUT>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   if (!CG2) {
@@ -871,7 +900,7 @@ cudaError_t launch_tc(TcArgs a, int max_words, const void* act, int rows_total, 
 
 cudaError_t launch_expert_gemm_tc(const uint8_t* packed, const uint8_t* fmt_host, int E, int H, int F, int T, int k,
                                   bool fp4, bool gateup, const Workspace& ws, int32_t* status, uint64_t* trace,
-                                  GemmHooks hooks, cudaStream_t stream) {
+                                  GemmHooks hooks, bool outliers, cudaStream_t stream) {
   // widest code format of the projections this launch reads (sizes the code slots),
   // and whether any of them is the 1-bit code (selects the kernels that decode it)
   int max_words = 1;
@@ -895,6 +924,20 @@ cudaError_t launch_expert_gemm_tc(const uint8_t* packed, const uint8_t* fmt_host
   a.topk = k;
   a.status = status;
   const int R = T * k;
+  // kernel variant: tile shape, 1-bit decoding, side lists
+  auto go = [&](auto nmat, auto cg2, const void* act) -> cudaError_t {
+    constexpr int NM = decltype(nmat)::value;
+    constexpr bool P = decltype(cg2)::value;
+    if (outliers)
+      return any1 ? launch_tc<NM, P, true, true>(a, max_words, act, R, stream)
+                  : launch_tc<NM, P, false, true>(a, max_words, act, R, stream);
+    return any1 ? launch_tc<NM, P, true, false>(a, max_words, act, R, stream)
+                : launch_tc<NM, P, false, false>(a, max_words, act, R, stream);
+  };
+  using Two = std::integral_constant<int, 2>;
+  using One = std::integral_constant<int, 1>;
+  using Pair = std::true_type;
+  using Single = std::false_type;
   if (gateup) {
     a.N = F;
     a.K = H;
@@ -902,27 +945,21 @@ cudaError_t launch_expert_gemm_tc(const uint8_t* packed, const uint8_t* fmt_host
     a.row_scale = fp4 ? ws.sx : nullptr;
     a.xinv = fp4 ? nullptr : ws.xinv;
     a.out = ws.h;
-    if ((F / kTcBM) % 2 == 0)  // weight tiles in pairs of CTAs
-      return any1 ? launch_tc<2, true, true>(a, max_words, ws.xs, R, stream)
-                  : launch_tc<2, true, false>(a, max_words, ws.xs, R, stream);
-    return any1 ? launch_tc<2, false, true>(a, max_words, ws.xs, R, stream)
-                : launch_tc<2, false, false>(a, max_words, ws.xs, R, stream);
+    if ((F / kTcBM) % 2 == 0) return go(Two{}, Pair{}, ws.xs);  // weight tiles in pairs of CTAs
+    return go(Two{}, Single{}, ws.xs);
   }
   a.N = H;
   a.K = F;
   a.proj = 2;
   a.row_scale = fp4 ? ws.sh : nullptr;
   a.out = ws.o;
+  const void* act = fp4 ? ws.hb : ws.h;
   if ((H / kTcBM) % 2 == 0) {  // pairs of weight tiles share each activation tile
     a.pair = 1;
-    if ((H / kTcBM) % 4 == 0)
-      return any1 ? launch_tc<2, true, true>(a, max_words, fp4 ? ws.hb : ws.h, R, stream)
-                  : launch_tc<2, true, false>(a, max_words, fp4 ? ws.hb : ws.h, R, stream);
-    return any1 ? launch_tc<2, false, true>(a, max_words, fp4 ? ws.hb : ws.h, R, stream)
-                : launch_tc<2, false, false>(a, max_words, fp4 ? ws.hb : ws.h, R, stream);
+    if ((H / kTcBM) % 4 == 0) return go(Two{}, Pair{}, act);
+    return go(Two{}, Single{}, act);
   }
-  return any1 ? launch_tc<1, false, true>(a, max_words, fp4 ? ws.hb : ws.h, R, stream)
-              : launch_tc<1, false, false>(a, max_words, fp4 ? ws.hb : ws.h, R, stream);
+  return go(One{}, Single{}, act);
 }
 
 }  // namespace moe

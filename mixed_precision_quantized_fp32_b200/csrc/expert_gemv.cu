@@ -81,6 +81,8 @@ struct GemvArgs {
   const int32_t* chunk_count;
   const float* row_scale; // NVFP4: gate/up -> per-token sx, down -> per-row sh; null for integer layers
   const float* xinv;      // integer gate/up: per-row 2^e undoing the activations' prescale (null otherwise)
+  const __half* act16;    // the fp16 activations [R][K] (the residual term of outlier side lists)
+  int outliers;           // the layer has outlier side lists
   const int32_t* perm;
   bool sums;              // integer layer: activation group sums are loaded with the tiles
   void* out;              // gate/up: h [R][F] (fp16, or fp32 for NVFP4); down: o fp32 [R][H]
@@ -372,7 +374,7 @@ __device__ __forceinline__ Item item_of(int it, int P, int nchunks) {
 struct ItemDesc {
   int it, chunk, nb, p, row0, rows, ntiles, f0, f1;
   float ts0, ts1;
-  int pad;
+  int e;  // expert
 };
 static_assert(sizeof(ItemDesc) == 48, "descriptor size");
 
@@ -395,6 +397,7 @@ __device__ __forceinline__ void load_item(ItemSrc<NMAT>& s, int it, int total, i
   const Item w = item_of(it, a.P, nchunks);
   const int e = a.chunks[3 * w.chunk];
   s.d.chunk = w.chunk;
+  s.d.e = e;
   s.d.nb = w.nb;
   s.d.p = w.p;
   s.d.row0 = a.chunks[3 * w.chunk + 1];
@@ -424,19 +427,36 @@ __device__ __forceinline__ void load_item(ItemSrc<NMAT>& s, int it, int total, i
 // (integer formats: already multiplied by 2^24).  Gate/up returns h as stored
 // (fp16-rounded for integer layers), for the group sums of the down GEMV, and
 // sets `range` when that fp16 h overflowed.
+// Outlier side lists add sum r * a over the row's outliers to the raw sums (in the
+// units of the fp16 activations, before the row and tensor scales).
 template <int NMAT>
 __device__ __forceinline__ float store_output(const GemvArgs& a, int r, int n, const float* v, const float* ts,
-                                              bool& range) {
+                                              bool& range, int e) {
+  float dot[NMAT];
+#pragma unroll
+  for (int m = 0; m < NMAT; ++m) dot[m] = 0.0f;
+  if (a.outliers) {
+    const LayerHdr L = hdr_view_side(a.packed, a.E, a.H, a.F);
+#pragma unroll
+    for (int m = 0; m < NMAT; ++m) dot[m] = outlier_dot(L, e * 3 + a.proj + m, a.N, n, a.act16 + (size_t)r * a.K);
+  }
   if (NMAT == 2) {
     float gv = v[0], uv = v[1];
     if (a.row_scale) {
       const float sx = a.row_scale[a.perm[r] / a.topk];
-      gv *= sx * ts[0];
-      uv *= sx * ts[1];
+      if (a.outliers) {
+        gv = (gv * ts[0] + dot[0]) * sx;
+        uv = (uv * ts[1] + dot[NMAT - 1]) * sx;
+      } else {
+        gv *= sx * ts[0];
+        uv *= sx * ts[1];
+      }
       const float h = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
       reinterpret_cast<float*>(a.out)[(size_t)r * a.N + n] = h;
       return h;
     }
+    gv += dot[0];
+    uv += dot[NMAT - 1];
     if (a.xinv) {
       const float xi = a.xinv[r];
       gv *= xi;
@@ -448,7 +468,8 @@ __device__ __forceinline__ float store_output(const GemvArgs& a, int r, int n, c
     return __half2float(h);
   }
   float o = v[0];
-  if (a.row_scale) o *= a.row_scale[r] * ts[0];
+  if (a.row_scale) o = a.outliers ? (o * ts[0] + dot[0]) * a.row_scale[r] : o * (a.row_scale[r] * ts[0]);
+  else o += dot[0];
   reinterpret_cast<float*>(a.out)[(size_t)r * a.N + n] = o;
   return o;
 }
@@ -630,7 +651,7 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m) v[m] = acc[m][t][nt][j] * fscale[m];
                 hs[j & 1] += store_output<NMAT>(a, row0 + tk, w.nb * kBlockRows + 32 * s + 4 * g + 2 * t + (j >> 1),
-                                                v, ts, range);
+                                                v, ts, range, w.e);
               }
             }
           if (a.out_sum) {  // warp s owns the 32 weight rows of one down-projection input group
@@ -702,7 +723,7 @@ __global__ void __launch_bounds__(256) gemv_fixup_kernel(GemvArgs a, const int32
       v[m] = sum;
     }
     bool range = false;
-    float h = store_output<NMAT>(a, r, n, v, ts, range);
+    float h = store_output<NMAT>(a, r, n, v, ts, range, e);
     if (range) report_range(a.status);
     if (a.out_sum) {
 #pragma unroll
@@ -847,8 +868,9 @@ int gemv_split(long long R, int E, int N, int K, int nmat) {
 cudaError_t launch_expert_gemv(const uint8_t* packed, uint64_t packed_bytes, const uint8_t* fmt_host, int E, int H,
                                int F, int R, int k, bool fp4, bool gateup, int max_chunks, int chunk_rows,
                                const Workspace& ws, int32_t* status, uint64_t* trace, GemmHooks hooks,
-                               cudaStream_t stream) {
+                               bool outliers, cudaStream_t stream) {
   GemvArgs g{};
+  g.outliers = outliers ? 1 : 0;
   g.trace = reinterpret_cast<unsigned long long*>(trace);
   g.wait = hooks.wait_cycles ? (long long)hooks.wait_cycles : kGemvWait;
   g.withhold = hooks.withhold ? 1 : 0;
@@ -894,6 +916,7 @@ cudaError_t launch_expert_gemv(const uint8_t* packed, uint64_t packed_bytes, con
   }
   const int nmat = gateup ? 2 : 1;
   g.P = gemv_split(R, E, g.N, g.K, nmat);
+  g.act16 = (const __half*)act;
   if (chunk_rows != 8) return cudaErrorInvalidValue;  // the host plans 8-row chunks (one token tile)
   bool any1 = false;  // a 1-bit matrix among this projection's
   for (int e = 0; e < E; ++e)

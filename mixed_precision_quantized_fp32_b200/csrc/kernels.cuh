@@ -4,9 +4,11 @@
 
 namespace moe {
 
+// fmt_host: the caller's codes (MOE_FMT_OUTLIERS kept); out_sec / side_off: the outlier
+// section and side-list offsets (0 when absent).
 cudaError_t launch_pack(const float* W, int e0, int ne, int E, int H, int F, const uint8_t* fmt_host,
-                        uint8_t* out, const uint64_t* code_off, const uint64_t* scale_off,
-                        cudaStream_t stream);
+                        uint8_t* out, const uint64_t* code_off, const uint64_t* scale_off, uint64_t out_sec,
+                        const uint64_t* side_off, cudaStream_t stream);
 
 // Router K parts (0: warp kernel, no parts); the workspace holds max(1, parts) logit planes.
 int router_parts(long long T, int H, int E);
@@ -37,7 +39,7 @@ constexpr int kFp4ChunkRows = 128;
 
 cudaError_t launch_expert_gemm_tc(const uint8_t* packed, const uint8_t* fmt_host, int E, int H, int F, int T, int k,
                                   bool fp4, bool gateup, const Workspace& ws, int32_t* status, uint64_t* trace,
-                                  GemmHooks hooks, cudaStream_t stream);
+                                  GemmHooks hooks, bool outliers, cudaStream_t stream);
 
 // K parts of the decode GEMV for R expert rows on an N x K projection (nmat
 // matrices); the workspace holds P*R*N*nmat fp32 partials when P > 1.
@@ -46,7 +48,7 @@ int gemv_split(long long R, int E, int N, int K, int nmat);
 cudaError_t launch_expert_gemv(const uint8_t* packed, uint64_t packed_bytes, const uint8_t* fmt_host, int E, int H,
                                int F, int R, int k, bool fp4, bool gateup, int max_chunks, int chunk_rows,
                                const Workspace& ws, int32_t* status, uint64_t* trace, GemmHooks hooks,
-                               cudaStream_t stream);
+                               bool outliers, cudaStream_t stream);
 
 // NVFP4 activations: per-token codes of x and their gather into sorted rows
 // (prefill: codes + block scales; decode: fp16 block values), and per-row codes of h.

@@ -19,10 +19,26 @@ constexpr uint32_t kOffScale = 6944u;
 constexpr uint32_t kOffTscale = 13088u;
 constexpr int kMaxE = 256;
 constexpr int kMaxK = 8;
+// Outlier side lists (MoE mixed-precision page sec. 4.2, tip 2: each expert matrix keeps
+// its top 0.05% of weights by |w| in fp16 beside the quantized rest).  A matrix opts in
+// with MOE_FMT_OUTLIERS on its format code; the header then holds the base format, a flag
+// and the offset of the outlier section appended after the expert sections:
+//   [u64 side_off[768]] [u32 selection scratch, kOutScratchWords] [one side list per
+//   opted-in matrix, 256-byte aligned: u32 row_ptr[N+1], u32 entry[n_out] with the column
+//   in bits 0-15 and the fp16 residual in bits 16-31, sorted by (row, column)].
+constexpr uint32_t kOffFlags = 20u;    // u32: bit 0 = the layer has an outlier section
+constexpr uint32_t kOffOutSec = 24u;   // u64: offset of the outlier section
+constexpr int kOutScratchWords = 64 + 65536;
+constexpr uint64_t kOutTableBytes = 8u * 3u * kMaxE;
 
 __host__ __device__ inline bool fmt_known(int f) {
   return f == MOE_FMT_INT1 || f == MOE_FMT_INT2 || f == MOE_FMT_INT3 || f == MOE_FMT_INT4 || f == MOE_FMT_NVFP4;
 }
+// Host format codes may carry MOE_FMT_OUTLIERS; the base format decides codes and scales.
+__host__ __device__ inline int fmt_base(int f) { return f & ~MOE_FMT_OUTLIERS; }
+__host__ __device__ inline bool fmt_outliers(int f) { return (f & MOE_FMT_OUTLIERS) != 0; }
+// Outliers of an N x K matrix: floor(N*K*5/10000), integer arithmetic.
+__host__ __device__ inline uint64_t outlier_count(uint64_t N, uint64_t K) { return N * K * 5u / 10000u; }
 // u32 words per group of 32 inputs
 __host__ __device__ inline int fmt_words(int f) { return f == MOE_FMT_NVFP4 ? 4 : f; }
 
@@ -61,6 +77,32 @@ __host__ __device__ inline bool layer_layout(int E, int H, int F, const uint8_t*
   return true;
 }
 
+// The outlier section after the expert sections (which end at `end`): its offset
+// (0 when no matrix opts in), each opted-in matrix's side-list offset in side[]
+// (0 for the others) and the new total size.  fmt: host codes (flags kept).
+__host__ __device__ inline uint64_t outlier_layout(int E, int H, int F, const uint8_t* fmt, uint64_t end,
+                                                   uint64_t* side, uint64_t* total) {
+  bool any = false;
+  for (int i = 0; i < 3 * E; ++i) any |= fmt_outliers(fmt[i]);
+  for (int i = 0; i < 3 * E; ++i) side[i] = 0;
+  if (!any) {
+    *total = end;
+    return 0;
+  }
+  const uint64_t sec = up256(end);
+  uint64_t pos = up256(sec + kOutTableBytes + 4u * (uint64_t)kOutScratchWords);
+  for (int e = 0; e < E; ++e)
+    for (int p = 0; p < 3; ++p) {
+      if (!fmt_outliers(fmt[e * 3 + p])) continue;
+      int N, K;
+      proj_shape(p, H, F, N, K);
+      side[e * 3 + p] = pos;
+      pos = up256(pos + 4u * ((uint64_t)N + 1u + outlier_count(N, K)));
+    }
+  *total = pos;
+  return sec;
+}
+
 // Word index (u32 units) of word w of the group holding input k of output n.
 __host__ __device__ inline uint64_t word_index(int n, int k, int K, int wpg, int w) {
   const uint64_t nb = (uint64_t)(n >> 7), kb = (uint64_t)(k >> 7);
@@ -81,6 +123,7 @@ struct LayerHdr {
   const uint64_t* scale_off;
   const float* tscale;
   const uint8_t* base;
+  const uint64_t* side;  // side-list offsets [768] (null: no outlier section)
 };
 
 __host__ __device__ inline LayerHdr hdr_view(const void* packed, int E, int H, int F) {
@@ -93,7 +136,31 @@ __host__ __device__ inline LayerHdr hdr_view(const void* packed, int E, int H, i
   h.code_off = (const uint64_t*)(h.base + kOffCode);
   h.scale_off = (const uint64_t*)(h.base + kOffScale);
   h.tscale = (const float*)(h.base + kOffTscale);
+  h.side = nullptr;
   return h;
+}
+// The same with the outlier table (reads the header's flag word on the device).
+__device__ inline LayerHdr hdr_view_side(const void* packed, int E, int H, int F) {
+  LayerHdr h = hdr_view(packed, E, H, F);
+  if (*(const uint32_t*)(h.base + kOffFlags) & 1u)
+    h.side = (const uint64_t*)(h.base + *(const uint64_t*)(h.base + kOffOutSec));
+  return h;
+}
+
+// Residual term of weight row n of matrix slot i (e*3+p) against activation row a
+// (fp16, length K): sum over the row's outliers of r * a[col].  0 without a side list.
+__device__ __forceinline__ float outlier_dot(const LayerHdr& L, int i, int N, int n, const __half* __restrict__ a) {
+  if (!L.side) return 0.0f;
+  const uint64_t off = L.side[i];
+  if (!off) return 0.0f;
+  const uint32_t* rp = (const uint32_t*)(L.base + off);
+  const uint32_t* ent = rp + N + 1;
+  float s = 0.0f;
+  for (uint32_t j = __ldg(rp + n), j1 = __ldg(rp + n + 1); j < j1; ++j) {
+    const uint32_t v = __ldg(ent + j);
+    s = fmaf(__half2float(__ushort_as_half((uint16_t)(v >> 16))), __half2float(a[v & 0xFFFFu]), s);
+  }
+  return s;
 }
 
 // e2m1 code (sign<<3 | exp<<1 | man) -> float

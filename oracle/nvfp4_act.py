@@ -6,7 +6,7 @@ form a block-scaled FP4 tensor-core product consumes on both operands
 per-token dynamic activation scales).
 
 TEST INFRASTRUCTURE, like the rest of ``oracle/``: numpy composition of the
-oracle's pinned functions.  The product library does not implement this mode.
+oracle's pinned functions.
 
 Readings:
   * a row of activations takes the weights' NVFP4 rule with the row as the

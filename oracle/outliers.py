@@ -5,8 +5,7 @@ expert's top 0.05% of weights by |w| out, store them in FP16, quantize the
 other 99.95%).
 
 TEST INFRASTRUCTURE, like the rest of ``oracle/``; plain numpy on top of the
-oracle's own quantize / pack / decode functions.  The product library does not
-implement this mode.
+oracle's own quantize / pack / decode functions.
 
 Readings (the page gives the fraction and the idea only):
   * per matrix (one expert, one projection) n_out = floor(frac * N * K),

@@ -162,6 +162,42 @@ def oracle_forward_rows_act4(layer_buf, x_bits, Wr, b, k, tokens=None, idx_overr
     return y, idx, w
 
 
+def oracle_forward_rows_dense(mats, x_bits, Wr, b, k, fp4=False, idx_override=None):
+    """The oracle's stages (router, top-k, FP8 activation quantization of NVFP4
+    layers) with the expert products taken on given float64 matrices: mats(e) ->
+    (W_gate [F,H], W_up [F,H], W_down [H,F]).  Used for layers whose matrices are
+    more than their packed dense part (outlier side lists): g = s_x * W_gate a,
+    u = s_x * W_up a, h = silu(g) * u, o = s_h * W_down h, y = sum_j w_j o_j."""
+    T = x_bits.shape[0]
+    logits = orc.router(x_bits, Wr, b)
+    idx, w = orc.topk_softmax(logits, k)
+    if idx_override is not None:
+        idx = np.ascontiguousarray(idx_override, np.int32)
+        sel = np.take_along_axis(logits, idx, 1).astype(np.float64)
+        ex = np.exp(sel - sel.max(1, keepdims=True))
+        w = (ex / ex.sum(1, keepdims=True)).astype(np.float32)
+    xf = gen.bf16_bits_to_f32(x_bits)
+    if fp4:
+        xq, sx = orc.act_quant_e4m3(xf)
+        a, a_scale = orc.e4m3_table()[xq], sx.astype(np.float64)
+    else:
+        a, a_scale = xf.astype(np.float64), np.ones(T)
+    y = np.zeros((T, x_bits.shape[1]))
+    for e in np.unique(idx):
+        ts, js = np.nonzero(idx == e)
+        Wg, Wu, Wd = mats(int(e))
+        g = (a[ts] @ Wg.T) * a_scale[ts, None]
+        u = (a[ts] @ Wu.T) * a_scale[ts, None]
+        h = g / (1.0 + np.exp(-g)) * u
+        h_scale = np.ones(len(ts))
+        if fp4:
+            hq, sh = orc.act_quant_e4m3(h.astype(np.float32))
+            h, h_scale = orc.e4m3_table()[hq], sh.astype(np.float64)
+        o = (h @ Wd.T) * h_scale[:, None]
+        y[ts] += w[ts, js].astype(np.float64)[:, None] * o
+    return y
+
+
 def check_output(y_gpu_bf16, y_ref):
     """|y_gpu - y_ref| <= TOL * max|y_ref|; returns the error ratio."""
     import torch

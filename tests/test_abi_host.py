@@ -170,3 +170,41 @@ def test_ctypes_structs_match_the_header(tmp_path):
         assert got[(cname, "size")] == C.sizeof(py), cname
         for fname, _ in py._fields_:
             assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
+
+
+def test_outlier_flag_layout_and_errors():
+    # MOE_FMT_OUTLIERS adds a section after the expert sections: 256-aligned start,
+    # a 3*256-entry u64 table and 4*(64+65536) bytes of scratch, then one side list
+    # (u32 row_ptr[N+1] + u32 entry[floor(N*K*5/10000)]) per flagged matrix, 256-aligned
+    E, H, F = 4, 256, 384
+    up = lambda v: (v + 255) // 256 * 256  # noqa: E731
+    base = np.array([[4, 3, 2], [1, 2, 4], [3, 4, 1], [2, 1, 3]], np.uint8)
+    flagged = base.copy()
+    flagged[0, :] |= moe.FMT_OUTLIERS
+    flagged[2, 2] |= moe.FMT_OUTLIERS
+    t_base, co, so = moe.pack_layout(E, H, F, base)
+    t_out, co2, so2 = moe.pack_layout(E, H, F, flagged)
+    np.testing.assert_array_equal(co, co2)  # expert sections do not move
+    np.testing.assert_array_equal(so, so2)
+    pos = up(up(t_base) + 8 * 768 + 4 * (64 + 65536))
+    for N, K in [(F, H), (F, H), (H, F), (H, F)]:  # gate, up, down of expert 0; down of expert 2
+        pos = up(pos + 4 * (N + 1 + N * K * 5 // 10000))
+    assert t_out == pos
+    for bad_flag in (0x40, 0x20):
+        bad = base.copy()
+        bad[1, 1] |= bad_flag
+        assert _pack(None, 0, 0, E, H, F, bad, None, 0)[0] == "MOE_ERR_FORMAT"
+    # a buffer sized for the unflagged layout is too small for the flagged one
+    assert _fwd(16, 2, E=E, H=H, F=F, fmt=flagged, packed_bytes=t_base)[0] == "MOE_ERR_WORKSPACE"
+    st, need = _fwd(16, 2, E=E, H=H, F=F, fmt=flagged, query=True)
+    assert st == "MOE_OK" and need > 0
+    # side lists are read with FP8 activations only: NVFP4 activations are rejected
+    fp4 = np.full((E, 3), 16, np.uint8)
+    fp4[1, 0] |= moe.FMT_OUTLIERS
+    f = np.ascontiguousarray(fp4).ravel()
+    for act, want in ((moe.ACT_FP8, "MOE_OK"), (moe.ACT_NVFP4, "MOE_ERR_FORMAT")):
+        w = _lib.MoeWeights(E, H, F, f.ctypes.data, FAKE, moe.pack_layout(E, H, F, f)[0], act)
+        need = C.c_uint64(0)
+        rc = _lib.load().moe_layer_forward(FAKE, 16, FAKE, None, C.byref(w), 2, FAKE, None, 0, C.byref(need),
+                                           None, None)
+        assert _lib.STATUS[rc] == want

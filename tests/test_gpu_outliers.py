@@ -1,0 +1,262 @@
+"""GPU parity of outlier isolation ("MoE混合精度量化实战", sec. 4.2, tip 2: the
+top 0.05% of each expert matrix's weights by |w| kept in fp16 beside the
+quantized rest), against the oracle's restatement in oracle/outliers.py.
+
+Bars:
+  * moe_pack of a layer whose format codes carry MOE_FMT_OUTLIERS: the expert
+    sections equal the oracle's packing of the weights with their outliers
+    zeroed, byte for byte; the header's flag word and section offset, the
+    side-list table and every side list (row offsets, then column | fp16
+    residual << 16 in (row, column) order) equal the oracle's selection and
+    residuals bit for bit (ties in |w| at the threshold, signed ties, the 1-bit
+    sign code's w - s residual, NVFP4 tensor scales taken without the outliers);
+  * forward: max |y_gpu - y_ref| <= 2e-2 * max |y_ref|, y_ref the oracle's stages
+    on the matrices dequant(codes) + residuals, with planted large outliers so
+    that a dropped or misplaced residual fails by far;
+  * NVFP4 activations with side lists are rejected (MOE_ERR_FORMAT).
+"""
+import numpy as np
+import pytest
+
+import gen
+import gen.workloads as W
+import oracle as orc
+from oracle import outliers as ol
+from tests import helpers as hp
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import mixed_precision_quantized_fp32_b200 as moe  # noqa: E402
+
+OUT = moe.FMT_OUTLIERS
+MAX_E = 256
+SCRATCH_WORDS = 64 + 65536
+
+
+def up256(x):
+    return (x + 255) // 256 * 256
+
+
+def shape(p, H, F):
+    return (F, H) if p < 2 else (H, F)
+
+
+def expected_side_layout(E, H, F, fmt, end):
+    """Section offset and per-matrix side-list offsets of the packed-layer format
+    (moe.h, "Outlier section"): the section starts at the first 256-byte boundary
+    after the expert sections; a table of 3*256 u64 offsets and the selection
+    scratch come first, then each opted-in matrix's list on a 256-byte boundary."""
+    if not np.any(fmt & OUT):
+        return 0, np.zeros(3 * E, np.uint64)
+    sec = up256(end)
+    pos = up256(sec + 8 * 3 * MAX_E + 4 * SCRATCH_WORDS)
+    side = np.zeros(3 * E, np.uint64)
+    for i in range(3 * E):
+        if fmt[i] & OUT:
+            N, K = shape(i % 3, H, F)
+            side[i] = pos
+            pos = up256(pos + 4 * (N + 1 + ol.count(N, K)))
+    return sec, side
+
+
+def oracle_outlier_layer(Wh, E, H, F, fmt):
+    """The oracle's view of the layer: the packed dense part (weights of the
+    opted-in matrices with their outliers zeroed), the isolation of each opted-in
+    matrix, and its end offset."""
+    base = (fmt & 0x7F).astype(np.uint8)
+    Wz = Wh.copy()
+    isos = {}
+    for e in range(E):
+        for p in range(3):
+            if fmt[e * 3 + p] & OUT:
+                N, K = shape(p, H, F)
+                iso = ol.isolate(Wh[e, p].reshape(N, K), int(base[e * 3 + p]))
+                isos[(e, p)] = iso
+                Wz[e, p].reshape(N, K)[iso["rows"], iso["cols"]] = 0.0
+    buf = orc.pack_layer(Wz, 0, E, H, F, base)
+    return buf, isos, orc.layer_layout(E, H, F, base)[2]
+
+
+def gpu_pack_host(Wh, E, H, F, fmt, per=None):
+    total = moe.pack_layout(E, H, F, fmt)[0]
+    packed = moe.alloc_packed(total)
+    packed.fill_(0xA5)  # every byte the layout defines must be written (scratch aside)
+    per = per or E
+    for e0 in range(0, E, per):
+        moe.moe_pack(torch.from_numpy(np.ascontiguousarray(Wh[e0:e0 + per])).cuda(), e0, E, H, F, fmt, packed)
+    torch.cuda.synchronize()
+    return moe.PackedLayer(E, H, F, fmt, packed), total
+
+
+def check_pack(Wh, E, H, F, fmt, per=None):
+    layer, total = gpu_pack_host(Wh, E, H, F, fmt, per)
+    got = layer.packed.cpu().numpy()
+    want, isos, end = oracle_outlier_layer(Wh, E, H, F, fmt)
+    sec, side = expected_side_layout(E, H, F, fmt, end)
+    # header: magic .. F, then the flag word and the section offset
+    np.testing.assert_array_equal(got[:20], want[:20])
+    assert got[20:24].view(np.uint32)[0] == (1 if sec else 0)
+    assert got[24:32].view(np.uint64)[0] == sec
+    np.testing.assert_array_equal(got[32:end], want[32:end])
+    if not sec:
+        assert total == end
+        return layer, isos
+    table = got[sec:sec + 8 * 3 * MAX_E].view(np.uint64)
+    np.testing.assert_array_equal(table[:3 * E], side)
+    assert not table[3 * E:].any()
+    for (e, p), iso in isos.items():
+        N, K = shape(p, H, F)
+        n_out = ol.count(N, K)
+        o = int(side[e * 3 + p])
+        words = got[o:o + 4 * (N + 1 + n_out)].view(np.uint32)
+        row_ptr = np.concatenate([[0], np.cumsum(np.bincount(iso["rows"], minlength=N))]).astype(np.uint32)
+        np.testing.assert_array_equal(words[:N + 1], row_ptr, err_msg=f"row offsets e{e} p{p}")
+        entries = iso["cols"].astype(np.uint32) | (iso["resid"].astype(np.uint32) << 16)
+        np.testing.assert_array_equal(words[N + 1:], entries, err_msg=f"entries e{e} p{p}")
+    last = max(int(side[i]) + 4 * (shape(i % 3, H, F)[0] + 1 + ol.count(*shape(i % 3, H, F)))
+               for i in range(3 * E) if fmt[i] & OUT)
+    assert total == up256(last)
+    return layer, isos
+
+
+def host_weights(E, H, F, seed_base=0):
+    return np.stack([W.expert_w(seed_base + e, H, F) for e in range(E)])
+
+
+def plant_outliers(Wh, H, F, seed):
+    """Heavy-tailed weights: per matrix count(N, K) positions set to +-(0.3 .. 1.0),
+    15x the Gaussian's 0.02 sigma and more, like the outlier weights of trained
+    LLM layers."""
+    rng = np.random.default_rng(seed)
+    for e in range(Wh.shape[0]):
+        for p in range(3):
+            N, K = shape(p, H, F)
+            n = ol.count(N, K)
+            pos = rng.choice(N * K, size=n, replace=False)
+            Wh[e, p, pos] = (rng.uniform(0.3, 1.0, n) * rng.choice([-1.0, 1.0], n)).astype(np.float32)
+    return Wh
+
+
+INT_FMT = np.array([[4 | OUT, 3 | OUT, 2 | OUT],
+                    [1 | OUT, 2, 4 | OUT],
+                    [3, 4 | OUT, 1 | OUT],
+                    [2 | OUT, 1 | OUT, 3]], np.uint8).reshape(-1)
+
+
+def test_pack_outliers_mixed_formats_bit_exact():
+    E, H, F = 4, 256, 384
+    check_pack(host_weights(E, H, F), E, H, F, INT_FMT, per=2)
+
+
+def test_pack_outliers_ties_at_the_threshold():
+    # weights on a 1/64 grid: hundreds of equal |w| (of both signs) straddle the cut
+    E, H, F = 4, 256, 512
+    Wh = np.round(host_weights(E, H, F, 40) * 64.0).astype(np.float32) / np.float32(64.0)
+    layer, isos = check_pack(Wh, E, H, F, INT_FMT)
+    N, K = F, H
+    mags = np.abs(Wh[0, 0].reshape(N, K))
+    thr = mags[isos[(0, 0)]["rows"], isos[(0, 0)]["cols"]].min()
+    assert (mags == thr).sum() > ol.count(N, K) // 4  # a real tie at the threshold
+
+
+def test_pack_outliers_nvfp4_bit_exact():
+    E, H, F = 3, 256, 384
+    fmt = np.array([[16 | OUT, 16 | OUT, 16 | OUT], [16, 16 | OUT, 16], [16 | OUT, 16, 16 | OUT]],
+                   np.uint8).reshape(-1)
+    Wh = plant_outliers(host_weights(E, H, F, 50), H, F, 7)
+    check_pack(Wh, E, H, F, fmt)
+
+
+def test_pack_outliers_full_size_projection():
+    # one expert of the 4096 x 14336 (Mixtral-shaped) layer: 29360 outliers per
+    # matrix, a 896-chunk tie search on 58.7M weights
+    E, H, F = 1, 4096, 14336
+    fmt = np.array([3 | OUT, 2 | OUT, 4 | OUT], np.uint8)
+    check_pack(host_weights(E, H, F, 60), E, H, F, fmt)
+
+
+def test_pack_without_flags_is_unchanged():
+    E, H, F = 2, 256, 256
+    fmt = np.array([4, 2, 1, 3, 4, 2], np.uint8)
+    Wh = host_weights(E, H, F, 70)
+    layer, _ = check_pack(Wh, E, H, F, fmt)
+    np.testing.assert_array_equal(layer.packed.cpu().numpy(), orc.pack_layer(Wh, 0, E, H, F, fmt))
+
+
+# ------------------------------------------------------------------ forward
+
+def dense_mats(buf, isos, fmt, E, H, F):
+    """Per expert, the float64 matrices the layer uses: the dense part decoded by the
+    oracle, plus the residuals at the outlier positions (oracle/outliers.py)."""
+    def mats(e):
+        out = []
+        for p in range(3):
+            Wd = orc.layer_decode_matrix(buf, e, p)
+            if (e, p) in isos:
+                iso = isos[(e, p)]
+                for n, kk, r in zip(iso["rows"], iso["cols"], iso["resid"]):
+                    Wd[n, kk] += orc.f16_value(int(r))
+            out.append(Wd)
+        return out
+    return mats
+
+
+def run_forward(layer, E, H, F, k, T, fp4, bias=None):
+    x = W.device_x(T, H)
+    Wr_h = W.router_w(E, H)
+    Wr = torch.from_numpy(Wr_h).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    idx = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    y = moe.moe_layer_forward(x, Wr, None, layer, k, debug=dict(status=status, topk_idx=idx))
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return y, Wr_h, idx.cpu().numpy().reshape(T, k)
+
+
+def check_forward(E, H, F, k, T, fmt, seed):
+    fp4 = bool(np.all((fmt & 0x7F) == 16))
+    Wh = plant_outliers(host_weights(E, H, F, seed), H, F, seed)
+    layer, _ = gpu_pack_host(Wh, E, H, F, fmt)
+    buf, isos, _ = oracle_outlier_layer(Wh, E, H, F, fmt)
+    y, Wr_h, idx_g = run_forward(layer, E, H, F, k, T, fp4)
+    x_bits = W.x_bf16_bits(T, H)
+    logits, idx_o, _ = hp.oracle_route(x_bits, Wr_h, None, k)
+    ties = hp.near_tie_tokens(logits, k, idx_g, idx_o)
+    mats = dense_mats(buf, isos, fmt, E, H, F)
+    y_ref = hp.oracle_forward_rows_dense(mats, x_bits, Wr_h, None, k, fp4=fp4,
+                                         idx_override=idx_g if ties else None)
+    ratio = hp.check_output(y, y_ref)
+    # without the residuals the reference is far off: the side lists carry real weight
+    y_dense = hp.oracle_forward_rows(buf, x_bits, Wr_h, None, k, idx_override=idx_g if ties else None,
+                                     fp4=fp4)[0]
+    assert np.abs(y_dense - y_ref).max() > 3 * hp.TOL * np.abs(y_ref).max()
+    return ratio
+
+
+# decode (GEMV) and prefill (tcgen05) batches; H=512/F=768 takes the CTA-pair
+# kernels (down weight tiles in pairs), H=384/F=640 the single-CTA ones
+@pytest.mark.parametrize("H,F,T", [(512, 768, 9), (512, 768, 600), (384, 640, 9), (384, 640, 600)])
+def test_forward_outliers_integer(H, F, T):
+    check_forward(4, H, F, 2, T, INT_FMT, 80 + T)
+
+
+@pytest.mark.parametrize("H,F,T", [(512, 768, 9), (512, 768, 300), (384, 640, 300)])
+def test_forward_outliers_nvfp4(H, F, T):
+    fmt = np.array([[16 | OUT, 16 | OUT, 16 | OUT], [16, 16 | OUT, 16 | OUT],
+                    [16 | OUT, 16, 16 | OUT], [16 | OUT, 16 | OUT, 16]], np.uint8).reshape(-1)
+    check_forward(4, H, F, 2, T, fmt, 90 + T)
+
+
+def test_outliers_with_nvfp4_activations_rejected():
+    E, H, F = 2, 256, 256
+    fmt = np.array([16 | OUT, 16, 16, 16, 16, 16], np.uint8)
+    layer, _ = gpu_pack_host(host_weights(E, H, F), E, H, F, fmt)
+    layer = moe.PackedLayer(E, H, F, fmt, layer.packed, moe.ACT_NVFP4)
+    x = W.device_x(4, H)
+    Wr = torch.from_numpy(W.router_w(E, H)).cuda()
+    with pytest.raises(moe.MoeError, match="MOE_ERR_FORMAT"):
+        moe.moe_layer_forward(x, Wr, None, layer, 1)
