@@ -58,6 +58,7 @@ __global__ void __launch_bounds__(256) act_quant_nvfp4_kernel(const Src* __restr
                                                               int ld, float* __restrict__ s_out, __half* __restrict__ bval,
                                                               uint8_t* __restrict__ dbg_codes,
                                                               uint8_t* __restrict__ dbg_sf, float* __restrict__ dbg_s) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   const int lane = threadIdx.x & 31;
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= rows) return;
@@ -121,6 +122,7 @@ __global__ void __launch_bounds__(256) act_quant_nvfp4_kernel(const Src* __restr
 __global__ void gather_nvfp4_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf,
                                     const int32_t* __restrict__ perm, int R, int K, int ld, int k,
                                     uint8_t* __restrict__ codes_out, uint8_t* __restrict__ sf_out) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   const int per_row = K / 32 + ld / 16;  // 16-byte pieces: codes, then scales
   const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (i >= (long long)R * per_row) return;
@@ -140,6 +142,7 @@ __global__ void gather_nvfp4_kernel(const uint8_t* __restrict__ codes, const uin
 __global__ void gather_nvfp4_f16_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf,
                                         const int32_t* __restrict__ perm, int R, int K, int ld, int k,
                                         __half* __restrict__ xs, int32_t* counters, int n_counters) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0;
   const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
@@ -161,15 +164,15 @@ __global__ void gather_nvfp4_f16_kernel(const uint8_t* __restrict__ codes, const
 cudaError_t launch_gather_nvfp4(const __nv_bfloat16* x, int T, int H, int k, bool tc, const Workspace& ws,
                                 uint8_t* dbg_xq, uint8_t* dbg_xsb, float* dbg_sx, cudaStream_t stream) {
   const int R = T * k;
-  act_quant_nvfp4_kernel<__nv_bfloat16><<<(T + 7) / 8, 256, 0, stream>>>(x, T, H, ws.xq, ws.xsf, ws.ldx, ws.sx,
+  launch_chained(act_quant_nvfp4_kernel<__nv_bfloat16>, dim3((T + 7) / 8), dim3(256), 0, stream, x, T, H, ws.xq, ws.xsf, ws.ldx, ws.sx,
                                                                          nullptr, dbg_xq, dbg_xsb, dbg_sx);
   if (tc) {
     const long long n = (long long)R * (H / 32 + ws.ldx / 16);
-    gather_nvfp4_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(ws.xq, ws.xsf, ws.perm, R, H, ws.ldx, k,
+    launch_chained(gather_nvfp4_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, stream, ws.xq, ws.xsf, ws.perm, R, H, ws.ldx, k,
                                                                        ws.xs4, ws.xsf4);
   } else {
     const long long n = (long long)R * (H / 16);
-    gather_nvfp4_f16_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(
+    launch_chained(gather_nvfp4_f16_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, stream,
         ws.xq, ws.xsf, ws.perm, R, H, ws.ldx, k, (__half*)ws.xs, ws.counters, ws.counter_len);
   }
   return cudaGetLastError();
@@ -177,7 +180,7 @@ cudaError_t launch_gather_nvfp4(const __nv_bfloat16* x, int T, int H, int k, boo
 
 cudaError_t launch_act_quant_h_nvfp4(int R, int F, bool tc, const Workspace& ws, uint8_t* dbg_hq, uint8_t* dbg_hsb,
                                      float* dbg_sh, cudaStream_t stream) {
-  act_quant_nvfp4_kernel<float><<<(R + 7) / 8, 256, 0, stream>>>(
+  launch_chained(act_quant_nvfp4_kernel<float>, dim3((R + 7) / 8), dim3(256), 0, stream,
       (const float*)ws.h, R, F, tc ? ws.hs4 : nullptr, tc ? ws.hsf4 : nullptr, ws.ldh, ws.sh,
       tc ? nullptr : (__half*)ws.hb, dbg_hq, dbg_hsb, dbg_sh);
   return cudaGetLastError();

@@ -9,6 +9,7 @@ namespace moe {
 __global__ void combine_kernel(const float* __restrict__ o, const float* __restrict__ wts,
                                const int32_t* __restrict__ inv, int k, int H,
                                __nv_bfloat16* __restrict__ y) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   const int t = blockIdx.x;
   int rows[kMaxK];
   float w[kMaxK];
@@ -37,7 +38,7 @@ __global__ void combine_kernel(const float* __restrict__ o, const float* __restr
 cudaError_t launch_combine(int T, int k, int H, const Workspace& ws, __nv_bfloat16* y, cudaStream_t stream) {
   int ny = T < 512 ? (H / 4 + 255) / 256 : 1;  // column blocks: more parallelism for few tokens
   if (ny > 8) ny = 8;
-  combine_kernel<<<dim3(T, ny), 256, 0, stream>>>(ws.o, ws.wts, ws.inv, k, H, y);
+  launch_chained(combine_kernel, dim3(T, ny), dim3(256), 0, stream, ws.o, ws.wts, ws.inv, k, H, y);
   return cudaGetLastError();
 }
 

@@ -113,6 +113,7 @@ __host__ __device__ constexpr uint32_t idesc_fp4(int N) {
 __global__ void __launch_bounds__(kF4Threads, 1)
     expert_gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_sfb,
                            const F4Args a) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kF4Slots * kF4SlotBytes);
@@ -505,7 +506,7 @@ cudaError_t launch_expert_gemm_fp4(const uint8_t* packed, int E, int H, int F, i
     return cudaErrorInvalidValue;
   cudaError_t err = cudaFuncSetAttribute(expert_gemm_fp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kF4Smem);
   if (err != cudaSuccess) return err;
-  expert_gemm_fp4_kernel<<<fp4_sm_count(), kF4Threads, kF4Smem, stream>>>(mb, ms, a);
+  launch_chained(expert_gemm_fp4_kernel, dim3(fp4_sm_count()), dim3(kF4Threads), kF4Smem, stream, mb, ms, a);
   return cudaGetLastError();
 }
 

@@ -400,6 +400,7 @@ __device__ __forceinline__ bool dequant_item_any(int f0, int f1, const Ring R, l
 template <int NMAT, bool CG2, bool I1, bool OUT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   using C = TcCfg<NMAT, CG2>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array by pointer arithmetic (an
@@ -871,17 +872,19 @@ cudaError_t launch_tc(TcArgs a, int max_words, const void* act, int rows_total, 
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   if (!CG2) {
-    kern<<<sm_count(), kTcThreads, smem, stream>>>(map, a);
+    launch_chained(kern, dim3(sm_count()), dim3(kTcThreads), smem, stream, map, a);
     return cudaGetLastError();
   }
   // one persistent pair of CTAs per pair of SMs: as many clusters as can be
   // resident at once (a GPC with an odd number of free SMs leaves one idle)
   cudaLaunchConfig_t cfg{};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // chained like the other kernels
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(kTcThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -893,6 +896,7 @@ cudaError_t launch_tc(TcArgs a, int max_words, const void* act, int rows_total, 
   if (err != cudaSuccess) return err;
   if (clusters < 1) return cudaErrorInvalidConfiguration;
   cfg.gridDim = dim3((unsigned)(2 * min(clusters, sm_count() / 2)));
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, map, a);
 }
 

@@ -487,6 +487,7 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
                                                                    const __grid_constant__ CUtensorMap tm_x,
                                                                    const __grid_constant__ CUtensorMap tm_s,
                                                                    const GemvArgs a) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array by pointer arithmetic
   uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -702,6 +703,7 @@ __global__ void __launch_bounds__(kGemvThreads, NT8 == 1 ? (NMAT == 1 ? 4 : 3) :
 // Gate/up of integer layers also writes the group sums of h for the down GEMV.
 template <int NMAT>
 __global__ void __launch_bounds__(256) gemv_fixup_kernel(GemvArgs a, const int32_t* idx) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   const int r = blockIdx.x;
   const int e = idx[a.perm[r]];
   const LayerHdr L = hdr_view(a.packed, a.E, a.H, a.F);
@@ -843,7 +845,7 @@ cudaError_t launch_n(GemvArgs g, const uint8_t* packed, uint64_t packed_bytes, c
   long long grid = (long long)gemv_sm_count() * (per_sm > 0 ? per_sm : 1);
   if (grid > items) grid = items;
   if (grid < 1) grid = 1;
-  kern<<<(unsigned)grid, kGemvThreads, smem, stream>>>(m1, m2, m3, m4, mx, ms, g);
+  launch_chained(kern, dim3((unsigned)grid), dim3(kGemvThreads), smem, stream, m1, m2, m3, m4, mx, ms, g);
   return cudaGetLastError();
 }
 
@@ -930,9 +932,9 @@ cudaError_t launch_expert_gemv(const uint8_t* packed, uint64_t packed_bytes, con
                : launch_n<1, 1, false>(g, packed, packed_bytes, act, sums, wmax, max_chunks, stream);
   if (err != cudaSuccess || g.P == 1) return err;
   if (gateup)
-    gemv_fixup_kernel<2><<<dim3(R, (g.N + 255) / 256), 256, 0, stream>>>(g, ws.idx);
+    launch_chained(gemv_fixup_kernel<2>, dim3(R, (g.N + 255) / 256), dim3(256), 0, stream, g, ws.idx);
   else
-    gemv_fixup_kernel<1><<<dim3(R, (g.N + 255) / 256), 256, 0, stream>>>(g, ws.idx);
+    launch_chained(gemv_fixup_kernel<1>, dim3(R, (g.N + 255) / 256), dim3(256), 0, stream, g, ws.idx);
   return cudaGetLastError();
 }
 

@@ -9,7 +9,40 @@
 
 #include "../../include/moe.h"
 
+#include <utility>
+
 namespace moe {
+
+// ---------------------------------------------------------------- launch chaining
+// The forward's kernels are launched with programmatic dependent launch: a kernel
+// may be scheduled while its predecessor on the stream is still draining, so its
+// launch and block setup overlap the predecessor's tail.  Every forward kernel
+// therefore starts with pdl_enter(): griddepcontrol.wait blocks until the
+// predecessor grid has completed and its memory is visible (a no-op for a plain
+// launch), and only then may the kernel read or write global memory.  Because each
+// kernel waits for its predecessor before it can complete, a kernel also sees the
+// results of every earlier kernel of the chain.  The trigger that follows lets the
+// next kernel be scheduled as soon as every block of this one has started.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... Exp, typename... Act>
+inline cudaError_t launch_chained(void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                  Act&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Act>(args)...);
+}
 
 constexpr uint32_t kMagic = 0x51454F4Du;
 constexpr uint32_t kHdrBytes = 16384u;

@@ -16,6 +16,7 @@ constexpr int kPermBlock = 1024;
 __global__ void __launch_bounds__(kPermBlock) perm_count_kernel(const int32_t* __restrict__ idx, int R,
                                                                 int E, int32_t* __restrict__ blk_hist,
                                                                 int32_t* __restrict__ rank) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   __shared__ int32_t wcnt[kPermBlock / 32][kMaxE];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i < (kPermBlock / 32) * kMaxE; i += kPermBlock) (&wcnt[0][0])[i] = 0;
@@ -48,6 +49,7 @@ __global__ void __launch_bounds__(256) perm_scan_kernel(int32_t* __restrict__ bl
                                                         int32_t* __restrict__ chunks,
                                                         int32_t* __restrict__ chunk_count,
                                                         int32_t* __restrict__ dbg_counts) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   __shared__ int32_t s_cnt[kMaxE], s_off[kMaxE + 1], s_nc[kMaxE], s_cstart[kMaxE + 1];
   const int e = threadIdx.x;
   int total = 0;
@@ -98,6 +100,7 @@ __global__ void __launch_bounds__(kPermBlock) perm_scatter_kernel(const int32_t*
                                                                   int32_t* __restrict__ inv,
                                                                   int32_t* __restrict__ dbg_perm,
                                                                   int32_t* __restrict__ dbg_inv) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   const int i = blockIdx.x * kPermBlock + threadIdx.x;
   if (i >= R) return;
   const int e = idx[i];
@@ -120,6 +123,7 @@ __global__ void __launch_bounds__(kPermBlock) perm_small_kernel(const int32_t* _
                                                                 int32_t* __restrict__ dbg_counts,
                                                                 int32_t* __restrict__ dbg_perm,
                                                                 int32_t* __restrict__ dbg_inv) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   __shared__ int32_t wcnt[kPermBlock / 32][kMaxE];
   __shared__ int32_t s_off[kMaxE + 1], s_cstart[kMaxE + 1], s_cnt[kMaxE];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -201,6 +205,7 @@ __global__ void __launch_bounds__(128) gather_f16_kernel(const __nv_bfloat16* __
                                                          __half* __restrict__ xs, float* __restrict__ xsum,
                                                          float* __restrict__ xinv, int32_t* counters,
                                                          int n_counters) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   __shared__ float s_max[4];
   if (blockIdx.x == 0 && blockIdx.y == 0) zero_counters(counters, n_counters);
   const int r = blockIdx.x;
@@ -255,6 +260,7 @@ __global__ void __launch_bounds__(128) gather_f16_kernel(const __nv_bfloat16* __
 __global__ void act_quant_x_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, uint8_t* __restrict__ xq,
                                    float* __restrict__ sx, uint8_t* __restrict__ dbg_xq,
                                    float* __restrict__ dbg_sx) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -289,6 +295,7 @@ __global__ void act_quant_x_kernel(const __nv_bfloat16* __restrict__ x, int T, i
 // thread per 16 codes (hardware e4m3x2 -> f16x2 conversion).
 __global__ void gather_fp8_kernel(const uint8_t* __restrict__ xq, const int32_t* __restrict__ perm, int R,
                                   int H, int k, __half* __restrict__ xs, int32_t* counters, int n_counters) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   if (blockIdx.x == 0) zero_counters(counters, n_counters);
   const int per_row = H / 16;
   const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
@@ -315,6 +322,7 @@ __global__ void gather_fp8_kernel(const uint8_t* __restrict__ xq, const int32_t*
 __global__ void act_quant_h_kernel(const float* __restrict__ h, int R, int F, uint8_t* __restrict__ hq,
                                    float* __restrict__ sh, __half* __restrict__ hb,
                                    uint8_t* __restrict__ dbg_hq, float* __restrict__ dbg_sh) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   const int lane = threadIdx.x & 31;
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= R) return;
@@ -352,14 +360,14 @@ cudaError_t launch_permute(int T, int k, int E, int chunk_rows, const Workspace&
   const int R = T * k;
   const int nblk = (R + kPermBlock - 1) / kPermBlock;
   if (nblk == 1) {
-    perm_small_kernel<<<1, kPermBlock, 0, stream>>>(ws.idx, R, E, chunk_rows, ws.counts, ws.offsets, ws.chunks,
+    launch_chained(perm_small_kernel, dim3(1), dim3(kPermBlock), 0, stream, ws.idx, R, E, chunk_rows, ws.counts, ws.offsets, ws.chunks,
                                                     ws.chunk_count, ws.perm, ws.inv, dbg_counts, dbg_perm, dbg_inv);
     return cudaGetLastError();
   }
-  perm_count_kernel<<<nblk, kPermBlock, 0, stream>>>(ws.idx, R, E, ws.blk_hist, ws.rank);
-  perm_scan_kernel<<<1, 256, 0, stream>>>(ws.blk_hist, nblk, E, R, chunk_rows, ws.counts, ws.offsets,
+  launch_chained(perm_count_kernel, dim3(nblk), dim3(kPermBlock), 0, stream, ws.idx, R, E, ws.blk_hist, ws.rank);
+  launch_chained(perm_scan_kernel, dim3(1), dim3(256), 0, stream, ws.blk_hist, nblk, E, R, chunk_rows, ws.counts, ws.offsets,
                                           ws.chunks, ws.chunk_count, dbg_counts);
-  perm_scatter_kernel<<<nblk, kPermBlock, 0, stream>>>(ws.idx, R, E, ws.blk_hist, ws.rank, ws.perm, ws.inv,
+  launch_chained(perm_scatter_kernel, dim3(nblk), dim3(kPermBlock), 0, stream, ws.idx, R, E, ws.blk_hist, ws.rank, ws.perm, ws.inv,
                                                        dbg_perm, dbg_inv);
   return cudaGetLastError();
 }
@@ -368,14 +376,14 @@ cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4,
                           uint8_t* dbg_xq, float* dbg_sx, cudaStream_t stream) {
   const int R = T * k;
   if (fp4) {
-    act_quant_x_kernel<<<(T + 7) / 8, 256, 0, stream>>>(x, T, H, ws.xq, ws.sx, dbg_xq, dbg_sx);
+    launch_chained(act_quant_x_kernel, dim3((T + 7) / 8), dim3(256), 0, stream, x, T, H, ws.xq, ws.sx, dbg_xq, dbg_sx);
     const long long n = (long long)R * (H / 16);
-    gather_fp8_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(ws.xq, ws.perm, R, H, k, (__half*)ws.xs,
+    launch_chained(gather_fp8_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, stream, ws.xq, ws.perm, R, H, k, (__half*)ws.xs,
                                                                      ws.counters, ws.counter_len);
   } else {
     int ny = R < 512 ? (H / 8 + 127) / 128 : 1;  // column blocks: more parallelism for few rows
     if (ny > 8) ny = 8;
-    gather_f16_kernel<<<dim3(R, ny), 128, 0, stream>>>(x, ws.perm, R, H, k, (__half*)ws.xs, ws.xsum, ws.xinv,
+    launch_chained(gather_f16_kernel, dim3(R, ny), dim3(128), 0, stream, x, ws.perm, R, H, k, (__half*)ws.xs, ws.xsum, ws.xinv,
                                                        ws.counters, ws.counter_len);
   }
   return cudaGetLastError();
@@ -383,7 +391,7 @@ cudaError_t launch_gather(const __nv_bfloat16* x, int T, int H, int k, bool fp4,
 
 cudaError_t launch_act_quant_h(int R, int F, const Workspace& ws, uint8_t* dbg_hq, float* dbg_sh,
                                cudaStream_t stream) {
-  act_quant_h_kernel<<<(R + 7) / 8, 256, 0, stream>>>((const float*)ws.h, R, F, ws.hq, ws.sh, (__half*)ws.hb,
+  launch_chained(act_quant_h_kernel, dim3((R + 7) / 8), dim3(256), 0, stream, (const float*)ws.h, R, F, ws.hq, ws.sh, (__half*)ws.hb,
                                                       dbg_hq, dbg_sh);
   return cudaGetLastError();
 }

@@ -15,6 +15,7 @@ namespace moe {
 __global__ void router_warp_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ Wr,
                                    const float* __restrict__ b, int T, int H, int E,
                                    float* __restrict__ logits) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.y * (blockDim.x >> 5) + warp;
   const int t = blockIdx.x;
@@ -43,6 +44,7 @@ __global__ void router_warp_kernel(const __nv_bfloat16* __restrict__ x, const fl
 __global__ void __launch_bounds__(128) router_dot_kernel(const __nv_bfloat16* __restrict__ x,
                                                          const float* __restrict__ Wr, const float* __restrict__ b,
                                                          int T, int H, int E, float* __restrict__ logits) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   __shared__ float red[4];
   const int t = blockIdx.x, e = blockIdx.y;
   const __nv_bfloat16* xr = x + (size_t)t * H;
@@ -79,6 +81,7 @@ __global__ void __launch_bounds__(128) router_dot_kernel(const __nv_bfloat16* __
 
 // Wr fp32 [E][H] -> Wb bf16 [3][E][H] (hi, mid, lo).
 __global__ void router_split_kernel(const float* __restrict__ Wr, long long n, __nv_bfloat16* __restrict__ Wb) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     const float w = Wr[i];
     const __nv_bfloat16 hi = __float2bfloat16_rn(w);
@@ -123,6 +126,7 @@ __global__ void __launch_bounds__(256, 2) router_mma_kernel(const __nv_bfloat16*
                                                          const __nv_bfloat16* __restrict__ Wb,
                                                          const float* __restrict__ b, int T, int H, int E,
                                                          float* __restrict__ logits) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   extern __shared__ __align__(16) __nv_bfloat16 rsm[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wm = warp & 3, wn = warp >> 2;
@@ -232,6 +236,7 @@ __global__ void __launch_bounds__(256, 2) router_mma_kernel(const __nv_bfloat16*
 __global__ void topk_softmax_kernel(const float* __restrict__ logits, int nparts, int T, int E, int k,
                                     int32_t* __restrict__ idx, float* __restrict__ wts,
                                     int32_t* __restrict__ dbg_idx, float* __restrict__ dbg_w) {
+  pdl_enter();  // before any global memory access (see moe_common.cuh)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= T) return;
@@ -315,21 +320,21 @@ cudaError_t launch_router_topk(const __nv_bfloat16* x, const float* Wr, const fl
                                cudaStream_t stream) {
   const int parts = router_parts(T, H, E);
   if (parts == 0 && T <= 64 && E <= 32) {  // decode, few experts: one block per dot product
-    router_dot_kernel<<<dim3(T, E), 128, 0, stream>>>(x, Wr, b, T, H, E, ws.logits);
+    launch_chained(router_dot_kernel, dim3(T, E), dim3(128), 0, stream, x, Wr, b, T, H, E, ws.logits);
   } else if (parts == 0) {  // many tokens, few experts: one warp per dot product
     dim3 grid(T, (E + 7) / 8);
-    router_warp_kernel<<<grid, 256, 0, stream>>>(x, Wr, b, T, H, E, ws.logits);
+    launch_chained(router_warp_kernel, dim3(grid), dim3(256), 0, stream, x, Wr, b, T, H, E, ws.logits);
   } else {
     const long long n = (long long)E * H;
-    router_split_kernel<<<(int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0, stream>>>(Wr, n, ws.wsplit);
+    launch_chained(router_split_kernel, dim3((int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096)), dim3(256), 0, stream, Wr, n, ws.wsplit);
     cudaError_t aerr = cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRSmem);
     if (aerr != cudaSuccess) return aerr;
     dim3 grid((T + kRT - 1) / kRT, (E + kRE - 1) / kRE, parts);
-    router_mma_kernel<<<grid, 256, kRSmem, stream>>>(x, ws.wsplit, b, T, H, E, ws.logits);
+    launch_chained(router_mma_kernel, dim3(grid), dim3(256), kRSmem, stream, x, ws.wsplit, b, T, H, E, ws.logits);
   }
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  topk_softmax_kernel<<<(T + 7) / 8, 256, 0, stream>>>(ws.logits, parts > 1 ? parts : 1, T, E, k, ws.idx, ws.wts,
+  launch_chained(topk_softmax_kernel, dim3((T + 7) / 8), dim3(256), 0, stream, ws.logits, parts > 1 ? parts : 1, T, E, k, ws.idx, ws.wts,
                                                         dbg_idx, dbg_w);
   return cudaGetLastError();
 }

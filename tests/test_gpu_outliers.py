@@ -237,9 +237,10 @@ def check_forward(E, H, F, k, T, fmt, seed):
     return ratio
 
 
-# decode (GEMV) and prefill (tcgen05) batches; H=512/F=768 takes the CTA-pair
-# kernels (down weight tiles in pairs), H=384/F=640 the single-CTA ones
-@pytest.mark.parametrize("H,F,T", [(512, 768, 9), (512, 768, 600), (384, 640, 9), (384, 640, 600)])
+# decode (GEMV: one chunk per expert at T=9, several at T=30) and prefill (tcgen05)
+# batches; H=512/F=768 takes the CTA-pair kernels (down weight tiles in pairs),
+# H=384/F=640 the single-CTA ones
+@pytest.mark.parametrize("H,F,T", [(512, 768, 9), (512, 768, 30), (512, 768, 600), (384, 640, 9), (384, 640, 600)])
 def test_forward_outliers_integer(H, F, T):
     check_forward(4, H, F, 2, T, INT_FMT, 80 + T)
 

@@ -239,6 +239,19 @@ def test_forward_ragged_mixed_formats():
     check_layer(L, 37)
 
 
+@pytest.mark.parametrize("fmt,act", [
+    ([[3, 2, 4], [1, 1, 1], [4, 1, 2], [2, 3, 3], [4, 4, 4], [2, 2, 1]], 0),
+    ([[16, 16, 16]] * 6, 0),
+    ([[16, 16, 16]] * 6, 1),
+], ids=["int", "nvfp4", "nvfp4-act4"])
+def test_forward_gemv_several_chunks_per_expert(fmt, act):
+    # 100 expert rows over 6 experts (about 17 each, below the tcgen05 threshold): the GEMV walks
+    # each expert's rows as two or three 8-row chunks over the same weight tiles, the last ragged
+    L = custom("gemvchunks" + str(fmt[0][0]) + str(fmt[1][0]) + str(act), 50, 384, 640, 6, 2, fmt)
+    r = check_layer(L, 50, act=act)
+    assert r["counts"].max() > 16  # some expert takes three chunks
+
+
 def test_forward_prefill_chunks_and_tails():
     # more than 16 rows per expert: 64-row chunks, several per expert, ragged tails
     L = custom("chunks", 300, 256, 384, 4, 2, [[4, 4, 4], [3, 2, 4], [2, 2, 2], [4, 3, 2]])
