@@ -279,6 +279,9 @@ def measure_batch(L: W.Layer, layer, T: int, moe, dev, pk, flush, n: int, seed: 
             out[key] = {"bound": "tensor", "achieved": round(f / t / 1e9, 1), "peak": round(peak, 1),
                         "unit": "TFLOP/s", "frac": round(f / t / 1e9 / peak, 4),
                         "algorithmic_flops_per_launch": f, "avg_launch_ms": round(t, 4)}
+            if pk.get("bf16_tflops_sustained"):  # the same against the sustained (power-capped) peak
+                ps = pk["bf16_tflops_sustained"] * (FP4_PER_BF16 if act else 1.0)
+                out[key]["frac_sustained"] = round(f / t / 1e9 / ps, 4)
             if act:
                 out[key]["peak_source"] = "measured dense bf16 burst x 4 (nominal FP4/bf16 ratio)"
     del ws, x, y
@@ -388,14 +391,23 @@ def run_ours(args, rank, world, local_rank):
     flops_gateup = 2.0 * T * L.k * 2 * L.H * L.F
     flops_down = 2.0 * T * L.k * L.H * L.F
     achieved = flops_gateup / (gateup_ms / 1e3) / 1e12
+    achieved_down = flops_down / (down_ms / 1e3) / 1e12
+    # The GEMMs run inside back-to-back steps of tens of milliseconds of tensor-core
+    # work, under the 1 kW power cap: the sustained GEMM peak is their denominator
+    # (the burst figure is kept beside it).
+    sustained = pk.get("bf16_tflops_sustained")
+    peak = sustained or pk["bf16_tflops"]
     roofline = {"bound": "tensor", "kernel": "expert GEMM gate/up + SwiGLU (tcgen05, fp16 operands)",
-                "achieved": round(achieved, 2), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": ncu_traffic(f"gateup_prefill_{name}"),
-                "peak_source": f"{pk_kind} dense bf16 (= fp16) burst, MEASURED_PEAKS.json"
-                if pk_kind == "measured" else "fallback 1.59 PFLOP/s",
+                "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": ncu_traffic(f"gateup_prefill_{name}"),
+                "peak_source": (f"{pk_kind} dense bf16 (= fp16) GEMM, sustained (back to back under the power "
+                                f"cap), MEASURED_PEAKS.json" if sustained else
+                                f"{pk_kind} dense bf16 (= fp16) burst" if pk_kind == "measured"
+                                else "fallback 1.59 PFLOP/s"),
+                "peak_burst": pk["bf16_tflops"], "frac_burst": round(achieved / pk["bf16_tflops"], 4),
                 "algorithmic_flops_per_launch": flops_gateup, "avg_launch_ms": round(gateup_ms, 4),
-                "down": {"achieved": round(flops_down / (down_ms / 1e3) / 1e12, 2),
-                         "frac": round(flops_down / (down_ms / 1e3) / 1e12 / pk["bf16_tflops"], 4),
+                "down": {"achieved": round(achieved_down, 2), "frac": round(achieved_down / peak, 4),
+                         "frac_burst": round(achieved_down / pk["bf16_tflops"], 4),
                          "avg_launch_ms": round(down_ms, 4),
                          "traffic": ncu_traffic(f"down_prefill_{name}")}}
     stages = dict(zip(STAGES, [round(float(v), 4) for v in stage_ms.mean(0)]))

@@ -399,7 +399,8 @@ __device__ __forceinline__ bool dequant_item_any(int f0, int f1, const Ring R, l
 // OUT: the layer has outlier side lists (their residuals are added in the epilogue)
 template <int NMAT, bool CG2, bool I1, bool OUT>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_b, const TcArgs a) {
+    expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_bh,
+                          const TcArgs a) {
   pdl_enter();  // before any global memory access (see moe_common.cuh)
   using C = TcCfg<NMAT, CG2>;
   extern __shared__ uint8_t smem_raw[];
@@ -447,7 +448,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ptx::tmem_relinquish();
     }
   }
-  if (warp == kBWarp && lane == 0) ptx::prefetch_tmap(&tmap_b);
+  if (warp == kBWarp && lane == 0) {
+    ptx::prefetch_tmap(&tmap_b);
+    ptx::prefetch_tmap(&tmap_bh);
+  }
   ptx::tc_fence_before();
   __syncthreads();
   if (CG2) ptx::cluster_sync();  // the peer's barriers are initialised before any remote arrival
@@ -539,14 +543,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // this CTA's token rows of the MMA's N = nmma columns: the first or second half
       const int nmma = min(kTcBN, (a.chunks[3 * c + 2] + 15) & ~15);
       const int row0 = a.chunks[3 * c + 1] + (int)rank * (nmma / 2);
+      // a chunk whose rows fit half the tile loads a half-height box: the MMA reads
+      // only the first rows of the slot, and the rest would be another chunk's rows
+      const bool half = (CG2 ? nmma / 2 : nmma) <= C::kBRows / 2;
+      const CUtensorMap* bmap = half ? &tmap_bh : &tmap_b;
+      const uint32_t bbytes = half ? (uint32_t)C::kBBytes / 2u : (uint32_t)C::kBBytes;
       for (int ks = 0; ks < ksteps; ++ks) {
         if (!wait_all(&B.b_empty[bs], bph ^ 1u)) {
           ok = false;
           break;
         }
         if (lane == 0 && !a.withhold) {
-          ptx::mbar_arrive_expect_tx(&B.b_full[bs], (uint32_t)C::kBBytes);
-          ptx::tma_load_2d(smem + R.off_b + bs * C::kBBytes, &tmap_b, ks * kTcBK, row0, &B.b_full[bs]);
+          ptx::mbar_arrive_expect_tx(&B.b_full[bs], bbytes);
+          ptx::tma_load_2d(smem + R.off_b + bs * C::kBBytes, bmap, ks * kTcBK, row0, &B.b_full[bs]);
         }
         __syncwarp();
         if (!a.withhold) {
@@ -701,9 +710,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ptx::tc_fence_after();
       const int nrow = (a.pair ? 2 * mt : mt) * kTcBM + q * 32 + lane;
       const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+      // the chunk's columns (tokens) split evenly over the kColGroups column groups, in
+      // steps of 16, so that every epilogue warp has work when a chunk holds few rows
+      const int cpw = ((rows + 16 * kColGroups - 1) / (16 * kColGroups)) * 16, c0 = cq * cpw;
       bool range = false;  // an fp16 SwiGLU output overflowed
       if (a.row_scale) {
-        // NVFP4 layers: the row scales of the warp's kColsPerWarp tokens (gate/up: the
+        // NVFP4 layers: the row scales of the warp's (at most 64) tokens (gate/up: the
         // token's sx through perm; down: the row's sh), two per lane, loaded before any
         // store and broadcast with shuffles -- loaded inside the store loop, each would
         // wait for the stores before it.
@@ -711,23 +723,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         float fac[2] = {0.0f, 0.0f};
 #pragma unroll
         for (int u2 = 0; u2 < 2; ++u2) {
-          const int tok = cq * kColsPerWarp + 32 * u2 + lane;
-          if (tok < rows) {
+          const int tok = c0 + 32 * u2 + lane;
+          if (32 * u2 + lane < cpw && tok < rows) {
             const int r = row0 + tok;
             fac[u2] = (NMAT == 2 && !a.pair) ? a.row_scale[a.perm[r] / a.topk] : a.row_scale[r];
           }
         }
         float* __restrict__ out = reinterpret_cast<float*>(a.out);
-        for (int cb = cq * kColsPerWarp; cb < cq * kColsPerWarp + kColsPerWarp && cb < rows; cb += 16) {
+        for (int cb = c0; cb < c0 + cpw && cb < rows; cb += 16) {
           uint32_t r0[16], r1[16];
           ptx::tmem_ld16(lane_base + (uint32_t)cb, r0);
           if (NMAT == 2) ptx::tmem_ld16(lane_base + 256u + (uint32_t)cb, r1);
           ptx::tmem_ld_wait();
-          const float fu = ((cb - cq * kColsPerWarp) >> 5) ? fac[1] : fac[0];  // warp-uniform choice
+          const float fu = ((cb - c0) >> 5) ? fac[1] : fac[0];  // warp-uniform choice
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int tok = cb + j;
-            const float f = __shfl_sync(0xffffffffu, fu, (tok - cq * kColsPerWarp) & 31);
+            const float f = __shfl_sync(0xffffffffu, fu, (tok - c0) & 31);
             if (tok >= rows) continue;
             const size_t o = (size_t)(row0 + tok) * a.N + nrow;
             if (OUT) {  // residuals of the side lists, in the units of the fp16 activations
@@ -761,7 +773,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       } else {
         // integer layers: SwiGLU into fp16 h (gate/up) or fp32 o (down)
-        for (int cb = cq * kColsPerWarp; cb < cq * kColsPerWarp + kColsPerWarp && cb < rows; cb += 16) {
+        for (int cb = c0; cb < c0 + cpw && cb < rows; cb += 16) {
           uint32_t r0[16], r1[16];
           ptx::tmem_ld16(lane_base + (uint32_t)cb, r0);
           if (NMAT == 2) ptx::tmem_ld16(lane_base + 256u + (uint32_t)cb, r1);
@@ -858,13 +870,17 @@ cudaError_t launch_tc(TcArgs a, int max_words, const void* act, int rows_total, 
   const int smem = ring_smem(a.ring);
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
-  CUtensorMap map;
+  CUtensorMap map, map_half;  // activation tiles of kBRows rows, and of kBRows / 2
   const cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)rows_total};
   const cuuint64_t strides[1] = {(cuuint64_t)a.K * 2u};
   const cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)C::kBRows};
+  const cuuint32_t box_half[2] = {(cuuint32_t)kTcBK, (cuuint32_t)(C::kBRows / 2)};
   const CUtensorMapSwizzle swz = kRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   const cuuint32_t estr[2] = {1u, 1u};
   if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(act), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+      enc(&map_half, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(act), dims, strides, box_half, estr,
           CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
@@ -872,7 +888,7 @@ cudaError_t launch_tc(TcArgs a, int max_words, const void* act, int rows_total, 
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   if (!CG2) {
-    launch_chained(kern, dim3(sm_count()), dim3(kTcThreads), smem, stream, map, a);
+    launch_chained(kern, dim3(sm_count()), dim3(kTcThreads), smem, stream, map, map_half, a);
     return cudaGetLastError();
   }
   // one persistent pair of CTAs per pair of SMs: as many clusters as can be
@@ -897,7 +913,7 @@ cudaError_t launch_tc(TcArgs a, int max_words, const void* act, int rows_total, 
   if (clusters < 1) return cudaErrorInvalidConfiguration;
   cfg.gridDim = dim3((unsigned)(2 * min(clusters, sm_count() / 2)));
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, map, a);
+  return cudaLaunchKernelEx(&cfg, kern, map, map_half, a);
 }
 
 }  // namespace
