@@ -360,8 +360,10 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       acc_phase ^= 1u;
       ptx::tc_fence_after();
       if (threadIdx.x == 0) f4_trace(a.trace, 6, item);
-      // epilogue: warp w reads TMEM lane quarter w%4, columns (tokens) [64*(w/4), +64)
+      // epilogue: warp w reads TMEM lane quarter w%4 and half w/4 of the chunk's columns
+      // (tokens), split in steps of 16 so both halves have work on short chunks
       const int q = warp & 3, ch = warp >> 2;
+      const int cpw = ((rows + 31) / 32) * 16, c0 = ch * cpw;
       const int nrow0 = (gate_up ? mi : 2 * mi) * kF4BM + q * 32 + lane;
       float ts[2];
 #pragma unroll
@@ -371,26 +373,26 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       float scl[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int tok = ch * 64 + 32 * u + lane;
+        const int tok = c0 + 32 * u + lane;
         scl[u] = 0.0f;
-        if (tok < rows) {
+        if (32 * u + lane < cpw && tok < rows) {
           const int r = row0 + tok;
           scl[u] = gate_up ? a.row_scale[a.perm[r] / a.topk] : a.row_scale[r];
         }
       }
       float* __restrict__ out = a.out;
       const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-      for (int cb = ch * 64; cb < ch * 64 + 64 && cb < rows; cb += 16) {
+      for (int cb = c0; cb < c0 + cpw && cb < rows; cb += 16) {
         uint32_t r0[16], r1[16];
         ptx::tmem_ld16(lane_base + (uint32_t)cb, r0);
         ptx::tmem_ld16(lane_base + (uint32_t)(kF4BN + cb), r1);
         ptx::tmem_ld_wait();
-        const int u = (cb - ch * 64) >> 5;  // which of the lane's two scales (warp-uniform)
+        const int u = (cb - c0) >> 5;  // which of the lane's two scales (warp-uniform)
         const float su = u ? scl[1] : scl[0];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int tok = cb + j;
-          const float sc = __shfl_sync(0xffffffffu, su, (tok - ch * 64) & 31);
+          const float sc = __shfl_sync(0xffffffffu, su, (tok - c0) & 31);
           if (tok >= rows) continue;
           const size_t o = (size_t)(row0 + tok) * a.N + nrow0;
           if (gate_up) {

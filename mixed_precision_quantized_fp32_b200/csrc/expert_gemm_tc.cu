@@ -103,8 +103,8 @@ template <int NMAT, bool CG2>
 Ring make_ring(int max_words) {
   using C = TcCfg<NMAT, CG2>;
   Ring r;
-  r.a_slots = CG2 ? 3 : 2;
-  r.b_slots = CG2 ? 5 : 3;
+  r.a_slots = CG2 ? 4 : 2;
+  r.b_slots = CG2 ? 4 : 3;
   r.code_bytes = kGroups * 512 * max_words;
   r.raw_bytes = (NMAT * (r.code_bytes + C::kScaleBytes) + 127) / 128 * 128;
   for (;;) {
