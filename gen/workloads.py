@@ -114,7 +114,7 @@ def _dev_lib():
     if _dev is None:
         path = os.path.join(HERE, "libmoegen.so")
         if not os.path.exists(path):
-            raise ImportError(f"{path} missing: build with python -m mixed_precision_quantized_fp32_b200.build")
+            raise ImportError(f"{path} missing: build with python mixed_precision_quantized_fp32_b200/build.py")
         L = C.CDLL(path)
         for fn in (L.moegen_fill_f32, L.moegen_fill_bf16):
             fn.restype = C.c_int

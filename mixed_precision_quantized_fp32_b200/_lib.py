@@ -57,7 +57,7 @@ def load() -> C.CDLL:
     if _lib is None:
         if not os.path.exists(LIB_PATH):
             raise ImportError(f"CUDA library not built: {LIB_PATH} is missing "
-                              "(run python -m mixed_precision_quantized_fp32_b200.build)")
+                              "(run python mixed_precision_quantized_fp32_b200/build.py)")
         L = C.CDLL(LIB_PATH)
         P, i32, u64 = C.c_void_p, C.c_int32, C.c_uint64
         L.moe_pack.restype = C.c_int
