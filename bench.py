@@ -465,7 +465,10 @@ def run_suite(args):
         for T in list(L.decode_T) + list(L.prefill_T):
             if args.batch and T != args.batch:
                 continue
-            print(json.dumps(measure_batch(L, layer, T, moe, dev, pk, flush, 10)), flush=True)
+            act = 1 if (args.act == "nvfp4" and L.fp4) else 0
+            if act:
+                layer = moe.PackedLayer(layer.E, layer.H, layer.F, layer.fmt, layer.packed, moe.ACT_NVFP4)
+            print(json.dumps(measure_batch(L, layer, T, moe, dev, pk, flush, 10, act=act)), flush=True)
         del layer
         torch.cuda.empty_cache()
 
@@ -558,6 +561,8 @@ def main():
     ap.add_argument("--suite", default="", help="comma-separated layers to report instead of the contract line "
                                                 "(tiny,mixtral,hotcold,nvfp4,large,graded)")
     ap.add_argument("--batch", type=int, default=0, help="with --suite: only this batch size")
+    ap.add_argument("--act", choices=["fp8", "nvfp4"], default="fp8",
+                    help="with --suite: activation format of NVFP4 layers")
     args = ap.parse_args()
     if args.suite:
         run_suite(args)
