@@ -9,25 +9,26 @@
 //   * persistent clusters of two CTAs (one CTA per SM) walk (token chunk, weight
 //     tiles) work items; chunk = up to 256 consecutive expert-sorted rows of one
 //     expert; each CTA owns 128-row weight tiles (gate + up, or two down tiles);
-//   * two rings of shared-memory slots per CTA: raw slots hold a stage's packed
+//   * three rings of shared-memory slots per CTA: raw slots hold a stage's packed
 //     codes + scales (64 inputs = two quantization groups) and are freed as soon
-//     as they are dequantized, so their copies run many stages ahead; operand
-//     slots hold the activation tile and the dequantized weight tiles the tensor
-//     core reads, and are freed by the MMA commit;
+//     as they are dequantized, so their copies run many stages ahead; A slots
+//     hold the dequantized weight tiles and B slots this CTA's half of the
+//     activation tile, both freed by the MMA commit;
 //   * warp 16 (one lane) streams the codes and scales of this CTA's weight tiles
-//     into the raw ring with 1D bulk copies; warp 18 (one lane) loads this CTA's
-//     half of the chunk's token rows into the operand ring with a 2D TMA load
-//     (128-byte swizzle); no copy is multicast;
+//     into the raw ring with 1D bulk copies; warp 18 (one lane) loads the
+//     activation half-tile into the B ring with a 2D TMA load (128-byte swizzle;
+//     a half-height box for chunks of at most 128 rows); no copy is multicast;
 //   * warps 0-15 turn codes into fp16 operands (exponent-bias unpack: a code u
-//     OR'ed into the mantissa of 1024.0 gives 1024+u exactly; one subtract
-//     and one multiply by the group scale), release the raw slot, and write
-//     the operands straight into the swizzled K-major layout the tensor core
-//     reads, then arrive on the even CTA's barrier;
-//   * warp 17 of the even CTA (one lane) issues tcgen05.mma.cta_group::2
-//     M=256 (128 weight rows from each CTA) x N<=256 (token rows, half from
-//     each CTA) x K=16 and commits to both CTAs' mbarriers;
+//     OR'ed into the mantissa of 1024.0 gives 1024+u exactly; one FMA removes
+//     the bias and the code offset, one multiply applies the group scale),
+//     release the raw slot, and write the operands straight into the swizzled
+//     K-major layout the tensor core reads, then arrive on the even CTA's barrier;
+//   * warp 17 of the even CTA issues tcgen05.mma.cta_group::2 M=256 (128 weight
+//     rows from each CTA) x N<=256 (token rows, half from each CTA) x K=16,
+//     warp-wide with one elected lane, and commits to both CTAs' mbarriers;
+//     warp 17 of the odd CTA reports its activation tiles to the even CTA;
 //   * warps 0-15 then drain their own TMEM (tcgen05.ld) into the SwiGLU / scale
-//     epilogue.
+//     epilogue (plus the outlier side lists' residual dot in OUT instantiations).
 // Shapes whose weight tiles do not pair run the same kernel on single CTAs
 // (cta_group::1, M=128, the whole token chunk per CTA).
 // Every mbarrier wait is bounded; a wait that gives up raises the abort flags
