@@ -1,12 +1,15 @@
 /*
  * moe.h -- C ABI of the B200 (sm_100a) quantized Mixture-of-Experts FFN layer.
  *
- * Two calls:
- *   moe_pack           quantizes fp32 expert weights into the packed layer buffer;
+ * Three calls:
+ *   moe_pack           quantizes fp32 expert weights into the packed layer buffer
+ *                      (optionally keeping each matrix's largest weights in an
+ *                      fp16 side list);
  *   moe_layer_forward  runs the layer: fp32 router -> top-k with a softmax over
  *                      the chosen k -> permutation of tokens by expert ->
  *                      per-expert SwiGLU FFN on dequantized weights -> weighted
- *                      combine.
+ *                      combine;
+ *   moe_layer_forward_noalloc  the same with a workspace inside the library.
  *
  * Where the method comes from (web pages; section numbers as printed there):
  *  - "quantized MoE LLM inference" (cloud.baidu.com article 9434801), expert
@@ -22,7 +25,13 @@
  *    bit widths chosen per expert and per projection (gate 3-bit, middle 2-bit,
  *    output 4-bit), group size 32.
  *  - "Expert-aware quantisation: near-Q4 quality at near-Q2 size?": frequently
- *    routed ("hot") experts at 4-bit, the rest ("cold") at 2-bit.
+ *    routed ("hot") experts at 4-bit, the rest ("cold") at 2-bit, and below
+ *    2 bits for the coldest (the 1-bit sign code here).
+ *  - The same mixed-precision page, sec. 4.2, tip 2: each expert's top 0.05% of
+ *    weights by |w| kept in fp16 beside the quantized rest (MOE_FMT_OUTLIERS).
+ *  - The NVFP4 remarks of the MoE inference page: e2m1 weights with e4m3 block
+ *    scales; with MOE_ACT_NVFP4 the activations take the same format and prefill
+ *    runs the tensor core's block-scaled FP4 MMA.
  *
  * Conventions for every call:
  *  - Pointers are DEVICE pointers unless marked HOST.  The caller owns all
