@@ -208,3 +208,31 @@ def test_outlier_flag_layout_and_errors():
         rc = _lib.load().moe_layer_forward(FAKE, 16, FAKE, None, C.byref(w), 2, FAKE, None, 0, C.byref(need),
                                            None, None)
         assert _lib.STATUS[rc] == want
+
+
+def test_outlier_layout_random_shapes():
+    # the outlier section's size for seeded random shapes and flag patterns, against the
+    # layout rule restated here (section after the expert sections, 256-byte aligned;
+    # 768-entry u64 table + 4*(64+65536) bytes of scratch; per flagged matrix, in
+    # (expert, projection) order, 4*(N+1+floor(N*K*5/10000)) bytes, 256-byte aligned)
+    rng = np.random.default_rng(11)
+    up = lambda v: (v + 255) // 256 * 256  # noqa: E731
+    for _ in range(25):
+        E = int(rng.integers(1, 33))
+        H, F = 128 * int(rng.integers(1, 17)), 128 * int(rng.integers(1, 17))
+        base = rng.choice([1, 2, 3, 4], size=(E, 3)).astype(np.uint8) if rng.random() < 0.7 \
+            else np.full((E, 3), 16, np.uint8)
+        flags = (rng.random((E, 3)) < 0.4).astype(np.uint8) * moe.FMT_OUTLIERS
+        fmt = (base | flags).astype(np.uint8)
+        t_base = moe.pack_layout(E, H, F, base)[0]
+        t_out = moe.pack_layout(E, H, F, fmt)[0]
+        if not flags.any():
+            assert t_out == t_base
+            continue
+        pos = up(up(t_base) + 8 * 768 + 4 * (64 + 65536))
+        for e in range(E):
+            for p in range(3):
+                if flags[e, p]:
+                    N, K = (F, H) if p < 2 else (H, F)
+                    pos = up(pos + 4 * (N + 1 + N * K * 5 // 10000))
+        assert t_out == pos, (E, H, F)

@@ -26,3 +26,17 @@ def test_traffic_summary_matches_or_is_null():
         assert t == d["kernels"]["gateup_prefill_large"]["dram_bytes_per_launch"]
     else:
         assert t is None
+
+
+def test_peaks_prefer_the_measured_file(tmp_path, monkeypatch):
+    # the measured peaks file, when present, supplies both GEMM figures; without it the
+    # stated fallback applies and no sustained figure is claimed
+    import json
+    f = tmp_path / "peaks.json"
+    f.write_text(json.dumps({"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1300.0}))
+    monkeypatch.setattr(bench, "PEAKS_FILE", str(f))
+    pk, kind = bench.peaks()
+    assert kind == "measured" and pk["bf16_tflops_sustained"] == 1300.0 and pk["hbm_gbs"] == 6000.0
+    monkeypatch.setattr(bench, "PEAKS_FILE", str(tmp_path / "absent.json"))
+    pk, kind = bench.peaks()
+    assert kind == "fallback" and pk == bench.FALLBACK_PEAKS and "bf16_tflops_sustained" not in pk
